@@ -1,0 +1,410 @@
+"""Benchmark of the paged decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 7b|gqa70b|prefix_cow|long|tiny]
+
+One step = the whole hot path over one batch: copy-on-write block copies (if
+the workload has any), the slot write of the step's new tokens, and decode
+attention, on the 7B-shaped decode layer by default (64 sequences, 32 query
+= 32 KV heads, head size 128, bf16, 20000-block shuffled pool, lengths
+min(4096, 100 + floor(Exp(400)))).
+
+Metric: effective KV HBM bandwidth in GB/s = algorithmic bytes of the step
+(K and V of every live token, q read, out written, plus the slot write's and
+copies' bytes) / device time; also seq-steps/s and % of the measured HBM
+peak.  The L2 is flushed (a 512 MiB write, untimed) before every timed step.
+
+Under torchrun (N > 1) every rank runs its own independent batch (the path
+shards by sequence with no collective): weak scaling, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: effective KV HBM GB/s (% of B200 peak); seq-steps/s"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
+KERNEL_SOURCES = ("paged_kv_cache_456_b200/csrc/decode_kernel.cuh",
+                  "paged_kv_cache_456_b200/csrc/decode_bf16.cu",
+                  "paged_kv_cache_456_b200/csrc/decode_f32.cu",
+                  "paged_kv_cache_456_b200/csrc/ptx.cuh",
+                  "paged_kv_cache_456_b200/csrc/pa_internal.h")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description="paged decode benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="7b")
+    ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=None)
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = d.get(workload)
+    if not entry or entry.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def step_bytes(w) -> int:
+    return w.decode_bytes() + w.reshape_bytes() + w.copy_bytes()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report no clocks rather than fail
+            self.max_mhz = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self._t.join(timeout=2)
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle as baseline / reference arm
+# ---------------------------------------------------------------------------
+def sub_workload(w, k: int):
+    """The first k sequences of a workload (same pool, same copy pairs)."""
+    import dataclasses
+    return dataclasses.replace(
+        w, context_lens=w.context_lens[:k], tables_compact=w.tables_compact[:k], q=w.q[:k],
+        new_key=None if w.new_key is None else w.new_key[:k],
+        new_value=None if w.new_value is None else w.new_value[:k],
+        slot_mapping_compact=None if w.slot_mapping_compact is None else w.slot_mapping_compact[:k])
+
+
+def oracle_sample(w, budget_s: float, repeat: bool = False):
+    """Time the oracle's whole step on the first k sequences of the workload,
+    k grown until one pass takes about budget_s (or all sequences are in);
+    with ``repeat``, whole passes are then repeated until budget_s is spent.
+    Returns (GB/s, seconds per pass, k, bytes per pass, threads)."""
+    import oracle
+
+    k = 1
+    while True:
+        ws = sub_workload(w, k)
+        t0 = time.perf_counter()
+        oracle.workload_step(ws)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or k >= w.num_seqs:
+            break
+        k = min(w.num_seqs, max(k + 1, int(k * min(8.0, budget_s / max(dt, 1e-3)))))
+    if repeat and dt < budget_s:
+        passes, t0 = 0, time.perf_counter()
+        while passes == 0 or time.perf_counter() - t0 < budget_s:
+            oracle.workload_step(ws)
+            passes += 1
+        dt = (time.perf_counter() - t0) / passes
+    nbytes = step_bytes(ws)
+    return nbytes / dt / 1e9, dt, k, nbytes, oracle.num_threads()
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    from paged_kv_cache_456_b200.workloads import build_workload
+    import oracle
+    w = build_workload(args.workload, seed=args.seed)
+    steps, warm = args.steps, args.warmup
+    per_step_budget = max(0.05, 150.0 / max(1, steps + warm))
+    _, dt, k, nbytes, threads = oracle_sample(w, per_step_budget)
+    ws = sub_workload(w, k)
+    for _ in range(warm):
+        oracle.workload_step(ws)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.workload_step(ws)
+    elapsed = time.perf_counter() - t0
+    value = nbytes * steps / elapsed / 1e9
+    sample = (f"first {k} of {w.num_seqs} sequences of the {w.name} workload per step "
+              f"({int(w.context_lens[:k].sum())} tokens)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": warm,
+        "ms_per_step": round(elapsed / steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "seq_steps_per_s": round(k * steps / elapsed, 3),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "num_blocks": w.num_blocks, "kv_dtype": w.dtype,
+            "context_tokens": int(w.context_lens.sum()),
+            "max_context_len": int(w.max_context_len),
+            "partition_size": int(w.partition_size),
+            "l2": "flushed before every timed step (512 MiB write, untimed)"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_456_b200 import ops
+    from paged_kv_cache_456_b200.workloads import build_workload, upload
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    # rank 0 runs the named workload's own seed; other ranks get independent batches
+    seed = args.seed if rank == 0 else (args.seed or 0) + 1000 * rank
+    w = build_workload(args.workload, seed=seed)
+    if args.partition_size is not None:
+        w.partition_size = args.partition_size
+    t = upload(w, dev)
+    stream = torch.cuda.current_stream(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    tdt = t["q"].dtype
+    ps = w.partition_size
+    ws = ops.make_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.max_context_len, ps, tdt, device=dev)
+    cfg = ops.launch_config(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.max_context_len, ps, tdt)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    launches_per_step = 1 + ("key" in t) + ("block_mapping" in t)
+
+    def step(ev_mid=None):
+        if "block_mapping" in t:
+            ops.copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err_flag=err)
+        if "key" in t:
+            ops.reshape_and_cache(t["key"], t["value"], t["k_cache"], t["v_cache"],
+                                  t["slot_mapping"], err_flag=err)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        ops.decode(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                   t["context_lens"], scale=w.scale, max_context_len=w.max_context_len,
+                   workspace=ws, partition_size=ps, err_flag=err)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        for i in range(K):
+            flush.fill_(1)                  # evict the previous step from L2 (untimed)
+            ev[i][0].record(stream)
+            step(ev[i][1])
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms = [a.elapsed_time(c) for a, b, c in ev]
+    dec_ms = [b.elapsed_time(c) for a, b, c in ev]
+    total_ms = sum(step_ms)
+    if err.item() != 0:
+        raise RuntimeError(f"device error flag {err.item()} during the benchmark")
+
+    # end to end through the public API: pinned host inputs in, output back
+    e2e = end_to_end(w, t, ws, ps, dev, stream, K, args.warmup)
+
+    total_t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(total_t, op=dist.ReduceOp.MAX)
+        e2e_t = torch.tensor([e2e["ms"]], dtype=torch.float64, device=dev)
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        e2e["ms"] = float(e2e_t.item())
+    max_ms = float(total_t.item())
+
+    nbytes = step_bytes(w)
+    peak, peak_kind = measured_peaks()
+    value = world * nbytes * K / (max_ms * 1e-3) / 1e9
+    dec_avg = statistics.mean(dec_ms)
+    achieved = w.decode_bytes() / (dec_avg * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(max_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if
+        w.dtype == "bf16" else "f32", "data": "synthetic", "config": workload_config(w),
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "seq_steps_per_s": round(world * w.num_seqs * K / (max_ms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "kernel": "paged_decode_kernel",
+                     "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
+                     "algorithmic_bytes_per_launch": w.decode_bytes(),
+                     "launch_ms_mean": round(dec_avg, 5),
+                     "launch_ms_median": round(statistics.median(dec_ms), 5)},
+        "e2e": {"value": round(world * nbytes * K / (e2e["ms"] * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": round(e2e["ms"] / K, 5)},
+        "gpu_launches": launches_per_step * K,
+        "launch": cfg,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, dt, k, nb, threads = oracle_sample(w, budget_s=10.0, repeat=True)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
+                                "kind": "oracle",
+                                "sample": f"first {k} of {w.num_seqs} sequences of the {w.name} "
+                                          f"step ({dt:.1f} s per pass)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def end_to_end(w, t, ws, ps, dev, stream, K, warmup):
+    """The step through the public API with the step's inputs in pinned host
+    memory: H2D copies of q, the new K/V, slot ids, block tables and lengths,
+    the kernels, and the D2H copy of the output, all inside the timed region.
+    The KV pool itself is resident device state and is not copied."""
+    import torch
+    from paged_kv_cache_456_b200 import ops
+
+    names = [n for n in ("q", "key", "value", "slot_mapping", "block_tables", "context_lens",
+                         "block_mapping") if n in t]
+    host = {n: t[n].cpu().pin_memory() for n in names}
+    out_h = torch.empty(t["out"].shape, dtype=t["out"].dtype).pin_memory()
+    dv = {n: torch.empty_like(t[n]) for n in names}
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def one():
+        for n in names:
+            dv[n].copy_(host[n], non_blocking=True)
+        if "block_mapping" in dv:
+            ops.copy_blocks(t["k_cache"], t["v_cache"], dv["block_mapping"], err_flag=err)
+        if "key" in dv:
+            ops.reshape_and_cache(dv["key"], dv["value"], t["k_cache"], t["v_cache"],
+                                  dv["slot_mapping"], err_flag=err)
+        ops.decode(t["out"], dv["q"], t["k_cache"], t["v_cache"], dv["block_tables"],
+                   dv["context_lens"], scale=w.scale, max_context_len=w.max_context_len,
+                   workspace=ws, partition_size=ps, err_flag=err)
+        out_h.copy_(t["out"], non_blocking=True)
+
+    for _ in range(max(3, warmup)):
+        one()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    if err.item():
+        raise RuntimeError(f"device error flag {err.item()} in the end-to-end loop")
+    return {"ms": a.elapsed_time(b), "h2d": h2d, "d2h": d2h}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/*
+ * paged_attention.h -- C ABI of libpa.so: PagedAttention decode for NVIDIA
+ * B200 (sm_100a), with the two cache-maintenance operations that feed it.
+ *
+ * The key/value cache of every sequence is cut into fixed-size blocks of
+ * block_size token slots (16, "typically 16 tokens per block"), and a
+ * per-sequence block table maps the sequence's logical block j to a physical
+ * block id in one shared pool (skandtandon.pages.dev day-9 post, section
+ * "Idea 1: PagedAttention"; "What vLLM Is and Why It Exists", section "The
+ * idea vLLM started from: pages").  The decode kernel reads a sequence's
+ * cached keys and values "from blocks scattered anywhere in the tensor,
+ * following the block table" (same section), so its result is ordinary
+ * attention over the sequence's tokens.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument except the function's own scalars is a DEVICE
+ *    pointer, owned by the caller; the library allocates nothing, keeps no
+ *    state between calls, and frees nothing.
+ *  - Element type (pa_dtype) is the same for q, out, key, value and both
+ *    caches: IEEE fp32 or bf16.  Arithmetic is fp32 in every case.
+ *  - Cache layout, for K and for V alike:
+ *        cache[num_blocks][num_kv_heads][block_size][head_dim]   (contiguous)
+ *    so one (block, kv head) tile of block_size * head_dim elements is
+ *    contiguous in memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  A returned PA_OK means "validated and launched".
+ *  - Host-checkable problems return a non-OK status BEFORE anything is
+ *    launched, and leave every buffer untouched.  These checks need no GPU.
+ *  - Problems only the device can see (an index read from device memory that
+ *    is out of range) never fault, trap or hang: the offending item is
+ *    skipped and a bit is OR-ed into *err_flag (a device int32 the caller
+ *    zeroes; may be NULL).  The bits are PA_ERRBIT_*.
+ *  - Every device-side wait is bounded (about one second); a wait that runs
+ *    out sets PA_ERRBIT_TIMEOUT and the kernel returns.
+ */
+#ifndef PAGED_ATTENTION_H
+#define PAGED_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,  /* a null pointer, a negative size, a misaligned buffer ... */
+    PA_ERR_UNSUPPORTED = 2,  /* a valid shape this build has no kernel for              */
+    PA_ERR_WORKSPACE = 3,    /* the decode workspace is missing or too small            */
+    PA_ERR_CUDA = 4          /* the CUDA runtime refused a query or a launch            */
+} pa_status;
+
+typedef enum pa_dtype {
+    PA_F32 = 0,
+    PA_BF16 = 1
+} pa_dtype;
+
+/* bits OR-ed into *err_flag by the device */
+#define PA_ERRBIT_BLOCK_ID    1   /* a live block-table entry outside [0, num_blocks): that
+                                     sequence's output rows are written as zeros            */
+#define PA_ERRBIT_CONTEXT_LEN 2   /* context_lens[s] outside [0, min(max_context_len,
+                                     max_blocks_per_seq * block_size)]: rows written as 0   */
+#define PA_ERRBIT_SLOT        4   /* slot_mapping[t] >= num_blocks * block_size: skipped    */
+#define PA_ERRBIT_PAIR        8   /* a copy pair with an id outside [0, num_blocks) or
+                                     src == dst: skipped                                  */
+#define PA_ERRBIT_TIMEOUT     16  /* a bounded device wait ran out; results are invalid and
+                                     the decode workspace must be re-initialised           */
+
+/* Human-readable name of a status code (static storage). */
+const char *pa_status_str(pa_status status);
+
+/* ------------------------------------------------------------------------
+ * Decode attention
+ * ------------------------------------------------------------------------
+ * For each sequence s (one new query token per head) and query head h:
+ *
+ *     n      = context_lens[s]                      (tokens in the cache)
+ *     token i (0 <= i < n) lives in physical block block_tables[s][i / 16],
+ *            slot i % 16, of KV head g = h / (num_q_heads / num_kv_heads)
+ *     x_i    = scale * dot(q[s][h][:], K_i[g][:])
+ *     out[s][h][:] = sum_i exp(x_i - max x) V_i[g][:] / sum_i exp(x_i - max x)
+ *
+ * Only tokens 0..n-1 are read; unused slots of a partial last block and
+ * table entries past ceil(n/16) may hold anything (NaN, -1).  n == 0 gives a
+ * zero row.  out is rounded once (nearest-even) to the element type.
+ *
+ * Arguments:
+ *   out            [num_seqs][num_q_heads][head_dim]            written
+ *   q              [num_seqs][num_q_heads][head_dim]            read
+ *   k_cache,
+ *   v_cache        [num_blocks][num_kv_heads][16][head_dim]     read
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq]         read
+ *   context_lens   int32 [num_seqs]                             read
+ *   max_context_len  host-side upper bound of context_lens (sizes the launch
+ *                  and the workspace without a device-to-host copy)
+ *   scale          logit scale, usually 1/sqrt(head_dim)
+ *   partition_size the most tokens one partial result may cover before the
+ *                  log-sum-exp merge (a multiple of 16); 0 lets the library
+ *                  cut each sequence only where it balances the work across
+ *                  the GPU.  Every split is merged exactly (up to rounding):
+ *                  M = max m_j, out = sum_j e^(m_j-M) o_j / sum_j e^(m_j-M) l_j.
+ *   workspace      device scratch of at least pa_decode_workspace_size()
+ *                  bytes, zero-filled once before its first use (for
+ *                  instance with pa_decode_workspace_init); every call leaves
+ *                  it zero-filled again where it must be.  Two calls that
+ *                  may run at the same time must not share a workspace.
+ *
+ * Supported: block_size == 16; head_dim 64 or 128; num_q_heads /
+ * num_kv_heads in {1, 2, 4, 8}; q, out, k_cache, v_cache 16-byte aligned.
+ * Shapes outside that return PA_ERR_UNSUPPORTED.
+ */
+pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int max_context_len, int partition_size,
+                                   pa_dtype dtype, size_t *bytes);
+
+/* cudaMemsetAsync(workspace, 0, bytes, stream): makes a fresh workspace usable. */
+pa_status pa_decode_workspace_init(void *workspace, size_t bytes, void *stream);
+
+/* The launch pa_decode would make for these arguments on the current device:
+ * CTAs in the grid, warps per CTA, pipeline depth (tiles in flight per warp)
+ * and dynamic shared memory per CTA.  Any output pointer may be NULL. */
+pa_status pa_decode_launch_config(int num_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int max_context_len, int partition_size,
+                                  pa_dtype dtype, int *grid, int *warps_per_cta,
+                                  int *pipeline_depth, int *smem_bytes);
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens,
+                    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int block_size, int max_blocks_per_seq, int num_blocks,
+                    int max_context_len, float scale, int partition_size, pa_dtype dtype,
+                    void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Slot write (reshape_and_cache)
+ * ------------------------------------------------------------------------
+ * Writes each step's new key/value rows into the cache: the cache "grows ...
+ * as the model generates new tokens" ("vLLM Solved the Wrong Bottleneck...",
+ * section "Paged Attention"), one new token per request per step ("What vLLM
+ * Is and Why It Exists", section "A picture").  For every token t and KV
+ * head h:
+ *     slot = slot_mapping[t];  if slot < 0: skip (padding)
+ *     k_cache[slot / block_size][h][slot % block_size][:] = key[t][h][:]
+ *     v_cache[...same...]                                 = value[t][h][:]
+ * A bit-exact copy.  key, value: [num_tokens][num_kv_heads][head_dim];
+ * slot_mapping: int64 [num_tokens].  Slots must be distinct within a call.
+ * head_dim * element size must be a multiple of 16 bytes; buffers 16-byte
+ * aligned; any block_size >= 1.
+ */
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache,
+                               void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               pa_dtype dtype, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Block copy-on-write (copy_blocks)
+ * ------------------------------------------------------------------------
+ * "When a shared block needs to diverge, only the changed block is copied"
+ * (day-9 post, section "Idea 1: PagedAttention").  For each pair p of
+ * block_mapping (int32 [num_pairs][2] = {src, dst}), the whole physical
+ * block src -- all KV heads, all block_size slots -- is copied to dst, in
+ * k_cache and in v_cache.  A bit-exact copy.  The dst ids must be distinct
+ * and disjoint from the src ids (otherwise the result is undefined).
+ */
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_mapping,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, int32_t *err_flag, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_ATTENTION_H */

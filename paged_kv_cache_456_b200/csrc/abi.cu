@@ -1,0 +1,313 @@
+// abi.cu -- the extern "C" entry points of libpa.so (include/paged_attention.h):
+// argument validation on the host, launch planning, launches.  No entry point
+// allocates memory or synchronises; everything after validation is
+// asynchronous on the caller's stream.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include <cuda_runtime.h>
+
+#include "paged_attention.h"
+#include "pa_internal.h"
+
+namespace pa {
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                     void* v_cache, const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int row_bytes, int block_size,
+                                     long long num_slots, int32_t* err_flag, int num_sms,
+                                     cudaStream_t stream);
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping,
+                               int num_pairs, long long block_bytes, int num_blocks,
+                               int32_t* err_flag, int num_sms, cudaStream_t stream);
+}  // namespace pa
+
+static_assert(pa::kErrBlockId == PA_ERRBIT_BLOCK_ID, "error bit mismatch");
+static_assert(pa::kErrContextLen == PA_ERRBIT_CONTEXT_LEN, "error bit mismatch");
+static_assert(pa::kErrSlot == PA_ERRBIT_SLOT, "error bit mismatch");
+static_assert(pa::kErrPair == PA_ERRBIT_PAIR, "error bit mismatch");
+static_assert(pa::kErrTimeout == PA_ERRBIT_TIMEOUT, "error bit mismatch");
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+// (device, kernel, dynamic smem) -> resident CTAs per SM; the kernel's smem
+// attributes are set when an entry is first made.
+std::map<std::tuple<int, const void*, size_t>, int> g_occupancy;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(pa_dtype dt) { return dt == PA_BF16 ? 2 : 4; }
+
+bool valid_dtype(pa_dtype dt) { return dt == PA_F32 || dt == PA_BF16; }
+
+pa_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return PA_ERR_CUDA;
+    d.ready = true;
+  }
+  *out = d;
+  return PA_OK;
+}
+
+struct DecodePlan {
+  pa::DecodeKernelInfo kernel{};
+  int grid = 0;
+  size_t smem = 0;
+  long long ranges = 0;      // most ranges the device can form
+  size_t counters_off = 0;   // workspace layout
+  size_t o_off = 0;
+  size_t ml_off = 0;
+  size_t ws_bytes = 0;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+pa_status occupancy(const pa::DecodeKernelInfo& k, size_t smem, int* occ) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const auto key = std::make_tuple(dev, k.fn, smem);
+  auto it = g_occupancy.find(key);
+  if (it != g_occupancy.end()) {
+    *occ = it->second;
+    return PA_OK;
+  }
+  if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return PA_ERR_CUDA;
+  cudaFuncSetAttribute(k.fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       cudaSharedmemCarveoutMaxShared);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, k.fn, k.warps * 32, smem) != cudaSuccess)
+    return PA_ERR_CUDA;
+  g_occupancy[key] = *occ;
+  return PA_OK;
+}
+
+// Shape checks shared by the decode entry points (no device needed).
+pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                             int max_context_len, int partition_size, pa_dtype dtype) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      max_context_len < 0 || partition_size < 0 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (partition_size % pa::kBlockSize != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_q_heads / num_kv_heads;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_UNSUPPORTED;
+  if (num_kv_heads > 0xffff) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int max_context_len, int partition_size, pa_dtype dtype, DecodePlan* p) {
+  pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                    max_context_len, partition_size, dtype);
+  if (st != PA_OK) return st;
+  const int group = num_q_heads / num_kv_heads;
+  const bool found = dtype == PA_BF16 ? pa::decode_kernel_bf16(head_dim, group, &p->kernel)
+                                      : pa::decode_kernel_f32(head_dim, group, &p->kernel);
+  if (!found) return PA_ERR_UNSUPPORTED;
+  // tiles: must fit the kernel's 32-bit tile counter
+  const long long blocks_max = (static_cast<long long>(max_context_len) + pa::kBlockSize - 1) /
+                               pa::kBlockSize;
+  const long long tiles_max = static_cast<long long>(num_seqs) * num_kv_heads * blocks_max;
+  if (tiles_max >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
+
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != PA_OK) return st;
+  const size_t seq_bytes = round_up((2 * static_cast<size_t>(num_seqs) + 1) * sizeof(int), 16);
+  p->smem = static_cast<size_t>(p->kernel.warps) * p->kernel.warp_bytes + seq_bytes;
+  if (p->smem > static_cast<size_t>(dev.smem_optin)) return PA_ERR_UNSUPPORTED;
+  int occ = 0;
+  if ((st = occupancy(p->kernel, p->smem, &occ)) != PA_OK) return st;
+  if (occ < 1) return PA_ERR_UNSUPPORTED;
+  const long long resident = static_cast<long long>(dev.sms) * occ;
+  const long long by_work = (tiles_max + p->kernel.warps - 1) / p->kernel.warps;
+  p->grid = static_cast<int>(by_work < resident ? (by_work > 0 ? by_work : 1) : resident);
+  const long long workers = static_cast<long long>(p->grid) * p->kernel.warps;
+  long long ranges = workers;
+  if (partition_size > 0) {
+    const long long per = workers * (partition_size / pa::kBlockSize);
+    const long long rounds = (tiles_max + per - 1) / per;
+    ranges = workers * (rounds > 1 ? rounds : 1);
+  }
+  if (ranges > tiles_max) ranges = tiles_max > 0 ? tiles_max : 1;
+  p->ranges = ranges;
+  const size_t slots = 2 * static_cast<size_t>(ranges);
+  p->counters_off = 0;
+  p->o_off = round_up(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int), 256);
+  p->ml_off = round_up(p->o_off + slots * group * head_dim * sizeof(float), 256);
+  p->ws_bytes = round_up(p->ml_off + slots * group * 2 * sizeof(float), 256);
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_str(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+  }
+  return "PA_ERR_UNKNOWN";
+}
+
+pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int max_context_len, int partition_size, pa_dtype dtype,
+                                   size_t* bytes) {
+  if (!bytes) return PA_ERR_INVALID_ARG;
+  DecodePlan p;
+  const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                 partition_size, dtype, &p);
+  if (st != PA_OK) return st;
+  *bytes = p.ws_bytes;
+  return PA_OK;
+}
+
+pa_status pa_decode_workspace_init(void* workspace, size_t bytes, void* stream) {
+  if (!workspace && bytes) return PA_ERR_INVALID_ARG;
+  if (!bytes) return PA_OK;
+  return cudaMemsetAsync(workspace, 0, bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_launch_config(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int max_context_len, int partition_size, pa_dtype dtype,
+                                  int* grid, int* warps_per_cta, int* pipeline_depth,
+                                  int* smem_bytes) {
+  DecodePlan p;
+  const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                 partition_size, dtype, &p);
+  if (st != PA_OK) return st;
+  if (grid) *grid = p.grid;
+  if (warps_per_cta) *warps_per_cta = p.kernel.warps;
+  if (pipeline_depth) *pipeline_depth = p.kernel.depth;
+  if (smem_bytes) *smem_bytes = static_cast<int>(p.smem);
+  return PA_OK;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                    int partition_size, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    int32_t* err_flag, void* stream) {
+  pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                    max_context_len, partition_size, dtype);
+  if (st != PA_OK) return st;
+  if (max_blocks_per_seq <= 0 || num_blocks <= 0 || block_size <= 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_seqs) * num_kv_heads * max_blocks_per_seq >= (1LL << 31))
+    return PA_ERR_UNSUPPORTED;
+  DecodePlan p;
+  if ((st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                      partition_size, dtype, &p)) != PA_OK)
+    return st;
+  if (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace))
+    return PA_ERR_WORKSPACE;
+
+  pa::DecodeArgs args;
+  args.out = out;
+  args.q = q;
+  args.k_cache = k_cache;
+  args.v_cache = v_cache;
+  args.block_tables = block_tables;
+  args.context_lens = context_lens;
+  args.num_seqs = num_seqs;
+  args.num_q_heads = num_q_heads;
+  args.num_kv_heads = num_kv_heads;
+  args.max_blocks_per_seq = max_blocks_per_seq;
+  args.num_blocks = num_blocks;
+  const long long cap = static_cast<long long>(max_blocks_per_seq) * pa::kBlockSize;
+  args.len_cap = static_cast<int>(max_context_len < cap ? max_context_len : cap);
+  args.part_blocks = partition_size / pa::kBlockSize;
+  args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  char* ws = static_cast<char*>(workspace);
+  args.counters = reinterpret_cast<int*>(ws + p.counters_off);
+  args.ws_o = reinterpret_cast<float*>(ws + p.o_off);
+  args.ws_ml = reinterpret_cast<float2*>(ws + p.ml_off);
+  args.err_flag = err_flag;
+
+  void* params[] = {&args};
+  const cudaError_t e =
+      cudaLaunchKernel(p.kernel.fn, dim3(p.grid), dim3(p.kernel.warps * 32), params, p.smem,
+                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               int32_t* err_flag, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  const long long row = static_cast<long long>(head_dim) * elem_bytes(dtype);
+  if (row % 16 != 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const pa_status st = device_info(&dev);
+  if (st != PA_OK) return st;
+  const cudaError_t e = pa::launch_reshape_and_cache(
+      key, value, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
+      static_cast<int>(row), block_size, static_cast<long long>(num_blocks) * block_size,
+      err_flag, dev.sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, int32_t* err_flag, void* stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0 || !valid_dtype(dtype))
+    return PA_ERR_INVALID_ARG;
+  const long long blk =
+      static_cast<long long>(num_kv_heads) * block_size * head_dim * elem_bytes(dtype);
+  if (blk % 16 != 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const pa_status st = device_info(&dev);
+  if (st != PA_OK) return st;
+  const cudaError_t e = pa::launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, blk,
+                                               num_blocks, err_flag, dev.sms,
+                                               static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"

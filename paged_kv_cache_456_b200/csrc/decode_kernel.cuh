@@ -1,0 +1,578 @@
+// decode_kernel.cuh -- PagedAttention decode for sm_100a.
+//
+// What it computes: for every sequence s and query head h, softmax attention
+// of q[s][h] over the context_lens[s] cached tokens, each token found through
+// the sequence's block table ("What vLLM Is and Why It Exists", section "The
+// idea vLLM started from: pages": attention reads a request's cache "from
+// blocks scattered anywhere in the tensor, following the block table").
+//
+// How (B200 design):
+//  * Work unit = one (sequence, KV head, block) tile: 16 tokens x head_dim,
+//    contiguous in the cache, read once for all G = Hq/Hkv query heads that
+//    share the KV head.  All units are laid end to end in (seq, kv head,
+//    block) order and cut into equal contiguous ranges, one or more per warp
+//    of a persistent grid (as many CTAs as fit on the 148 SMs): every warp
+//    gets the same number of tiles however skewed the context lengths are.
+//  * Each warp streams its tiles through a private ring of DEPTH shared-memory
+//    slots with the 1-D bulk-copy engine (cp.async.bulk, one mbarrier per
+//    slot, completion counted in bytes).  Only the live rows of a partial last
+//    block are fetched.  Block-table entries for the next 32-64 tiles are
+//    loaded one per lane well ahead of use.
+//  * Arithmetic is fp32 on the CUDA cores (a one-token query is a
+//    bandwidth-bound gather, not a dense contraction): lanes split head_dim
+//    16 bytes at a time, partial dot products are combined by a butterfly
+//    reduce-scatter of warp shuffles, the softmax is online (base 2, rescaled
+//    only when the running max grows by more than 2^8), and P.V accumulates
+//    in registers.
+//  * A sequence cut by a range boundary leaves partial results (m, l, o) in
+//    the workspace; the warp that finishes the last piece of a (seq, kv head)
+//    merges them by log-sum-exp and writes the output (a counter per (seq,
+//    kv head), no waiting, so nothing can hang).
+//  * Device-side index checks skip bad items and set err_flag bits; every
+//    wait is bounded.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "pa_internal.h"
+#include "ptx.cuh"
+
+namespace pa {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// -- element conversion ---------------------------------------------------------
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+  __device__ __forceinline__ static void unpack(const uint4& r, float* f) {
+    f[0] = __uint_as_float(r.x);
+    f[1] = __uint_as_float(r.y);
+    f[2] = __uint_as_float(r.z);
+    f[3] = __uint_as_float(r.w);
+  }
+  __device__ __forceinline__ static uint4 pack(const float* f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+  // bf16 -> fp32 is exact: the bf16 pattern is the high half of the fp32 one.
+  __device__ __forceinline__ static void unpack(const uint4& r, float* f) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ __forceinline__ static uint4 pack(const float* f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+// -- compile-time geometry --------------------------------------------------------
+template <typename T, int D, int G, int DEPTH, int WARPS>
+struct DecodeCfg {
+  static constexpr int EB = sizeof(T);
+  static constexpr int ROW = D * EB;          // bytes of one token's row of one KV head
+  static constexpr int VEC = 16 / EB;         // elements a lane holds per row
+  static constexpr int LPR = D / VEC;         // lanes per row
+  static constexpr int RPI = 32 / LPR;        // rows one warp instruction covers (row groups)
+  static constexpr int RL = kBlockSize / RPI; // rows per lane per block
+  static constexpr int TILE = kBlockSize * ROW;
+  static constexpr int QB = G * ROW;          // q rows of the G query heads
+  static constexpr int SLOT = 2 * TILE + QB;  // K tile, V tile, q
+  static constexpr int XS = kBlockSize * G * 4;
+  static constexpr int ALPHA = ((G * 4 + 15) / 16) * 16;
+  static constexpr int WARP_BYTES = ((DEPTH * SLOT + XS + ALPHA + DEPTH * 8 + 127) / 128) * 128;
+  // QK is done CH rows at a time; V = CH*G partial dots are reduce-scattered
+  // over the LPR lanes of a row, leaving NV finished logits per lane.
+  static constexpr int CH = cmin(RL, LPR / G >= 1 ? LPR / G : 1);
+  static constexpr int NCH = RL / CH;
+  static constexpr int V = CH * G;
+  static constexpr int LS = ilog2(LPR);
+  static constexpr int LSC = cmin(LS, ilog2(V));
+  static constexpr int NV = V >> LSC;
+  static constexpr int TPL = G >= 2 ? G / 2 : 1;  // softmax tokens per lane
+  static_assert(VEC * LPR == D, "head_dim must be a multiple of 16 bytes");
+  static_assert(RPI * LPR == 32 && RL * RPI == kBlockSize, "bad lane geometry");
+  static_assert(NCH * CH == RL, "bad chunking");
+  static_assert(32 % G == 0 && G <= 16, "group size");
+};
+
+// -- per-warp ranges of the global tile order ------------------------------------
+struct Ranges {
+  long long W;  // tiles in total
+  long long R;  // ranges (each non-empty: R <= W)
+  __device__ __forceinline__ long long start(long long r) const { return r * W / R; }
+  __device__ __forceinline__ long long of(long long x) const { return ((x + 1) * R - 1) / W; }
+  __device__ __forceinline__ bool is_start(long long x) const {
+    return x <= 0 || x >= W || start(of(x)) == x;
+  }
+};
+
+// One tile of a warp's stream, as 3 words (kept one per lane, 32 tiles per batch).
+struct StageDesc {
+  int phys;  // physical block id (0 if bad)
+  int seq;
+  int meta;  // kv head (bits 0-15) | live rows (16-20) | flags
+};
+constexpr int kFirst = 1 << 24;  // first tile of a piece: reset state, fetch q
+constexpr int kLast = 1 << 25;   // last tile of a piece: finish it
+constexpr int kBad = 1 << 26;    // block-table entry out of range
+
+__device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
+                                               const int* s_len, const Ranges& rg,
+                                               const DecodeArgs& a) {
+  StageDesc d{0, 0, 0};
+  if (g >= hi) return d;
+  // largest s with s_start[s] <= g (sequences without blocks share their start)
+  int lo = 0, up = a.num_seqs - 1;
+  while (lo < up) {
+    const int mid = (lo + up + 1) >> 1;
+    if (s_start[mid] <= g) lo = mid; else up = mid - 1;
+  }
+  const int s = lo;
+  const int n = s_len[s];
+  const int nb = (n + kBlockSize - 1) / kBlockSize;
+  const int off = static_cast<int>(g - s_start[s]);
+  const int kvh = off / nb;
+  const int blk = off - kvh * nb;
+  const long long item_a = s_start[s] + static_cast<long long>(kvh) * nb;
+  int flags = 0;
+  if (g == item_a || rg.is_start(g)) flags |= kFirst;
+  if (g + 1 == item_a + nb || rg.is_start(g + 1)) flags |= kLast;
+  int phys = __ldg(a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + blk);
+  if (phys < 0 || phys >= a.num_blocks) {
+    flags |= kBad;
+    phys = 0;
+    if (a.err_flag) atomicOr(a.err_flag, kErrBlockId);
+  }
+  const int rows = min(kBlockSize, n - blk * kBlockSize);
+  d.phys = phys;
+  d.seq = s;
+  d.meta = kvh | (rows << 16) | flags;
+  return d;
+}
+
+__device__ __forceinline__ StageDesc pick_desc(const StageDesc& A, const StageDesc& B, int rel) {
+  const bool in_a = rel < 32;
+  const int src = rel & 31;
+  StageDesc d;
+  d.phys = __shfl_sync(kFull, in_a ? A.phys : B.phys, src);
+  d.seq = __shfl_sync(kFull, in_a ? A.seq : B.seq, src);
+  d.meta = __shfl_sync(kFull, in_a ? A.meta : B.meta, src);
+  return d;
+}
+
+// Butterfly reduce-scatter of V values over the LPR lanes of a row group:
+// afterwards v[0..NV) of lane dl hold complete sums of value indices
+// (dl >> (LS - LSC)) * NV + r.
+template <int LPR, int V>
+__device__ __forceinline__ void reduce_scatter(float (&v)[V], int dl) {
+#pragma unroll
+  for (int st = 0; (1 << st) < LPR; ++st) {
+    const int o = LPR >> (st + 1);
+    const int len = V >> st;
+    if (len >= 2) {
+      const bool upper = (dl & o) != 0;
+#pragma unroll
+      for (int i = 0; i < len / 2; ++i) {
+        const float send = upper ? v[i] : v[len / 2 + i];
+        const float keep = upper ? v[len / 2 + i] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, o);
+      }
+    } else {
+      v[0] += __shfl_xor_sync(kFull, v[0], o);
+    }
+  }
+}
+
+template <typename T, int D, int G, int DEPTH, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32)
+paged_decode_kernel(const DecodeArgs a) {
+  using C = DecodeCfg<T, D, G, DEPTH, WARPS>;
+  using E = Elem<T>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_wsum[WARPS];
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int S = a.num_seqs;
+  const int Hkv = a.num_kv_heads;
+  const int Hq = a.num_q_heads;
+  int* s_start = reinterpret_cast<int*>(smem + WARPS * C::WARP_BYTES);  // [S + 1]
+  int* s_len = s_start + S + 1;                                         // [S]
+
+  // ---- prologue: block counts and their prefix sums, in tiles ----------------
+  {
+    const int per = (S + WARPS * 32 - 1) / (WARPS * 32);
+    const int s0 = min(S, tid * per);
+    const int s1 = min(S, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; ++s) {
+      int n = a.context_lens[s];
+      if (n < 0 || n > a.len_cap) n = 0;
+      s_len[s] = n;
+      local += (n + kBlockSize - 1) / kBlockSize;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+      const int v = s_wsum[w];
+      if (w < warp) before += v;
+      total += v;
+    }
+    int run = before + incl - local;
+    for (int s = s0; s < s1; ++s) {
+      s_start[s] = run * Hkv;
+      run += (s_len[s] + kBlockSize - 1) / kBlockSize;
+    }
+    if (tid == 0) s_start[S] = total * Hkv;
+    __syncthreads();
+  }
+
+  // ---- rows of empty or invalid sequences are zero --------------------------------
+  for (int s = blockIdx.x; s < S; s += gridDim.x) {
+    if (s_len[s] != 0) continue;
+    if (tid == 0 && a.err_flag) {
+      const int n = a.context_lens[s];
+      if (n < 0 || n > a.len_cap) atomicOr(a.err_flag, kErrContextLen);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(a.out) +
+                                          static_cast<size_t>(s) * Hq * C::ROW);
+    for (int i = tid; i < Hq * C::ROW / 16; i += WARPS * 32) dst[i] = make_uint4(0, 0, 0, 0);
+  }
+
+  // ---- this warp's share of the tiles -------------------------------------------
+  const long long W = s_start[S];
+  if (W == 0) return;
+  const long long NWK = static_cast<long long>(gridDim.x) * WARPS;
+  long long R = NWK;
+  if (a.part_blocks > 0) {
+    const long long per = NWK * a.part_blocks;
+    R = NWK * max(1LL, (W + per - 1) / per);
+  }
+  if (R > W) R = W;
+  const Ranges rg{W, R};
+  const long long gw = static_cast<long long>(blockIdx.x) * WARPS + warp;
+  const long long lo = rg.start(gw * R / NWK);
+  const long long hi = rg.start((gw + 1) * R / NWK);
+  if (lo >= hi) return;
+  const int nst = static_cast<int>(hi - lo);
+
+  unsigned char* wbase = smem + warp * C::WARP_BYTES;
+  const uint32_t slot0 = smem_addr(wbase);
+  float* xs = reinterpret_cast<float*>(wbase + DEPTH * C::SLOT);
+  float* alpha_s = reinterpret_cast<float*>(wbase + DEPTH * C::SLOT + C::XS);
+  const uint32_t bar0 = smem_addr(wbase + DEPTH * C::SLOT + C::XS + C::ALPHA);
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < DEPTH; ++j) mbar_init(bar0 + 8 * j, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  const int dl = lane % C::LPR;  // which 16 bytes of a row
+  const int rgp = lane / C::LPR; // which row group
+  const int hs = lane % G;       // softmax: head of this lane
+
+  StageDesc A = make_desc(lo + lane, hi, s_start, s_len, rg, a);
+  StageDesc B = make_desc(lo + 32 + lane, hi, s_start, s_len, rg, a);
+  int base = 0;
+
+  // Fill ring slot j % DEPTH with tile j: K and V rows, plus q on a piece start.
+  auto issue = [&](int j) {
+    const StageDesc e = pick_desc(A, B, j - base);
+    if (lane == 0) {
+      const int slot = j % DEPTH;
+      const uint32_t bar = bar0 + 8 * slot;
+      if (e.meta & kBad) {
+        mbar_arrive(bar);  // nothing to fetch; complete the phase
+      } else {
+        const int kvh = e.meta & 0xffff;
+        const int rows = (e.meta >> 16) & 31;
+        const bool with_q = (e.meta & kFirst) != 0;
+        const uint32_t kv_bytes = static_cast<uint32_t>(rows) * C::ROW;
+        const uint32_t dst = slot0 + slot * C::SLOT;
+        const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, 2 * kv_bytes + (with_q ? C::QB : 0));
+        bulk_copy_g2s(dst, static_cast<const char*>(a.k_cache) + off, kv_bytes, bar);
+        bulk_copy_g2s(dst + C::TILE, static_cast<const char*>(a.v_cache) + off, kv_bytes, bar);
+        if (with_q)
+          bulk_copy_g2s(dst + 2 * C::TILE,
+                        static_cast<const char*>(a.q) +
+                            (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * G) *
+                                C::ROW,
+                        C::QB, bar);
+      }
+    }
+  };
+
+  for (int j = 0; j < DEPTH && j < nst; ++j) issue(j);
+
+  float qv[G][C::VEC];
+  float o[G][C::VEC];
+  float m_run = -INFINITY, l_run = 0.f;
+  bool poisoned = false;
+
+  for (int k = 0; k < nst; ++k) {
+    const StageDesc d = pick_desc(A, B, k - base);
+    const int slot = k % DEPTH;
+    const bool ok = mbar_wait_bounded(bar0 + 8 * slot, (k / DEPTH) & 1);
+    if (!__all_sync(kFull, ok)) {
+      if (lane == 0 && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
+      // let copies already in flight land before the warp leaves
+      for (int j = k; j < nst && j < k + DEPTH; ++j)
+        mbar_wait_bounded(bar0 + 8 * (j % DEPTH), (j / DEPTH) & 1);
+      return;
+    }
+    const int flags = d.meta;
+    const int kvh = d.meta & 0xffff;
+    const int rows = (d.meta >> 16) & 31;
+    const unsigned char* pk = wbase + slot * C::SLOT;
+    const unsigned char* pv = pk + C::TILE;
+
+    if (flags & kFirst) {
+      const unsigned char* pq = pk + 2 * C::TILE;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(pq + h * C::ROW + dl * 16);
+        E::unpack(raw, qv[h]);
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) {
+          qv[h][e] *= a.scale_log2;
+          o[h][e] = 0.f;
+        }
+      }
+      m_run = -INFINITY;
+      l_run = 0.f;
+      poisoned = false;
+    }
+
+    if (flags & kBad) {
+      poisoned = true;
+    } else {
+      // ---- logits x = q.k (base-2 scaled) for the 16 rows x G heads ----------
+#pragma unroll
+      for (int c = 0; c < C::NCH; ++c) {
+        float v[C::V];
+#pragma unroll
+        for (int i = 0; i < C::CH; ++i) {
+          const int row = (c * C::CH + i) * C::RPI + rgp;
+          if (row < rows) {
+            float kf[C::VEC];
+            E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              float acc = 0.f;
+#pragma unroll
+              for (int e = 0; e < C::VEC; ++e) acc = fmaf(qv[h][e], kf[e], acc);
+              v[i * G + h] = acc;
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < G; ++h) v[i * G + h] = 0.f;
+          }
+        }
+        reduce_scatter<C::LPR, C::V>(v, dl);
+        if ((dl & ((C::LPR >> C::LSC) - 1)) == 0) {
+          const int sel = dl >> (C::LS - C::LSC);
+#pragma unroll
+          for (int r = 0; r < C::NV; ++r) {
+            const int f = sel * C::NV + r;
+            const int row = (c * C::CH + f / G) * C::RPI + rgp;
+            xs[row * G + f % G] = row < rows ? v[r] : -INFINITY;
+          }
+        }
+      }
+      __syncwarp();
+
+      // ---- online softmax: lane owns head hs, tokens lane/G + k*(32/G) ---------
+      float xv[C::TPL];
+      float mb = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < C::TPL; ++t) {
+        const int tok = lane / G + t * (32 / G);
+        xv[t] = tok < kBlockSize ? xs[tok * G + hs] : -INFINITY;
+        mb = fmaxf(mb, xv[t]);
+      }
+#pragma unroll
+      for (int off = G; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
+      const bool grow = mb > m_run + kRescaleThreshold;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = exp2f(m_run - mb);
+        m_run = mb;
+        l_run *= alpha;
+      }
+      if (__any_sync(kFull, grow)) {
+        if (lane < G) alpha_s[lane] = alpha;
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float al = alpha_s[h];
+#pragma unroll
+          for (int e = 0; e < C::VEC; ++e) o[h][e] *= al;
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < C::TPL; ++t) {
+        const int tok = lane / G + t * (32 / G);
+        const float p = exp2f(xv[t] - m_run);
+        if (tok < kBlockSize) {
+          l_run += p;
+          xs[tok * G + hs] = p;
+        }
+      }
+      __syncwarp();
+
+      // ---- o += p . V --------------------------------------------------------
+#pragma unroll
+      for (int i = 0; i < C::RL; ++i) {
+        const int row = i * C::RPI + rgp;
+        if (row < rows) {
+          float vf[C::VEC];
+          E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
+          float p[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) p[h] = xs[row * G + h];
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) o[h][e] = fmaf(p[h], vf[e], o[h][e]);
+        }
+      }
+    }
+    __syncwarp();
+    if (k + DEPTH < nst) issue(k + DEPTH);
+
+    // ---- end of a piece: write the output or a partial -------------------------
+    if (flags & kLast) {
+#pragma unroll
+      for (int off = C::LPR; off < 32; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int e = 0; e < C::VEC; ++e) o[h][e] += __shfl_xor_sync(kFull, o[h][e], off);
+      float lsum = l_run;
+#pragma unroll
+      for (int off = G; off < 32; off <<= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
+      const bool bad = __any_sync(kFull, poisoned);
+      const int s = d.seq;
+      const int nb = (s_len[s] + kBlockSize - 1) / kBlockSize;
+      const long long item_a = s_start[s] + static_cast<long long>(kvh) * nb;
+      const long long ra = rg.of(item_a);
+      const long long rb = rg.of(item_a + nb - 1);
+      const size_t orow = (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D;
+      if (ra == rb) {
+        // the whole (seq, kv head) was this piece: normalise and store
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float lh = __shfl_sync(kFull, lsum, h);
+          if (h % C::RPI != rgp) continue;
+          float r[C::VEC];
+          const float inv = bad ? 0.f : 1.f / lh;
+#pragma unroll
+          for (int e = 0; e < C::VEC; ++e) r[e] = bad ? 0.f : o[h][e] * inv;
+          *reinterpret_cast<uint4*>(static_cast<T*>(a.out) + orow + h * D + dl * C::VEC) =
+              E::pack(r);
+        }
+      } else {
+        const long long r = rg.of(lo + k);
+        const long long sl = 2 * r + (item_a <= rg.start(r) ? 0 : 1);
+        float* wo = a.ws_o + sl * G * D;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          if (h % C::RPI != rgp) continue;
+#pragma unroll
+          for (int e = 0; e < C::VEC; e += 4)
+            *reinterpret_cast<float4*>(wo + h * D + dl * C::VEC + e) =
+                make_float4(o[h][e], o[h][e + 1], o[h][e + 2], o[h][e + 3]);
+        }
+        if (lane < G) a.ws_ml[sl * G + lane] = make_float2(m_run, bad ? -1.f : lsum);
+        __threadfence();
+        __syncwarp();
+        int prev = 0;
+        int* cnt = a.counters + static_cast<size_t>(s) * Hkv + kvh;
+        if (lane == 0) prev = atomicAdd(cnt, 1);
+        prev = __shfl_sync(kFull, prev, 0);
+        if (prev == static_cast<int>(rb - ra)) {
+          // last piece of this (seq, kv head): merge all pieces by log-sum-exp
+          __threadfence();
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            if (h % C::RPI != rgp) continue;
+            float M = -INFINITY;
+            bool any_bad = false;
+            for (long long rr = ra; rr <= rb; ++rr) {
+              const long long ss = 2 * rr + ((rr == ra && item_a > rg.start(rr)) ? 1 : 0);
+              const float2 ml = __ldcg(a.ws_ml + ss * G + h);
+              any_bad |= ml.y < 0.f;
+              M = fmaxf(M, ml.x);
+            }
+            float L = 0.f;
+            float acc[C::VEC];
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) acc[e] = 0.f;
+            for (long long rr = ra; rr <= rb; ++rr) {
+              const long long ss = 2 * rr + ((rr == ra && item_a > rg.start(rr)) ? 1 : 0);
+              const float2 ml = __ldcg(a.ws_ml + ss * G + h);
+              const float w = exp2f(ml.x - M);
+              L += w * ml.y;
+              const float* po = a.ws_o + ss * G * D + h * D + dl * C::VEC;
+#pragma unroll
+              for (int e = 0; e < C::VEC; e += 4) {
+                const float4 t4 = __ldcg(reinterpret_cast<const float4*>(po + e));
+                acc[e] = fmaf(w, t4.x, acc[e]);
+                acc[e + 1] = fmaf(w, t4.y, acc[e + 1]);
+                acc[e + 2] = fmaf(w, t4.z, acc[e + 2]);
+                acc[e + 3] = fmaf(w, t4.w, acc[e + 3]);
+              }
+            }
+            const float inv = any_bad ? 0.f : 1.f / L;
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) acc[e] = any_bad ? 0.f : acc[e] * inv;
+            *reinterpret_cast<uint4*>(static_cast<T*>(a.out) + orow + h * D + dl * C::VEC) =
+                E::pack(acc);
+          }
+          if (lane == 0) *cnt = 0;  // leave the workspace zeroed for the next call
+        }
+      }
+    }
+
+    if (k - base == 31) {
+      A = B;
+      base += 32;
+      B = make_desc(lo + base + 32 + lane, hi, s_start, s_len, rg, a);
+    }
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,49 @@
+// pa_internal.h -- definitions shared by the library's translation units
+// (not part of the public ABI, which is include/paged_attention.h).
+#pragma once
+
+#include <cstdint>
+
+namespace pa {
+
+constexpr int kBlockSize = 16;            // token slots per KV block
+constexpr float kRescaleThreshold = 8.f;  // log2 growth of the running max before o is rescaled
+
+constexpr int kErrBlockId = 1;
+constexpr int kErrContextLen = 2;
+constexpr int kErrSlot = 4;
+constexpr int kErrPair = 8;
+constexpr int kErrTimeout = 16;
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int len_cap;       // longest valid context: min(max_context_len, max_blocks_per_seq * 16)
+  int part_blocks;   // most blocks one partial covers (0 = balanced share)
+  float scale_log2;  // scale * log2(e)
+  int* counters;     // [num_seqs * num_kv_heads] pieces finished, zero between calls
+  float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
+  float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
+  int32_t* err_flag;
+};
+
+struct DecodeKernelInfo {
+  const void* fn;   // the __global__ function
+  int warps;        // warps per CTA
+  int depth;        // ring slots per warp
+  int warp_bytes;   // dynamic shared memory per warp
+};
+
+bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);
+bool decode_kernel_f32(int head_dim, int group, DecodeKernelInfo* info);
+
+}  // namespace pa

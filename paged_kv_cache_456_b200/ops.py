@@ -1,0 +1,172 @@
+"""Python binding of ``libpa.so`` (include/paged_attention.h).
+
+Argument marshalling only: tensors are turned into device pointers and sizes
+and handed to the C ABI on the current CUDA stream.  Every step of the path
+runs in the library's CUDA kernels; there is no fallback.  If the library has
+not been built, :func:`library` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = range(5)
+PA_F32, PA_BF16 = 0, 1
+
+ERRBIT_BLOCK_ID = 1
+ERRBIT_CONTEXT_LEN = 2
+ERRBIT_SLOT = 4
+ERRBIT_PAIR = 8
+ERRBIT_TIMEOUT = 16
+
+EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_init",
+            "pa_decode_launch_config", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks")
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_str(status)}")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library(path: Optional[str] = None) -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m paged_kv_cache_456_b200.build`"
+                           " (the CUDA library is the only implementation)")
+    lib = ctypes.CDLL(p)
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    lib.pa_status_str.argtypes = [i]
+    lib.pa_status_str.restype = ctypes.c_char_p
+    lib.pa_decode_workspace_size.argtypes = [i] * 7 + [ctypes.POINTER(sz)]
+    lib.pa_decode_workspace_size.restype = i
+    lib.pa_decode_workspace_init.argtypes = [vp, sz, vp]
+    lib.pa_decode_workspace_init.restype = i
+    lib.pa_decode_launch_config.argtypes = [i] * 7 + [ctypes.POINTER(i)] * 4
+    lib.pa_decode_launch_config.restype = i
+    lib.pa_decode.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
+    lib.pa_decode.restype = i
+    lib.pa_reshape_and_cache.argtypes = [vp] * 5 + [i] * 6 + [vp, vp]
+    lib.pa_reshape_and_cache.restype = i
+    lib.pa_copy_blocks.argtypes = [vp] * 3 + [i] * 6 + [vp, vp]
+    lib.pa_copy_blocks.restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    return library().pa_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        raise PagedAttentionError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype == torch.float32:
+        return PA_F32
+    raise TypeError(f"unsupported element type {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libpa must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+def workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                   max_context_len: int, partition_size: int = 0,
+                   dtype: torch.dtype = torch.bfloat16) -> int:
+    out = ctypes.c_size_t(0)
+    code = PA_BF16 if dtype == torch.bfloat16 else PA_F32
+    _check(library().pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              max_context_len, partition_size, code,
+                                              ctypes.byref(out)), "pa_decode_workspace_size")
+    return int(out.value)
+
+
+def make_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                   max_context_len: int, partition_size: int = 0,
+                   dtype: torch.dtype = torch.bfloat16, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size ``pa_decode`` needs."""
+    n = workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                       partition_size, dtype)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def launch_config(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                  max_context_len: int, partition_size: int = 0,
+                  dtype: torch.dtype = torch.bfloat16) -> dict:
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    code = PA_BF16 if dtype == torch.bfloat16 else PA_F32
+    _check(library().pa_decode_launch_config(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                             max_context_len, partition_size, code,
+                                             *[ctypes.byref(v) for v in vals]),
+           "pa_decode_launch_config")
+    return dict(zip(("grid", "warps_per_cta", "pipeline_depth", "smem_bytes"),
+                    (v.value for v in vals)))
+
+
+def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           block_tables: torch.Tensor, context_lens: torch.Tensor, *, scale: float,
+           max_context_len: int, workspace: torch.Tensor, partition_size: int = 0,
+           err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """PagedAttention decode into ``out`` ``[S][Hq][D]``; see ``pa_decode``."""
+    S, Hq, D = q.shape
+    N, Hkv, bs, _ = k_cache.shape
+    _check(library().pa_decode(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        S, Hq, Hkv, D, bs, block_tables.shape[1], N, int(max_context_len), float(scale),
+        int(partition_size), _dtype_code(q), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream)), "pa_decode")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# cache maintenance
+# ---------------------------------------------------------------------------
+def reshape_and_cache(key: torch.Tensor, value: torch.Tensor, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                      err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Write ``key``/``value`` ``[T][Hkv][D]`` into the cache slots of ``slot_mapping``."""
+    T = key.shape[0]
+    N, Hkv, bs, D = k_cache.shape
+    _check(library().pa_reshape_and_cache(
+        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, bs, N,
+        _dtype_code(k_cache), _ptr(err_flag), _stream(stream)), "pa_reshape_and_cache")
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor,
+                err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Copy whole blocks ``src -> dst`` for each row of ``block_mapping`` ``[M][2]``."""
+    N, Hkv, bs, D = k_cache.shape
+    _check(library().pa_copy_blocks(
+        _ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), block_mapping.shape[0], Hkv, D, bs, N,
+        _dtype_code(k_cache), _ptr(err_flag), _stream(stream)), "pa_copy_blocks")
