@@ -16,7 +16,8 @@
  * ---------------------------------------
  *  - Every pointer argument except the function's own scalars is a DEVICE
  *    pointer, owned by the caller; the library allocates nothing, keeps no
- *    state between calls, and frees nothing.
+ *    state between calls (apart from the fixed scratch array used by
+ *    pa_decode_noalloc), and frees nothing.
  *  - Element type (pa_dtype) is the same for q, out, key, value and both
  *    caches: IEEE fp32 or bf16.  Arithmetic is fp32 in every case.
  *  - Cache layout, for K and for V alike:
@@ -132,6 +133,37 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     int block_size, int max_blocks_per_seq, int num_blocks,
                     int max_context_len, float scale, int partition_size, pa_dtype dtype,
                     void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode attention without a caller-provided workspace
+ * ------------------------------------------------------------------------
+ * The pages describe no counterpart of this entry point; it exists for
+ * callers that cannot allocate device memory while they run -- an engine
+ * whose memory pool already owns the device, a step loop that cannot take
+ * the device synchronisation cudaMalloc/cudaFree may cause, or a caller with
+ * no allocator at all.
+ *
+ * Same arguments and results as pa_decode, minus the workspace: the scratch
+ * it needs comes from one array of PA_NOALLOC_SCRATCH_BYTES inside the
+ * library (every GPU that loads libpa.so holds it until the process exits).
+ * It allocates nothing and frees nothing.
+ *  - A call whose pa_decode_workspace_size exceeds PA_NOALLOC_SCRATCH_BYTES
+ *    returns PA_ERR_WORKSPACE and launches nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture begins.
+ *  - All calls share the one array.  Each call first clears, on `stream`,
+ *    the part that must start at zero; calls that can run at the same time
+ *    on the GPU (different streams without ordering) race on the array.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int max_blocks_per_seq, int num_blocks,
+                            int max_context_len, float scale, int partition_size,
+                            pa_dtype dtype, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
  * Slot write (reshape_and_cache)
