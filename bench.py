@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--partition-size", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=None)
+    ap.add_argument("--num-blocks", type=int, default=None,
+                    help="pool size override (same lengths; for small profiler captures)")
     return ap.parse_args(argv)
 
 
@@ -187,7 +189,7 @@ def run_reference(args, rank: int, world: int):
         return
     from paged_kv_cache_456_b200.workloads import build_workload
     import oracle
-    w = build_workload(args.workload, seed=args.seed)
+    w = build_workload(args.workload, seed=args.seed, num_blocks=args.num_blocks)
     steps, warm = args.steps, args.warmup
     per_step_budget = max(0.05, 150.0 / max(1, steps + warm))
     _, dt, k, nbytes, threads = oracle_sample(w, per_step_budget)
@@ -239,7 +241,7 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.set_device(dev)
     # rank 0 runs the named workload's own seed; other ranks get independent batches
     seed = args.seed if rank == 0 else (args.seed or 0) + 1000 * rank
-    w = build_workload(args.workload, seed=seed)
+    w = build_workload(args.workload, seed=seed, num_blocks=args.num_blocks)
     if args.partition_size is not None:
         w.partition_size = args.partition_size
     t = upload(w, dev)

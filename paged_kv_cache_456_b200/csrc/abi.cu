@@ -74,7 +74,13 @@ struct DecodePlan {
   int grid = 0;
   size_t smem = 0;
   long long ranges = 0;      // most ranges the device can form
-  size_t counters_off = 0;   // workspace layout
+  int sms = 0;
+  // workspace layout; everything before zero_bytes must be zero on entry
+  size_t heavy_off = 0;      // [2] ints: merge-pass item count, merge CTAs done
+  size_t list_off = 0;       // [S*Hkv] ints: items for the merge pass
+  size_t counters_off = 0;   // [S*Hkv] ints
+  size_t zero_bytes = 0;
+  size_t seq_start_off = 0;  // [S + 1] ints
   size_t o_off = 0;
   size_t ml_off = 0;
   size_t ws_bytes = 0;
@@ -153,15 +159,26 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   }
   if (ranges > tiles_max) ranges = tiles_max > 0 ? tiles_max : 1;
   p->ranges = ranges;
+  p->sms = dev.sms;
   const size_t slots = 2 * static_cast<size_t>(ranges);
-  p->counters_off = 0;
-  p->o_off = round_up(static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int), 256);
+  const size_t items = static_cast<size_t>(num_seqs) * num_kv_heads;
+  // zero-on-entry fields first: the merge pass's count/done pair, the piece counters
+  p->heavy_off = 0;
+  p->counters_off = 2 * sizeof(int);
+  p->zero_bytes = pa::decode_zero_prefix_bytes(num_seqs, num_kv_heads);
+  p->list_off = p->zero_bytes;
+  p->seq_start_off = round_up(p->list_off + items * sizeof(int), 16);
+  p->o_off = round_up(p->seq_start_off + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
   p->ml_off = round_up(p->o_off + slots * group * head_dim * sizeof(float), 256);
   p->ws_bytes = round_up(p->ml_off + slots * group * 2 * sizeof(float), 256);
   return PA_OK;
 }
 
 }  // namespace
+
+size_t pa::decode_zero_prefix_bytes(int num_seqs, int num_kv_heads) {
+  return 2 * sizeof(int) + static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
+}
 
 extern "C" {
 
@@ -255,15 +272,34 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   char* ws = static_cast<char*>(workspace);
   args.counters = reinterpret_cast<int*>(ws + p.counters_off);
+  args.seq_start = reinterpret_cast<int*>(ws + p.seq_start_off);
+  args.heavy = reinterpret_cast<int*>(ws + p.heavy_off);
+  args.heavy_list = reinterpret_cast<int*>(ws + p.list_off);
   args.ws_o = reinterpret_cast<float*>(ws + p.o_off);
   args.ws_ml = reinterpret_cast<float2*>(ws + p.ml_off);
   args.err_flag = err_flag;
 
   void* params[] = {&args};
-  const cudaError_t e =
-      cudaLaunchKernel(p.kernel.fn, dim3(p.grid), dim3(p.kernel.warps * 32), params, p.smem,
-                       static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  if (cudaLaunchKernel(p.kernel.fn, dim3(p.grid), dim3(p.kernel.warps * 32), params, p.smem,
+                       st_) != cudaSuccess)
+    return PA_ERR_CUDA;
+  // merge pass for items split into many pieces, launched behind the decode
+  // kernel with programmatic dependent launch (it waits for the decode grid)
+  int workers = p.grid * p.kernel.warps;
+  void* mparams[] = {&args, &workers};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * p.sms);
+  cfg.blockDim = dim3(pa::kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st_;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, p.kernel.merge_fn, mparams) == cudaSuccess ? PA_OK
+                                                                               : PA_ERR_CUDA;
 }
 
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

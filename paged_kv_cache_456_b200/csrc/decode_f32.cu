@@ -8,6 +8,7 @@ namespace pa {
 template <int D, int G, int DEPTH, int WARPS>
 static bool fill(DecodeKernelInfo* info) {
   info->fn = reinterpret_cast<const void*>(&paged_decode_kernel<float, D, G, DEPTH, WARPS>);
+  info->merge_fn = reinterpret_cast<const void*>(&paged_decode_merge_kernel<float, D, G>);
   info->warps = WARPS;
   info->depth = DEPTH;
   info->warp_bytes = DecodeCfg<float, D, G, DEPTH, WARPS>::WARP_BYTES;

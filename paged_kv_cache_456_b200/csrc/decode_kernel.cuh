@@ -33,6 +33,8 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -42,6 +44,7 @@
 namespace pa {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kMaxOwnRanges = 32;  // range starts a warp keeps in shared memory
 
 // -- element conversion ---------------------------------------------------------
 template <typename T>
@@ -83,6 +86,78 @@ struct Elem<__nv_bfloat16> {
   }
 };
 
+// How tiles reach shared memory: 0 = one bulk copy per K/V tile issued by
+// lane 0 (completion counted in bytes); 1 = every lane copies 16-byte pieces
+// with cp.async and arrives on the slot's mbarrier when its copies land.
+#ifndef PA_COPY_ENGINE
+#define PA_COPY_ENGINE 0
+#endif
+constexpr bool kLaneCopies = PA_COPY_ENGINE == 1;
+
+// Tiles ahead of the shared-memory ring that are prefetched into L2, so the
+// ring only has to cover L2 latency while DRAM sees a deep queue (0 = off).
+#ifndef PA_L2_PREFETCH
+#define PA_L2_PREFETCH 0
+#endif
+constexpr int kPrefetch = PA_L2_PREFETCH;
+
+// -- the two inner loops, on packed fp32 pairs (sm_100 FFMA2) or scalar FMAs ---
+#ifndef PA_PACKED_FMA
+#define PA_PACKED_FMA 1
+#endif
+
+// sum_e q[e] * k[e] over one lane's VEC elements
+template <int VEC>
+__device__ __forceinline__ float dot_vec(const float* q, const float* k) {
+#if PA_PACKED_FMA
+  float2 acc = __fmul2_rn(make_float2(q[0], q[1]), make_float2(k[0], k[1]));
+#pragma unroll
+  for (int j = 1; j < VEC / 2; ++j)
+    acc = __ffma2_rn(make_float2(q[2 * j], q[2 * j + 1]), make_float2(k[2 * j], k[2 * j + 1]), acc);
+  return acc.x + acc.y;
+#else
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc = fmaf(q[e], k[e], acc);
+  return acc;
+#endif
+}
+
+// o[e] += p * v[e]
+template <int VEC>
+__device__ __forceinline__ void axpy_vec(float p, const float* v, float* o) {
+#if PA_PACKED_FMA
+  const float2 pp = make_float2(p, p);
+#pragma unroll
+  for (int j = 0; j < VEC / 2; ++j) {
+    const float2 r =
+        __ffma2_rn(pp, make_float2(v[2 * j], v[2 * j + 1]), make_float2(o[2 * j], o[2 * j + 1]));
+    o[2 * j] = r.x;
+    o[2 * j + 1] = r.y;
+  }
+#else
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) o[e] = fmaf(p, v[e], o[e]);
+#endif
+}
+
+// o[e] *= s
+template <int VEC>
+__device__ __forceinline__ void scale_vec(float s, float* o) {
+#if PA_PACKED_FMA
+  const float2 ss = make_float2(s, s);
+#pragma unroll
+  for (int j = 0; j < VEC / 2; ++j) {
+    const float2 r = __fmul2_rn(ss, make_float2(o[2 * j], o[2 * j + 1]));
+    o[2 * j] = r.x;
+    o[2 * j + 1] = r.y;
+  }
+#else
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) o[e] *= s;
+#endif
+}
+
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
@@ -100,14 +175,18 @@ struct DecodeCfg {
   static constexpr int SLOT = 2 * TILE + QB;  // K tile, V tile, q
   static constexpr int XS = kBlockSize * G * 4;
   static constexpr int ALPHA = ((G * 4 + 15) / 16) * 16;
-  static constexpr int WARP_BYTES = ((DEPTH * SLOT + XS + ALPHA + DEPTH * 8 + 127) / 128) * 128;
+  static constexpr int BND = (kMaxOwnRanges + 1) * 8;
+  static constexpr int WARP_BYTES =
+      ((DEPTH * SLOT + XS + ALPHA + DEPTH * 8 + BND + 127) / 128) * 128;
   // QK is done CH rows at a time; V = CH*G partial dots are reduce-scattered
   // over the LPR lanes of a row, leaving NV finished logits per lane.
   static constexpr int CH = cmin(RL, LPR / G >= 1 ? LPR / G : 1);
   static constexpr int NCH = RL / CH;
   static constexpr int V = CH * G;
   static constexpr int LS = ilog2(LPR);
-  static constexpr int LSC = cmin(LS, ilog2(V));
+  static constexpr int LV = ilog2(V);
+  static constexpr int LG = ilog2(G);
+  static constexpr int LSC = cmin(LS, LV);
   static constexpr int NV = V >> LSC;
   static constexpr int TPL = G >= 2 ? G / 2 : 1;  // softmax tokens per lane
   static_assert(VEC * LPR == D, "head_dim must be a multiple of 16 bytes");
@@ -127,6 +206,39 @@ struct Ranges {
   }
 };
 
+// Starts of the ranges one warp owns, kept in shared memory so that the
+// per-tile "does a range start here" test needs no 64-bit division.
+struct OwnRanges {
+  const long long* b;  // b[0] = first tile of the warp ... b[n] = one past its last
+  int n;               // ranges owned; 0 = more than kMaxOwnRanges (fall back to division)
+  __device__ __forceinline__ bool is_start(long long x, const Ranges& rg) const {
+    if (n == 0) return rg.is_start(x);
+    int l = 0, u = n;
+    while (l < u) {
+      const int m = (l + u) >> 1;
+      if (b[m] < x) l = m + 1; else u = m;
+    }
+    return b[l] == x;
+  }
+};
+
+// The cut of W tiles over `workers` warps: one range per warp, or more so
+// that no range exceeds part_blocks tiles (part_blocks = 0: no bound).
+__device__ __forceinline__ Ranges make_ranges(long long W, long long workers, int part_blocks) {
+  long long R = workers;
+  if (part_blocks > 0) {
+    const long long per = workers * part_blocks;
+    R = workers * max(1LL, (W + per - 1) / per);
+  }
+  if (R > W) R = W;
+  return Ranges{W, R};
+}
+
+// Partial-result slot of the piece of item [item_a, ...) that lies in range r.
+__device__ __forceinline__ long long piece_slot(const Ranges& rg, long long r, long long item_a) {
+  return 2 * r + (item_a <= rg.start(r) ? 0 : 1);
+}
+
 // One tile of a warp's stream, as 3 words (kept one per lane, 32 tiles per batch).
 struct StageDesc {
   int phys;  // physical block id (0 if bad)
@@ -139,7 +251,7 @@ constexpr int kBad = 1 << 26;    // block-table entry out of range
 
 __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
                                                const int* s_len, const Ranges& rg,
-                                               const DecodeArgs& a) {
+                                               const OwnRanges& own, const DecodeArgs& a) {
   StageDesc d{0, 0, 0};
   if (g >= hi) return d;
   // largest s with s_start[s] <= g (sequences without blocks share their start)
@@ -156,8 +268,8 @@ __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const 
   const int blk = off - kvh * nb;
   const long long item_a = s_start[s] + static_cast<long long>(kvh) * nb;
   int flags = 0;
-  if (g == item_a || rg.is_start(g)) flags |= kFirst;
-  if (g + 1 == item_a + nb || rg.is_start(g + 1)) flags |= kLast;
+  if (g == item_a || own.is_start(g, rg)) flags |= kFirst;
+  if (g + 1 == item_a + nb || own.is_start(g + 1, rg)) flags |= kLast;
   int phys = __ldg(a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + blk);
   if (phys < 0 || phys >= a.num_blocks) {
     flags |= kBad;
@@ -181,23 +293,21 @@ __device__ __forceinline__ StageDesc pick_desc(const StageDesc& A, const StageDe
   return d;
 }
 
-// Butterfly reduce-scatter of V values over the LPR lanes of a row group:
-// afterwards v[0..NV) of lane dl hold complete sums of value indices
-// (dl >> (LS - LSC)) * NV + r.
+// Butterfly reduce-scatter of V values over the LPR lanes of a row group.
+// Each lane computes its partials in a lane-dependent order (array index f
+// holds logical index f ^ mask, mask = the lane's bits above the kept part),
+// so at every stage all lanes keep the lower half and send the upper half:
+// no per-element selects.  Afterwards v[0..NV) of lane dl hold complete sums
+// of logical indices (dl >> (LS - LSC)) * NV + r.
 template <int LPR, int V>
-__device__ __forceinline__ void reduce_scatter(float (&v)[V], int dl) {
+__device__ __forceinline__ void reduce_scatter(float (&v)[V]) {
 #pragma unroll
   for (int st = 0; (1 << st) < LPR; ++st) {
     const int o = LPR >> (st + 1);
     const int len = V >> st;
     if (len >= 2) {
-      const bool upper = (dl & o) != 0;
 #pragma unroll
-      for (int i = 0; i < len / 2; ++i) {
-        const float send = upper ? v[i] : v[len / 2 + i];
-        const float keep = upper ? v[len / 2 + i] : v[i];
-        v[i] = keep + __shfl_xor_sync(kFull, send, o);
-      }
+      for (int i = 0; i < len / 2; ++i) v[i] += __shfl_xor_sync(kFull, v[len / 2 + i], o);
     } else {
       v[0] += __shfl_xor_sync(kFull, v[0], o);
     }
@@ -270,30 +380,42 @@ paged_decode_kernel(const DecodeArgs a) {
   }
 
   // ---- this warp's share of the tiles -------------------------------------------
+  // the merge pass (launched after this kernel) may start its prologue now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (blockIdx.x == 0)
+    for (int s = tid; s <= S; s += WARPS * 32) a.seq_start[s] = s_start[s];
+
   const long long W = s_start[S];
   if (W == 0) return;
   const long long NWK = static_cast<long long>(gridDim.x) * WARPS;
-  long long R = NWK;
-  if (a.part_blocks > 0) {
-    const long long per = NWK * a.part_blocks;
-    R = NWK * max(1LL, (W + per - 1) / per);
-  }
-  if (R > W) R = W;
-  const Ranges rg{W, R};
+  const Ranges rg = make_ranges(W, NWK, a.part_blocks);
   const long long gw = static_cast<long long>(blockIdx.x) * WARPS + warp;
-  const long long lo = rg.start(gw * R / NWK);
-  const long long hi = rg.start((gw + 1) * R / NWK);
-  if (lo >= hi) return;
-  const int nst = static_cast<int>(hi - lo);
+  const long long r0 = gw * rg.R / NWK;
+  const long long r1 = (gw + 1) * rg.R / NWK;
+  if (r0 >= r1) return;  // more warps than ranges
 
   unsigned char* wbase = smem + warp * C::WARP_BYTES;
+  long long* bnd = reinterpret_cast<long long*>(wbase + DEPTH * C::SLOT + C::XS + C::ALPHA +
+                                                DEPTH * 8);
+  OwnRanges own{bnd, r1 - r0 <= kMaxOwnRanges ? static_cast<int>(r1 - r0) : 0};
+  long long lo, hi;
+  if (own.n > 0) {
+    if (lane <= own.n) bnd[lane] = rg.start(r0 + lane);  // one division per lane, in parallel
+    __syncwarp();
+    lo = bnd[0];
+    hi = bnd[own.n];
+  } else {
+    lo = rg.start(r0);
+    hi = rg.start(r1);
+  }
+  const int nst = static_cast<int>(hi - lo);
   const uint32_t slot0 = smem_addr(wbase);
   float* xs = reinterpret_cast<float*>(wbase + DEPTH * C::SLOT);
   float* alpha_s = reinterpret_cast<float*>(wbase + DEPTH * C::SLOT + C::XS);
   const uint32_t bar0 = smem_addr(wbase + DEPTH * C::SLOT + C::XS + C::ALPHA);
   if (lane == 0) {
 #pragma unroll
-    for (int j = 0; j < DEPTH; ++j) mbar_init(bar0 + 8 * j, 1);
+    for (int j = 0; j < DEPTH; ++j) mbar_init(bar0 + 8 * j, kLaneCopies ? 32 : 1);
     fence_barrier_init();
   }
   __syncwarp();
@@ -301,17 +423,57 @@ paged_decode_kernel(const DecodeArgs a) {
   const int dl = lane % C::LPR;  // which 16 bytes of a row
   const int rgp = lane / C::LPR; // which row group
   const int hs = lane % G;       // softmax: head of this lane
+  // reduce-scatter order of this lane: its partial at array index i*G + h is
+  // the logical (row i ^ imask, head h ^ hmask) of the chunk
+  const int perm = (dl >> (C::LS - C::LSC)) << (C::LV - C::LSC);
+  const int imask = perm >> C::LG;
+  const int hmask = perm & (G - 1);
 
-  StageDesc A = make_desc(lo + lane, hi, s_start, s_len, rg, a);
-  StageDesc B = make_desc(lo + 32 + lane, hi, s_start, s_len, rg, a);
+  StageDesc A = make_desc(lo + lane, hi, s_start, s_len, rg, own, a);
+  StageDesc B = make_desc(lo + 32 + lane, hi, s_start, s_len, rg, own, a);
   int base = 0;
 
   // Fill ring slot j % DEPTH with tile j: K and V rows, plus q on a piece start.
+  // L2 prefetch of tile j by the lane that holds its descriptor (j - base < 64)
+  auto prefetch = [&](int j) {
+    if (kPrefetch == 0 || j >= nst) return;
+    const int rel = j - base;
+    const StageDesc& e = rel < 32 ? A : B;
+    if (lane == (rel & 31) && !(e.meta & kBad)) {
+      const int kvh = e.meta & 0xffff;
+      const uint32_t bytes = static_cast<uint32_t>((e.meta >> 16) & 31) * C::ROW;
+      const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
+      bulk_prefetch_l2(static_cast<const char*>(a.k_cache) + off, bytes);
+      bulk_prefetch_l2(static_cast<const char*>(a.v_cache) + off, bytes);
+    }
+  };
+
   auto issue = [&](int j) {
+    if (kPrefetch > 0) prefetch(j + kPrefetch);
     const StageDesc e = pick_desc(A, B, j - base);
-    if (lane == 0) {
-      const int slot = j % DEPTH;
-      const uint32_t bar = bar0 + 8 * slot;
+    const int slot = j % DEPTH;
+    const uint32_t bar = bar0 + 8 * slot;
+    if constexpr (kLaneCopies) {
+      if (!(e.meta & kBad)) {
+        const int kvh = e.meta & 0xffff;
+        const int rows = (e.meta >> 16) & 31;
+        const uint32_t dst = slot0 + slot * C::SLOT;
+        const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
+        const char* ks = static_cast<const char*>(a.k_cache) + off;
+        const char* vs = static_cast<const char*>(a.v_cache) + off;
+        const int chunks = rows * (C::ROW / 16);
+        for (int c = lane; c < chunks; c += 32) {
+          cp_async_16(dst + 16 * c, ks + 16 * c);
+          cp_async_16(dst + C::TILE + 16 * c, vs + 16 * c);
+        }
+        if (e.meta & kFirst) {
+          const char* qs = static_cast<const char*>(a.q) +
+                           (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * G) * C::ROW;
+          for (int c = lane; c < C::QB / 16; c += 32) cp_async_16(dst + 2 * C::TILE + 16 * c, qs + 16 * c);
+        }
+      }
+      cp_async_mbar_arrive(bar);
+    } else if (lane == 0) {
       if (e.meta & kBad) {
         mbar_arrive(bar);  // nothing to fetch; complete the phase
       } else {
@@ -335,6 +497,8 @@ paged_decode_kernel(const DecodeArgs a) {
     }
   };
 
+  static_assert(kPrefetch + DEPTH < 32, "prefetch distance must stay within two batches");
+  for (int j = DEPTH; j < DEPTH + kPrefetch && j < kPrefetch; ++j) prefetch(j);
   for (int j = 0; j < DEPTH && j < nst; ++j) issue(j);
 
   float qv[G][C::VEC];
@@ -363,7 +527,9 @@ paged_decode_kernel(const DecodeArgs a) {
       const unsigned char* pq = pk + 2 * C::TILE;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(pq + h * C::ROW + dl * 16);
+        // one head keeps the natural order; more heads are permuted (see reduce_scatter)
+        const int hq = G == 1 ? h : (h ^ hmask);
+        const uint4 raw = *reinterpret_cast<const uint4*>(pq + hq * C::ROW + dl * 16);
         E::unpack(raw, qv[h]);
 #pragma unroll
         for (int e = 0; e < C::VEC; ++e) {
@@ -376,99 +542,141 @@ paged_decode_kernel(const DecodeArgs a) {
       poisoned = false;
     }
 
-    if (flags & kBad) {
-      poisoned = true;
-    } else {
-      // ---- logits x = q.k (base-2 scaled) for the 16 rows x G heads ----------
+    // One tile: MASK = the tile has fewer than 16 live rows (only the last
+    // tile of a sequence); full tiles take the branch-free path.
+    auto compute_tile = [&](auto mask_tag) {
+      constexpr bool MASK = decltype(mask_tag)::value;
+      if constexpr (G == 1) {
+        // ---- one query head: every lane keeps the logits of its row group ----
+        float x[C::RL];
 #pragma unroll
-      for (int c = 0; c < C::NCH; ++c) {
-        float v[C::V];
-#pragma unroll
-        for (int i = 0; i < C::CH; ++i) {
-          const int row = (c * C::CH + i) * C::RPI + rgp;
-          if (row < rows) {
+        for (int i = 0; i < C::RL; ++i) {
+          const int row = i * C::RPI + rgp;
+          x[i] = 0.f;
+          if (!MASK || row < rows) {
             float kf[C::VEC];
             E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              float acc = 0.f;
-#pragma unroll
-              for (int e = 0; e < C::VEC; ++e) acc = fmaf(qv[h][e], kf[e], acc);
-              v[i * G + h] = acc;
-            }
-          } else {
-#pragma unroll
-            for (int h = 0; h < G; ++h) v[i * G + h] = 0.f;
+            x[i] = dot_vec<C::VEC>(qv[0], kf);
           }
         }
-        reduce_scatter<C::LPR, C::V>(v, dl);
-        if ((dl & ((C::LPR >> C::LSC) - 1)) == 0) {
-          const int sel = dl >> (C::LS - C::LSC);
 #pragma unroll
-          for (int r = 0; r < C::NV; ++r) {
-            const int f = sel * C::NV + r;
-            const int row = (c * C::CH + f / G) * C::RPI + rgp;
-            xs[row * G + f % G] = row < rows ? v[r] : -INFINITY;
-          }
+        for (int off = C::LPR / 2; off >= 1; off >>= 1)
+#pragma unroll
+          for (int i = 0; i < C::RL; ++i) x[i] += __shfl_xor_sync(kFull, x[i], off);
+        float mb = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < C::RL; ++i) {
+          if (MASK && i * C::RPI + rgp >= rows) x[i] = -INFINITY;
+          mb = fmaxf(mb, x[i]);
         }
-      }
-      __syncwarp();
-
-      // ---- online softmax: lane owns head hs, tokens lane/G + k*(32/G) ---------
-      float xv[C::TPL];
-      float mb = -INFINITY;
 #pragma unroll
-      for (int t = 0; t < C::TPL; ++t) {
-        const int tok = lane / G + t * (32 / G);
-        xv[t] = tok < kBlockSize ? xs[tok * G + hs] : -INFINITY;
-        mb = fmaxf(mb, xv[t]);
-      }
-#pragma unroll
-      for (int off = G; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
-      const bool grow = mb > m_run + kRescaleThreshold;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = exp2f(m_run - mb);
-        m_run = mb;
-        l_run *= alpha;
-      }
-      if (__any_sync(kFull, grow)) {
-        if (lane < G) alpha_s[lane] = alpha;
-        __syncwarp();
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float al = alpha_s[h];
-#pragma unroll
-          for (int e = 0; e < C::VEC; ++e) o[h][e] *= al;
+        for (int off = C::LPR; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
+        if (mb > m_run + kRescaleThreshold) {  // warp-uniform
+          const float alpha = exp2f(m_run - mb);
+          m_run = mb;
+          l_run *= alpha;
+          scale_vec<C::VEC>(alpha, o[0]);
         }
-      }
 #pragma unroll
-      for (int t = 0; t < C::TPL; ++t) {
-        const int tok = lane / G + t * (32 / G);
-        const float p = exp2f(xv[t] - m_run);
-        if (tok < kBlockSize) {
+        for (int i = 0; i < C::RL; ++i) {
+          const int row = i * C::RPI + rgp;
+          const float p = exp2f(x[i] - m_run);
           l_run += p;
-          xs[tok * G + hs] = p;
+          if (!MASK || row < rows) {
+            float vf[C::VEC];
+            E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
+            axpy_vec<C::VEC>(p, vf, o[0]);
+          }
         }
-      }
-      __syncwarp();
+      } else {
+        // ---- logits x = q.k (base-2 scaled) for the 16 rows x G heads --------
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          float v[C::V];
+#pragma unroll
+          for (int i = 0; i < C::CH; ++i) {
+            const int row = (c * C::CH + (i ^ imask)) * C::RPI + rgp;
+            if (!MASK || row < rows) {
+              float kf[C::VEC];
+              E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
+#pragma unroll
+              for (int h = 0; h < G; ++h) v[i * G + h] = dot_vec<C::VEC>(qv[h], kf);
+            } else {
+#pragma unroll
+              for (int h = 0; h < G; ++h) v[i * G + h] = 0.f;
+            }
+          }
+          reduce_scatter<C::LPR, C::V>(v);
+          if ((dl & ((C::LPR >> C::LSC) - 1)) == 0) {
+            const int sel = dl >> (C::LS - C::LSC);
+#pragma unroll
+            for (int r = 0; r < C::NV; ++r) {
+              const int f = sel * C::NV + r;
+              const int row = (c * C::CH + f / G) * C::RPI + rgp;
+              xs[row * G + f % G] = (!MASK || row < rows) ? v[r] : -INFINITY;
+            }
+          }
+        }
+        __syncwarp();
 
-      // ---- o += p . V --------------------------------------------------------
+        // ---- online softmax: lane owns head hs, tokens lane/G + k*(32/G) -------
+        float xv[C::TPL];
+        float mb = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < C::RL; ++i) {
-        const int row = i * C::RPI + rgp;
-        if (row < rows) {
-          float vf[C::VEC];
-          E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
-          float p[G];
+        for (int t = 0; t < C::TPL; ++t) {
+          const int tok = lane / G + t * (32 / G);
+          xv[t] = tok < kBlockSize ? xs[tok * G + hs] : -INFINITY;
+          mb = fmaxf(mb, xv[t]);
+        }
 #pragma unroll
-          for (int h = 0; h < G; ++h) p[h] = xs[row * G + h];
+        for (int off = G; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, off));
+        const bool grow = mb > m_run + kRescaleThreshold;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = exp2f(m_run - mb);
+          m_run = mb;
+          l_run *= alpha;
+        }
+        if (__any_sync(kFull, grow)) {
+          if (lane < G) alpha_s[lane] = alpha;
+          __syncwarp();
 #pragma unroll
-          for (int h = 0; h < G; ++h)
+          for (int h = 0; h < G; ++h) scale_vec<C::VEC>(alpha_s[h], o[h]);
+        }
 #pragma unroll
-            for (int e = 0; e < C::VEC; ++e) o[h][e] = fmaf(p[h], vf[e], o[h][e]);
+        for (int t = 0; t < C::TPL; ++t) {
+          const int tok = lane / G + t * (32 / G);
+          const float p = exp2f(xv[t] - m_run);
+          if (tok < kBlockSize) {
+            l_run += p;
+            xs[tok * G + hs] = p;
+          }
+        }
+        __syncwarp();
+
+        // ---- o += p . V ------------------------------------------------------
+#pragma unroll
+        for (int i = 0; i < C::RL; ++i) {
+          const int row = i * C::RPI + rgp;
+          if (!MASK || row < rows) {
+            float vf[C::VEC];
+            E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
+            float p[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) p[h] = xs[row * G + h];
+#pragma unroll
+            for (int h = 0; h < G; ++h) axpy_vec<C::VEC>(p[h], vf, o[h]);
+          }
         }
       }
+    };
+
+    if (flags & kBad) {
+      poisoned = true;
+    } else if (rows == kBlockSize) {
+      compute_tile(std::false_type{});
+    } else {
+      compute_tile(std::true_type{});
     }
     __syncwarp();
     if (k + DEPTH < nst) issue(k + DEPTH);
@@ -481,9 +689,12 @@ paged_decode_kernel(const DecodeArgs a) {
         for (int h = 0; h < G; ++h)
 #pragma unroll
           for (int e = 0; e < C::VEC; ++e) o[h][e] += __shfl_xor_sync(kFull, o[h][e], off);
+      // l: with one head every lane of a row group holds that group's sum;
+      // otherwise lanes sharing a head hold disjoint token sums
       float lsum = l_run;
 #pragma unroll
-      for (int off = G; off < 32; off <<= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
+      for (int off = (G == 1 ? C::LPR : G); off < 32; off <<= 1)
+        lsum += __shfl_xor_sync(kFull, lsum, off);
       const bool bad = __any_sync(kFull, poisoned);
       const int s = d.seq;
       const int nb = (s_len[s] + kBlockSize - 1) / kBlockSize;
@@ -506,7 +717,7 @@ paged_decode_kernel(const DecodeArgs a) {
         }
       } else {
         const long long r = rg.of(lo + k);
-        const long long sl = 2 * r + (item_a <= rg.start(r) ? 0 : 1);
+        const long long sl = piece_slot(rg, r, item_a);
         float* wo = a.ws_o + sl * G * D;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -517,52 +728,61 @@ paged_decode_kernel(const DecodeArgs a) {
                 make_float4(o[h][e], o[h][e + 1], o[h][e + 2], o[h][e + 3]);
         }
         if (lane < G) a.ws_ml[sl * G + lane] = make_float2(m_run, bad ? -1.f : lsum);
-        __threadfence();
-        __syncwarp();
-        int prev = 0;
-        int* cnt = a.counters + static_cast<size_t>(s) * Hkv + kvh;
-        if (lane == 0) prev = atomicAdd(cnt, 1);
-        prev = __shfl_sync(kFull, prev, 0);
-        if (prev == static_cast<int>(rb - ra)) {
-          // last piece of this (seq, kv head): merge all pieces by log-sum-exp
-          __threadfence();
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            if (h % C::RPI != rgp) continue;
-            float M = -INFINITY;
-            bool any_bad = false;
-            for (long long rr = ra; rr <= rb; ++rr) {
-              const long long ss = 2 * rr + ((rr == ra && item_a > rg.start(rr)) ? 1 : 0);
-              const float2 ml = __ldcg(a.ws_ml + ss * G + h);
-              any_bad |= ml.y < 0.f;
-              M = fmaxf(M, ml.x);
-            }
-            float L = 0.f;
-            float acc[C::VEC];
-#pragma unroll
-            for (int e = 0; e < C::VEC; ++e) acc[e] = 0.f;
-            for (long long rr = ra; rr <= rb; ++rr) {
-              const long long ss = 2 * rr + ((rr == ra && item_a > rg.start(rr)) ? 1 : 0);
-              const float2 ml = __ldcg(a.ws_ml + ss * G + h);
-              const float w = exp2f(ml.x - M);
-              L += w * ml.y;
-              const float* po = a.ws_o + ss * G * D + h * D + dl * C::VEC;
-#pragma unroll
-              for (int e = 0; e < C::VEC; e += 4) {
-                const float4 t4 = __ldcg(reinterpret_cast<const float4*>(po + e));
-                acc[e] = fmaf(w, t4.x, acc[e]);
-                acc[e + 1] = fmaf(w, t4.y, acc[e + 1]);
-                acc[e + 2] = fmaf(w, t4.z, acc[e + 2]);
-                acc[e + 3] = fmaf(w, t4.w, acc[e + 3]);
-              }
-            }
-            const float inv = any_bad ? 0.f : 1.f / L;
-#pragma unroll
-            for (int e = 0; e < C::VEC; ++e) acc[e] = any_bad ? 0.f : acc[e] * inv;
-            *reinterpret_cast<uint4*>(static_cast<T*>(a.out) + orow + h * D + dl * C::VEC) =
-                E::pack(acc);
+        const bool heavy = (rb - ra + 1) * G > kFuseMaxValues;
+        if (heavy) {
+          // many pieces: the merge pass combines them; the first piece lists the item
+          if (r == ra && lane == 0) {
+            const int idx = atomicAdd(a.heavy, 1);
+            a.heavy_list[idx] = s * Hkv + kvh;
           }
-          if (lane == 0) *cnt = 0;  // leave the workspace zeroed for the next call
+        } else {
+          __threadfence();
+          __syncwarp();
+          int prev = 0;
+          int* cnt = a.counters + static_cast<size_t>(s) * Hkv + kvh;
+          if (lane == 0) prev = atomicAdd(cnt, 1);
+          prev = __shfl_sync(kFull, prev, 0);
+          if (prev == static_cast<int>(rb - ra)) {
+            // last piece of this (seq, kv head): merge all pieces by log-sum-exp
+            __threadfence();
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              if (h % C::RPI != rgp) continue;
+              float M = -INFINITY;
+              bool any_bad = false;
+              for (long long rr = ra; rr <= rb; ++rr) {
+                const long long ss = piece_slot(rg, rr, item_a);
+                const float2 ml = __ldcg(a.ws_ml + ss * G + h);
+                any_bad |= ml.y < 0.f;
+                M = fmaxf(M, ml.x);
+              }
+              float L = 0.f;
+              float acc[C::VEC];
+#pragma unroll
+              for (int e = 0; e < C::VEC; ++e) acc[e] = 0.f;
+              for (long long rr = ra; rr <= rb; ++rr) {
+                const long long ss = piece_slot(rg, rr, item_a);
+                const float2 ml = __ldcg(a.ws_ml + ss * G + h);
+                const float w = exp2f(ml.x - M);
+                L += w * ml.y;
+                const float* po = a.ws_o + ss * G * D + h * D + dl * C::VEC;
+#pragma unroll
+                for (int e = 0; e < C::VEC; e += 4) {
+                  const float4 t4 = __ldcg(reinterpret_cast<const float4*>(po + e));
+                  acc[e] = fmaf(w, t4.x, acc[e]);
+                  acc[e + 1] = fmaf(w, t4.y, acc[e + 1]);
+                  acc[e + 2] = fmaf(w, t4.z, acc[e + 2]);
+                  acc[e + 3] = fmaf(w, t4.w, acc[e + 3]);
+                }
+              }
+              const float inv = any_bad ? 0.f : 1.f / L;
+#pragma unroll
+              for (int e = 0; e < C::VEC; ++e) acc[e] = any_bad ? 0.f : acc[e] * inv;
+              *reinterpret_cast<uint4*>(static_cast<T*>(a.out) + orow + h * D + dl * C::VEC) =
+                  E::pack(acc);
+            }
+            if (lane == 0) *cnt = 0;  // leave the workspace zeroed for the next call
+          }
         }
       }
     }
@@ -570,7 +790,106 @@ paged_decode_kernel(const DecodeArgs a) {
     if (k - base == 31) {
       A = B;
       base += 32;
-      B = make_desc(lo + base + 32 + lane, hi, s_start, s_len, rg, a);
+      B = make_desc(lo + base + 32 + lane, hi, s_start, s_len, rg, own, a);
+    }
+  }
+}
+
+// Merge pass for (seq, kv head) items split into many pieces (long contexts):
+// one CTA per (item, query head) at a time, kMergeThreads / 32 groups of lanes
+// taking every GROUPS-th piece, combined in shared memory:
+//     M = max_j m_j,  out = sum_j 2^(m_j - M) o_j / sum_j 2^(m_j - M) l_j.
+// Launched right behind the decode kernel with programmatic dependent launch;
+// griddepcontrol.wait returns once the decode grid has finished and its
+// writes are visible.  The last CTA to finish resets the item list.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kMergeThreads)
+paged_decode_merge_kernel(const DecodeArgs a, int workers) {
+  constexpr int GROUPS = kMergeThreads / 32;
+  constexpr int DPL = D / 32;  // dims per lane
+  __shared__ float s_m[GROUPS];
+  __shared__ float s_l[GROUPS];
+  __shared__ int s_bad[GROUPS];
+  __shared__ __align__(16) float s_acc[GROUPS][D];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int tid = threadIdx.x, grp = tid >> 5, lane = tid & 31;
+  const int S = a.num_seqs, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
+  const int count = __ldcg(a.heavy);
+  const long long W = __ldcg(a.seq_start + S);
+  if (W > 0) {
+    const Ranges rg = make_ranges(W, workers, a.part_blocks);
+    for (int p = blockIdx.x; p < count * G; p += gridDim.x) {
+      const int item = __ldcg(a.heavy_list + p / G);
+      const int hl = p % G;
+      const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
+      const int st = __ldcg(a.seq_start + s);
+      const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
+      const long long item_a = st + static_cast<long long>(kvh) * nb;
+      const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
+
+      float M = -INFINITY;
+      int bad = 0;
+      for (long long r = ra + grp; r <= rb; r += GROUPS) {
+        const float2 ml = __ldcg(a.ws_ml + piece_slot(rg, r, item_a) * G + hl);
+        M = fmaxf(M, ml.x);
+        bad |= ml.y < 0.f;
+      }
+      if (lane == 0) {
+        s_m[grp] = M;
+        s_bad[grp] = bad;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) {
+        M = fmaxf(M, s_m[g]);
+        bad |= s_bad[g];
+      }
+      float acc[DPL];
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+      float L = 0.f;
+      for (long long r = ra + grp; r <= rb; r += GROUPS) {
+        const long long sl = piece_slot(rg, r, item_a);
+        const float2 ml = __ldcg(a.ws_ml + sl * G + hl);
+        const float w = exp2f(ml.x - M);
+        L = fmaf(w, ml.y, L);
+        const float* po = a.ws_o + (sl * G + hl) * D + lane * DPL;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, __ldcg(po + d), acc[d]);
+      }
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) s_acc[grp][lane * DPL + d] = acc[d];
+      if (lane == 0) s_l[grp] = L;
+      __syncthreads();
+      if (grp == 0) {
+        float Lt = 0.f;
+#pragma unroll
+        for (int g = 0; g < GROUPS; ++g) Lt += s_l[g];
+        float r[DPL];
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) {
+          float t = 0.f;
+#pragma unroll
+          for (int g = 0; g < GROUPS; ++g) t += s_acc[g][lane * DPL + d];
+          r[d] = bad ? 0.f : t / Lt;
+        }
+        T* dst = static_cast<T*>(a.out) +
+                 (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G + hl) * D + lane * DPL;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) dst[d] = static_cast<T>(r[d]);
+      }
+      __syncthreads();
+    }
+  }
+  // the last CTA out clears the item list for the next call
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(a.heavy + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      a.heavy[0] = 0;
+      a.heavy[1] = 0;
+      __threadfence();
     }
   }
 }

@@ -16,8 +16,8 @@
 // that pointer is what the launch receives.
 //
 // Every call shares the one array and it keeps whatever the last call left
-// there.  The part that must start at zero (the per-(sequence, KV head)
-// piece counters) is cleared with cudaMemsetAsync on the caller's stream
+// there.  The part that must start at zero (the merge-pass header and the
+// per-(sequence, KV head) piece counters) is cleared with cudaMemsetAsync on the caller's stream
 // before each launch.  Calls whose work can overlap on the GPU (different
 // streams, no ordering between them) race on the array.
 #include <cmath>
@@ -28,6 +28,7 @@
 #include <cuda_runtime.h>
 
 #include "paged_attention.h"
+#include "pa_internal.h"
 
 namespace {
 
@@ -82,10 +83,9 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
   if (need > static_cast<size_t>(PA_NOALLOC_SCRATCH_BYTES)) return PA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = scratch_for(&scratch)) != PA_OK) return st;
-  // the piece counters sit at the start of the scratch and must begin at zero
-  const size_t counters = static_cast<size_t>(num_seqs) * static_cast<size_t>(num_kv_heads) *
-                          sizeof(int32_t);
-  if (cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // the fields that must begin at zero sit at the start of the scratch
+  const size_t zero = pa::decode_zero_prefix_bytes(num_seqs, num_kv_heads);
+  if (cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return PA_ERR_CUDA;
   return pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
                    num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,

@@ -2,6 +2,7 @@
 // (not part of the public ABI, which is include/paged_attention.h).
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 
 namespace pa {
@@ -31,19 +32,32 @@ struct DecodeArgs {
   int part_blocks;   // most blocks one partial covers (0 = balanced share)
   float scale_log2;  // scale * log2(e)
   int* counters;     // [num_seqs * num_kv_heads] pieces finished, zero between calls
+  int* seq_start;    // [num_seqs + 1] first tile of each sequence (written for the merge pass)
+  int* heavy;        // [2]: items listed for the merge pass, merge CTAs done (zero between calls)
+  int* heavy_list;   // [num_seqs * num_kv_heads] (seq * Hkv + kv head) of those items
   float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
   float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
   int32_t* err_flag;
 };
 
+// A split (seq, kv head) whose pieces x G exceed this is merged by the
+// separate merge pass (many CTAs) instead of by one warp of the decode kernel.
+constexpr int kFuseMaxValues = 16;
+constexpr int kMergeThreads = 256;
+
 struct DecodeKernelInfo {
   const void* fn;   // the __global__ function
+  const void* merge_fn;  // the merge pass for the same element type / shape
   int warps;        // warps per CTA
   int depth;        // ring slots per warp
   int warp_bytes;   // dynamic shared memory per warp
 };
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);
+
+// Bytes at the start of a decode workspace that must be zero when a call
+// begins (the merge-pass header and the piece counters).
+size_t decode_zero_prefix_bytes(int num_seqs, int num_kv_heads);
 bool decode_kernel_f32(int head_dim, int group, DecodeKernelInfo* info);
 
 }  // namespace pa

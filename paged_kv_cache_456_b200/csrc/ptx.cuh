@@ -10,8 +10,12 @@ namespace pa {
 
 // A device-side wait gives up after this long (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
-// Hint passed to mbarrier.try_wait: the longest one poll may suspend the thread.
-constexpr uint32_t kSuspendHintNs = 20000u;
+// Hint passed to mbarrier.try_wait: the longest one poll may suspend the
+// thread (0: use the form without a hint).
+#ifndef PA_SUSPEND_HINT_NS
+#define PA_SUSPEND_HINT_NS 20000u
+#endif
+constexpr uint32_t kSuspendHintNs = PA_SUSPEND_HINT_NS;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -50,6 +54,16 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+  if (kSuspendHintNs == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+  }
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -81,6 +95,23 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
           dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// Ask the bulk-copy engine to bring `bytes` (multiple of 16, 16-byte aligned)
+// of global memory into L2 ahead of use; nothing is written anywhere else.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared, bypassing L1 (cp.async.cg).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Arrive on the mbarrier once all of this thread's earlier cp.async copies
+// have landed (the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 }  // namespace pa

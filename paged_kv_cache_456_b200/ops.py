@@ -13,7 +13,9 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+# PA_LIBRARY selects another build of the library (e.g. a tuning variant)
+_LIB_PATH = os.environ.get("PA_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libpa.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = range(5)
 PA_F32, PA_BF16 = 0, 1

@@ -321,31 +321,43 @@ def make_workload(rng: np.random.Generator, *, name: str, dtype: str,
         block_mapping_compact=bmap, refcount=alloc.refcount.copy())
 
 
-def build_workload(name: str, seed: Optional[int] = None) -> Workload:
-    """One of the five named workloads (see the module docstring)."""
+def build_workload(name: str, seed: Optional[int] = None,
+                   num_blocks: Optional[int] = None) -> Workload:
+    """One of the five named workloads (see the module docstring).
+
+    ``num_blocks`` overrides the pool size (the same lengths in a smaller or
+    larger shuffled pool; q, K and V are then drawn from a different point of
+    the stream), e.g. to keep a profiler's device footprint small."""
     idx = WORKLOAD_NAMES.index(name)
     rng = np.random.default_rng(idx + 1 if seed is None else seed)
+    return _build_named(name, rng, num_blocks)
+
+
+def _build_named(name: str, rng: np.random.Generator, pool: Optional[int]) -> Workload:
+    def n(default: int) -> int:
+        return default if pool is None else pool
+
     if name == "tiny":
         return make_workload(rng, name=name, dtype="f32", num_q_heads=4, num_kv_heads=4,
-                             head_dim=64, context_lens=[1, 15, 16, 33], num_blocks=16,
+                             head_dim=64, context_lens=[1, 15, 16, 33], num_blocks=n(16),
                              scale=1.0 / 8.0, new_token=True)
     if name == "7b":
         lens = exp_lengths(rng, 64)
         return make_workload(rng, name=name, dtype="bf16", num_q_heads=32, num_kv_heads=32,
-                             head_dim=128, context_lens=lens, num_blocks=20000, new_token=True)
+                             head_dim=128, context_lens=lens, num_blocks=n(20000), new_token=True)
     if name == "gqa70b":
         lens = exp_lengths(rng, 256)
         return make_workload(rng, name=name, dtype="bf16", num_q_heads=64, num_kv_heads=8,
-                             head_dim=128, context_lens=lens, num_blocks=40000)
+                             head_dim=128, context_lens=lens, num_blocks=n(40000))
     if name == "prefix_cow":
         suffix = np.floor(rng.exponential(300.0, size=128)).astype(np.int64)
         lens = (2048 + suffix).astype(np.int32)
         return make_workload(rng, name=name, dtype="bf16", num_q_heads=32, num_kv_heads=8,
-                             head_dim=128, context_lens=lens, num_blocks=4096,
+                             head_dim=128, context_lens=lens, num_blocks=n(4096),
                              prefix_tokens=2048, cow_count=64)
     if name == "long":
         return make_workload(rng, name=name, dtype="bf16", num_q_heads=32, num_kv_heads=8,
-                             head_dim=128, context_lens=[32768] * 8, num_blocks=16384,
+                             head_dim=128, context_lens=[32768] * 8, num_blocks=n(16384),
                              partition_size=512)
     raise KeyError(name)
 
