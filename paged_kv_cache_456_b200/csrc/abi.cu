@@ -78,7 +78,7 @@ struct DecodePlan {
   // workspace layout; everything before zero_bytes must be zero on entry
   size_t heavy_off = 0;      // [2] ints: merge-pass item count, merge CTAs done
   size_t list_off = 0;       // [S*Hkv] ints: items for the merge pass
-  size_t counters_off = 0;   // [S*Hkv] ints
+  size_t counters_off = 0;   // [S*Hkv*2] ints
   size_t zero_bytes = 0;
   size_t seq_start_off = 0;  // [S + 1] ints
   size_t o_off = 0;
@@ -142,15 +142,15 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   DeviceInfo dev;
   if ((st = device_info(&dev)) != PA_OK) return st;
   const size_t seq_bytes = round_up((2 * static_cast<size_t>(num_seqs) + 1) * sizeof(int), 16);
-  p->smem = static_cast<size_t>(p->kernel.warps) * p->kernel.warp_bytes + seq_bytes;
+  p->smem = static_cast<size_t>(p->kernel.cta_bytes) + seq_bytes;
   if (p->smem > static_cast<size_t>(dev.smem_optin)) return PA_ERR_UNSUPPORTED;
   int occ = 0;
   if ((st = occupancy(p->kernel, p->smem, &occ)) != PA_OK) return st;
   if (occ < 1) return PA_ERR_UNSUPPORTED;
   const long long resident = static_cast<long long>(dev.sms) * occ;
-  const long long by_work = (tiles_max + p->kernel.warps - 1) / p->kernel.warps;
+  const long long by_work = (tiles_max + p->kernel.workers - 1) / p->kernel.workers;
   p->grid = static_cast<int>(by_work < resident ? (by_work > 0 ? by_work : 1) : resident);
-  const long long workers = static_cast<long long>(p->grid) * p->kernel.warps;
+  const long long workers = static_cast<long long>(p->grid) * p->kernel.workers;
   long long ranges = workers;
   if (partition_size > 0) {
     const long long per = workers * (partition_size / pa::kBlockSize);
@@ -177,7 +177,7 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 }  // namespace
 
 size_t pa::decode_zero_prefix_bytes(int num_seqs, int num_kv_heads) {
-  return 2 * sizeof(int) + static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
+  return 2 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
 }
 
 extern "C" {
@@ -286,7 +286,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     return PA_ERR_CUDA;
   // merge pass for items split into many pieces, launched behind the decode
   // kernel with programmatic dependent launch (it waits for the decode grid)
-  int workers = p.grid * p.kernel.warps;
+  int workers = p.grid * p.kernel.workers;
   void* mparams[] = {&args, &workers};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.sms);

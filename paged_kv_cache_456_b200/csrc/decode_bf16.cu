@@ -1,17 +1,19 @@
 // decode_bf16.cu -- decode kernel instances with bf16 elements.
-// Ring depth and warps per CTA are chosen per shape so that two or more CTAs
-// fit in an SM's shared memory with several tiles in flight per warp.
+// Ring depth, warps per CTA and head split are chosen per shape so that three
+// CTAs (12 warps) fit an SM's registers and shared memory; a group of 8 query
+// heads is split over two warps that share one ring.
 #include "decode_kernel.cuh"
 
 namespace pa {
 
-template <int D, int G, int DEPTH, int WARPS>
+template <int D, int G, int HS, int DEPTH, int WARPS, int MIN_CTAS = 1>
 static bool fill(DecodeKernelInfo* info) {
-  info->fn = reinterpret_cast<const void*>(&paged_decode_kernel<__nv_bfloat16, D, G, DEPTH, WARPS>);
+  info->fn = reinterpret_cast<const void*>(&paged_decode_kernel<__nv_bfloat16, D, G, HS, DEPTH, WARPS, MIN_CTAS>);
   info->merge_fn = reinterpret_cast<const void*>(&paged_decode_merge_kernel<__nv_bfloat16, D, G>);
   info->warps = WARPS;
+  info->workers = WARPS / HS;
   info->depth = DEPTH;
-  info->warp_bytes = DecodeCfg<__nv_bfloat16, D, G, DEPTH, WARPS>::WARP_BYTES;
+  info->cta_bytes = DecodeCfg<__nv_bfloat16, D, G / HS, G, HS, DEPTH, WARPS>::CTA_BYTES;
   return true;
 }
 
@@ -20,7 +22,7 @@ static bool fill(DecodeKernelInfo* info) {
 #define PA_BF16_128_DEPTH 2
 #endif
 #ifndef PA_BF16_128_DEPTH_G8
-#define PA_BF16_128_DEPTH_G8 2
+#define PA_BF16_128_DEPTH_G8 3
 #endif
 #ifndef PA_BF16_128_WARPS
 #define PA_BF16_128_WARPS 4
@@ -29,14 +31,14 @@ static bool fill(DecodeKernelInfo* info) {
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info) {
   constexpr int kD = PA_BF16_128_DEPTH, kD8 = PA_BF16_128_DEPTH_G8, kW = PA_BF16_128_WARPS;
   switch (head_dim * 100 + group) {
-    case 6401: return fill<64, 1, 4, 4>(info);
-    case 6402: return fill<64, 2, 4, 4>(info);
-    case 6404: return fill<64, 4, 4, 4>(info);
-    case 6408: return fill<64, 8, 4, 4>(info);
-    case 12801: return fill<128, 1, kD, kW>(info);
-    case 12802: return fill<128, 2, kD, kW>(info);
-    case 12804: return fill<128, 4, kD, kW>(info);
-    case 12808: return fill<128, 8, kD8, kW>(info);
+    case 6401: return fill<64, 1, 1, 4, 4, 3>(info);
+    case 6402: return fill<64, 2, 1, 4, 4, 3>(info);
+    case 6404: return fill<64, 4, 1, 4, 4, 3>(info);
+    case 6408: return fill<64, 8, 2, 4, 4, 3>(info);
+    case 12801: return fill<128, 1, 1, kD, kW, 3>(info);
+    case 12802: return fill<128, 2, 1, kD, kW, 3>(info);
+    case 12804: return fill<128, 4, 1, kD, kW, 3>(info);
+    case 12808: return fill<128, 8, 2, kD8, kW, 3>(info);
     default: return false;
   }
 }

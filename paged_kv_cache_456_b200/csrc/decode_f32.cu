@@ -5,26 +5,27 @@
 
 namespace pa {
 
-template <int D, int G, int DEPTH, int WARPS>
+template <int D, int G, int HS, int DEPTH, int WARPS, int MIN_CTAS = 1>
 static bool fill(DecodeKernelInfo* info) {
-  info->fn = reinterpret_cast<const void*>(&paged_decode_kernel<float, D, G, DEPTH, WARPS>);
+  info->fn = reinterpret_cast<const void*>(&paged_decode_kernel<float, D, G, HS, DEPTH, WARPS, MIN_CTAS>);
   info->merge_fn = reinterpret_cast<const void*>(&paged_decode_merge_kernel<float, D, G>);
   info->warps = WARPS;
+  info->workers = WARPS / HS;
   info->depth = DEPTH;
-  info->warp_bytes = DecodeCfg<float, D, G, DEPTH, WARPS>::WARP_BYTES;
+  info->cta_bytes = DecodeCfg<float, D, G / HS, G, HS, DEPTH, WARPS>::CTA_BYTES;
   return true;
 }
 
 bool decode_kernel_f32(int head_dim, int group, DecodeKernelInfo* info) {
   switch (head_dim * 100 + group) {
-    case 6401: return fill<64, 1, 3, 4>(info);
-    case 6402: return fill<64, 2, 3, 4>(info);
-    case 6404: return fill<64, 4, 3, 4>(info);
-    case 6408: return fill<64, 8, 2, 4>(info);
-    case 12801: return fill<128, 1, 2, 2>(info);
-    case 12802: return fill<128, 2, 2, 2>(info);
-    case 12804: return fill<128, 4, 2, 2>(info);
-    case 12808: return fill<128, 8, 2, 2>(info);
+    case 6401: return fill<64, 1, 1, 3, 4, 3>(info);
+    case 6402: return fill<64, 2, 1, 3, 4>(info);
+    case 6404: return fill<64, 4, 1, 3, 4>(info);
+    case 6408: return fill<64, 8, 2, 2, 4>(info);
+    case 12801: return fill<128, 1, 1, 2, 2>(info);
+    case 12802: return fill<128, 2, 1, 2, 2>(info);
+    case 12804: return fill<128, 4, 1, 2, 2>(info);
+    case 12808: return fill<128, 8, 2, 2, 2>(info);
     default: return false;
   }
 }

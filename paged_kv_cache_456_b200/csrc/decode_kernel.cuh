@@ -44,7 +44,7 @@
 namespace pa {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kMaxOwnRanges = 32;  // range starts a warp keeps in shared memory
+constexpr int kMaxOwnRanges = 8;  // range starts a warp keeps in shared memory
 
 // -- element conversion ---------------------------------------------------------
 template <typename T>
@@ -86,20 +86,11 @@ struct Elem<__nv_bfloat16> {
   }
 };
 
-// How tiles reach shared memory: 0 = one bulk copy per K/V tile issued by
-// lane 0 (completion counted in bytes); 1 = every lane copies 16-byte pieces
-// with cp.async and arrives on the slot's mbarrier when its copies land.
-#ifndef PA_COPY_ENGINE
-#define PA_COPY_ENGINE 0
+// When the one-head path hands its ring slot back (see compute_tile).
+#ifndef PA_G1_RELEASE
+#define PA_G1_RELEASE 0
 #endif
-constexpr bool kLaneCopies = PA_COPY_ENGINE == 1;
-
-// Tiles ahead of the shared-memory ring that are prefetched into L2, so the
-// ring only has to cover L2 latency while DRAM sees a deep queue (0 = off).
-#ifndef PA_L2_PREFETCH
-#define PA_L2_PREFETCH 0
-#endif
-constexpr int kPrefetch = PA_L2_PREFETCH;
+constexpr int kG1Release = PA_G1_RELEASE;
 
 // -- the two inner loops, on packed fp32 pairs (sm_100 FFMA2) or scalar FMAs ---
 #ifndef PA_PACKED_FMA
@@ -162,7 +153,7 @@ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 // -- compile-time geometry --------------------------------------------------------
-template <typename T, int D, int G, int DEPTH, int WARPS>
+template <typename T, int D, int G, int GT, int HS, int DEPTH, int WARPS>
 struct DecodeCfg {
   static constexpr int EB = sizeof(T);
   static constexpr int ROW = D * EB;          // bytes of one token's row of one KV head
@@ -171,13 +162,16 @@ struct DecodeCfg {
   static constexpr int RPI = 32 / LPR;        // rows one warp instruction covers (row groups)
   static constexpr int RL = kBlockSize / RPI; // rows per lane per block
   static constexpr int TILE = kBlockSize * ROW;
-  static constexpr int QB = G * ROW;          // q rows of the G query heads
+  static constexpr int QB = GT * ROW;         // q rows of the whole group
   static constexpr int SLOT = 2 * TILE + QB;  // K tile, V tile, q
   static constexpr int XS = kBlockSize * G * 4;
   static constexpr int ALPHA = ((G * 4 + 15) / 16) * 16;
   static constexpr int BND = (kMaxOwnRanges + 1) * 8;
-  static constexpr int WARP_BYTES =
-      ((DEPTH * SLOT + XS + ALPHA + DEPTH * 8 + BND + 127) / 128) * 128;
+  static constexpr int AUX = XS + ALPHA + BND;        // per warp
+  static constexpr int BAR_OFF = DEPTH * SLOT;         // full[DEPTH], empty[DEPTH]
+  static constexpr int AUX_OFF = BAR_OFF + 2 * DEPTH * 8;
+  static constexpr int WORKER_BYTES = ((AUX_OFF + HS * AUX + 127) / 128) * 128;
+  static constexpr int CTA_BYTES = (WARPS / HS) * WORKER_BYTES;
   // QK is done CH rows at a time; V = CH*G partial dots are reduce-scattered
   // over the LPR lanes of a row, leaving NV finished logits per lane.
   static constexpr int CH = cmin(RL, LPR / G >= 1 ? LPR / G : 1);
@@ -192,7 +186,7 @@ struct DecodeCfg {
   static_assert(VEC * LPR == D, "head_dim must be a multiple of 16 bytes");
   static_assert(RPI * LPR == 32 && RL * RPI == kBlockSize, "bad lane geometry");
   static_assert(NCH * CH == RL, "bad chunking");
-  static_assert(32 % G == 0 && G <= 16, "group size");
+  static_assert(32 % G == 0 && G <= 16 && GT == G * HS, "group size");
 };
 
 // -- per-warp ranges of the global tile order ------------------------------------
@@ -314,22 +308,48 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[V]) {
   }
 }
 
-template <typename T, int D, int G, int DEPTH, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32)
+// One "worker" = HS warps that stream the same tiles through one ring and
+// split the query heads of the group between them (HS = 2 halves the
+// registers each warp needs when the group is large).  The first warp of a
+// worker (the leader) issues the copies; every warp waits on the slot's
+// "full" barrier and releases the slot on its "empty" barrier, which the
+// leader waits on (bounded) before refilling the slot.
+template <typename T, int D, int GT, int HS, int DEPTH, int WARPS, int MIN_CTAS>
+__global__ void __launch_bounds__(WARPS * 32, MIN_CTAS)
 paged_decode_kernel(const DecodeArgs a) {
-  using C = DecodeCfg<T, D, G, DEPTH, WARPS>;
+  constexpr int G = GT / HS;  // query heads handled by one warp
+  using C = DecodeCfg<T, D, G, GT, HS, DEPTH, WARPS>;
   using E = Elem<T>;
+  static_assert(WARPS % HS == 0, "warps per CTA must be a multiple of the head split");
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_wsum[WARPS];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const int half = warp % HS;      // which share of the heads this warp computes
+  const int hoff = half * G;       // first head (within the group) of that share
+  const bool leader = half == 0;
   const int S = a.num_seqs;
   const int Hkv = a.num_kv_heads;
   const int Hq = a.num_q_heads;
-  int* s_start = reinterpret_cast<int*>(smem + WARPS * C::WARP_BYTES);  // [S + 1]
-  int* s_len = s_start + S + 1;                                         // [S]
+  constexpr int WORKERS = WARPS / HS;
+  unsigned char* wkbase = smem + (warp / HS) * C::WORKER_BYTES;
+  unsigned char* aux = wkbase + C::AUX_OFF + half * C::AUX;
+  const uint32_t slot0 = smem_addr(wkbase);
+  const uint32_t full0 = smem_addr(wkbase + C::BAR_OFF);
+  const uint32_t empty0 = full0 + 8 * DEPTH;
+  int* s_start = reinterpret_cast<int*>(smem + WORKERS * C::WORKER_BYTES);  // [S + 1]
+  int* s_len = s_start + S + 1;                                              // [S]
+
+  if (leader && lane == 0) {
+#pragma unroll
+    for (int j = 0; j < DEPTH; ++j) {
+      mbar_init(full0 + 8 * j, 1);
+      mbar_init(empty0 + 8 * j, HS);
+    }
+    fence_barrier_init();
+  }
 
   // ---- prologue: block counts and their prefix sums, in tiles ----------------
   {
@@ -364,7 +384,7 @@ paged_decode_kernel(const DecodeArgs a) {
       run += (s_len[s] + kBlockSize - 1) / kBlockSize;
     }
     if (tid == 0) s_start[S] = total * Hkv;
-    __syncthreads();
+    __syncthreads();  // also publishes the barrier initialisation to the whole CTA
   }
 
   // ---- rows of empty or invalid sequences are zero --------------------------------
@@ -379,7 +399,7 @@ paged_decode_kernel(const DecodeArgs a) {
     for (int i = tid; i < Hq * C::ROW / 16; i += WARPS * 32) dst[i] = make_uint4(0, 0, 0, 0);
   }
 
-  // ---- this warp's share of the tiles -------------------------------------------
+  // ---- this worker's share of the tiles -------------------------------------------
   // the merge pass (launched after this kernel) may start its prologue now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (blockIdx.x == 0)
@@ -387,16 +407,14 @@ paged_decode_kernel(const DecodeArgs a) {
 
   const long long W = s_start[S];
   if (W == 0) return;
-  const long long NWK = static_cast<long long>(gridDim.x) * WARPS;
+  const long long NWK = static_cast<long long>(gridDim.x) * WORKERS;
   const Ranges rg = make_ranges(W, NWK, a.part_blocks);
-  const long long gw = static_cast<long long>(blockIdx.x) * WARPS + warp;
+  const long long gw = static_cast<long long>(blockIdx.x) * WORKERS + warp / HS;
   const long long r0 = gw * rg.R / NWK;
   const long long r1 = (gw + 1) * rg.R / NWK;
-  if (r0 >= r1) return;  // more warps than ranges
+  if (r0 >= r1) return;  // more workers than ranges
 
-  unsigned char* wbase = smem + warp * C::WARP_BYTES;
-  long long* bnd = reinterpret_cast<long long*>(wbase + DEPTH * C::SLOT + C::XS + C::ALPHA +
-                                                DEPTH * 8);
+  long long* bnd = reinterpret_cast<long long*>(aux + C::XS + C::ALPHA);
   OwnRanges own{bnd, r1 - r0 <= kMaxOwnRanges ? static_cast<int>(r1 - r0) : 0};
   long long lo, hi;
   if (own.n > 0) {
@@ -409,16 +427,8 @@ paged_decode_kernel(const DecodeArgs a) {
     hi = rg.start(r1);
   }
   const int nst = static_cast<int>(hi - lo);
-  const uint32_t slot0 = smem_addr(wbase);
-  float* xs = reinterpret_cast<float*>(wbase + DEPTH * C::SLOT);
-  float* alpha_s = reinterpret_cast<float*>(wbase + DEPTH * C::SLOT + C::XS);
-  const uint32_t bar0 = smem_addr(wbase + DEPTH * C::SLOT + C::XS + C::ALPHA);
-  if (lane == 0) {
-#pragma unroll
-    for (int j = 0; j < DEPTH; ++j) mbar_init(bar0 + 8 * j, kLaneCopies ? 32 : 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
+  float* xs = reinterpret_cast<float*>(aux);
+  float* alpha_s = reinterpret_cast<float*>(aux + C::XS);
 
   const int dl = lane % C::LPR;  // which 16 bytes of a row
   const int rgp = lane / C::LPR; // which row group
@@ -433,47 +443,17 @@ paged_decode_kernel(const DecodeArgs a) {
   StageDesc B = make_desc(lo + 32 + lane, hi, s_start, s_len, rg, own, a);
   int base = 0;
 
-  // Fill ring slot j % DEPTH with tile j: K and V rows, plus q on a piece start.
-  // L2 prefetch of tile j by the lane that holds its descriptor (j - base < 64)
-  auto prefetch = [&](int j) {
-    if (kPrefetch == 0 || j >= nst) return;
-    const int rel = j - base;
-    const StageDesc& e = rel < 32 ? A : B;
-    if (lane == (rel & 31) && !(e.meta & kBad)) {
-      const int kvh = e.meta & 0xffff;
-      const uint32_t bytes = static_cast<uint32_t>((e.meta >> 16) & 31) * C::ROW;
-      const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
-      bulk_prefetch_l2(static_cast<const char*>(a.k_cache) + off, bytes);
-      bulk_prefetch_l2(static_cast<const char*>(a.v_cache) + off, bytes);
-    }
-  };
-
-  auto issue = [&](int j) {
-    if (kPrefetch > 0) prefetch(j + kPrefetch);
+  // Leader: fill ring slot j % DEPTH with tile j (K and V rows, plus the q rows
+  // of all GT heads on a piece start), once every warp has released the slot.
+  auto issue = [&](int j) -> bool {
     const StageDesc e = pick_desc(A, B, j - base);
     const int slot = j % DEPTH;
-    const uint32_t bar = bar0 + 8 * slot;
-    if constexpr (kLaneCopies) {
-      if (!(e.meta & kBad)) {
-        const int kvh = e.meta & 0xffff;
-        const int rows = (e.meta >> 16) & 31;
-        const uint32_t dst = slot0 + slot * C::SLOT;
-        const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
-        const char* ks = static_cast<const char*>(a.k_cache) + off;
-        const char* vs = static_cast<const char*>(a.v_cache) + off;
-        const int chunks = rows * (C::ROW / 16);
-        for (int c = lane; c < chunks; c += 32) {
-          cp_async_16(dst + 16 * c, ks + 16 * c);
-          cp_async_16(dst + C::TILE + 16 * c, vs + 16 * c);
-        }
-        if (e.meta & kFirst) {
-          const char* qs = static_cast<const char*>(a.q) +
-                           (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * G) * C::ROW;
-          for (int c = lane; c < C::QB / 16; c += 32) cp_async_16(dst + 2 * C::TILE + 16 * c, qs + 16 * c);
-        }
-      }
-      cp_async_mbar_arrive(bar);
-    } else if (lane == 0) {
+    if (HS > 1 && j >= DEPTH) {
+      if (!__all_sync(kFull, mbar_wait_bounded(empty0 + 8 * slot, ((j / DEPTH) - 1) & 1)))
+        return false;
+    }
+    if (lane == 0) {
+      const uint32_t bar = full0 + 8 * slot;
       if (e.meta & kBad) {
         mbar_arrive(bar);  // nothing to fetch; complete the phase
       } else {
@@ -490,16 +470,24 @@ paged_decode_kernel(const DecodeArgs a) {
         if (with_q)
           bulk_copy_g2s(dst + 2 * C::TILE,
                         static_cast<const char*>(a.q) +
-                            (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * G) *
+                            (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * GT) *
                                 C::ROW,
                         C::QB, bar);
       }
     }
+    return true;
   };
 
-  static_assert(kPrefetch + DEPTH < 32, "prefetch distance must stay within two batches");
-  for (int j = DEPTH; j < DEPTH + kPrefetch && j < kPrefetch; ++j) prefetch(j);
-  for (int j = 0; j < DEPTH && j < nst; ++j) issue(j);
+  // A bounded wait ran out: flag it, let this warp's copies in flight land, leave.
+  auto bail_out = [&](int k) {
+    if (lane == 0 && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
+    if (leader)
+      for (int j = k; j < nst && j < k + DEPTH; ++j)
+        mbar_wait_bounded(full0 + 8 * (j % DEPTH), (j / DEPTH) & 1);
+  };
+
+  if (leader)
+    for (int j = 0; j < DEPTH && j < nst; ++j) issue(j);
 
   float qv[G][C::VEC];
   float o[G][C::VEC];
@@ -509,18 +497,14 @@ paged_decode_kernel(const DecodeArgs a) {
   for (int k = 0; k < nst; ++k) {
     const StageDesc d = pick_desc(A, B, k - base);
     const int slot = k % DEPTH;
-    const bool ok = mbar_wait_bounded(bar0 + 8 * slot, (k / DEPTH) & 1);
-    if (!__all_sync(kFull, ok)) {
-      if (lane == 0 && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
-      // let copies already in flight land before the warp leaves
-      for (int j = k; j < nst && j < k + DEPTH; ++j)
-        mbar_wait_bounded(bar0 + 8 * (j % DEPTH), (j / DEPTH) & 1);
+    if (!__all_sync(kFull, mbar_wait_bounded(full0 + 8 * slot, (k / DEPTH) & 1))) {
+      bail_out(k);
       return;
     }
     const int flags = d.meta;
     const int kvh = d.meta & 0xffff;
     const int rows = (d.meta >> 16) & 31;
-    const unsigned char* pk = wbase + slot * C::SLOT;
+    const unsigned char* pk = wkbase + slot * C::SLOT;
     const unsigned char* pv = pk + C::TILE;
 
     if (flags & kFirst) {
@@ -528,7 +512,7 @@ paged_decode_kernel(const DecodeArgs a) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         // one head keeps the natural order; more heads are permuted (see reduce_scatter)
-        const int hq = G == 1 ? h : (h ^ hmask);
+        const int hq = hoff + (G == 1 ? h : (h ^ hmask));
         const uint4 raw = *reinterpret_cast<const uint4*>(pq + hq * C::ROW + dl * 16);
         E::unpack(raw, qv[h]);
 #pragma unroll
@@ -542,12 +526,36 @@ paged_decode_kernel(const DecodeArgs a) {
       poisoned = false;
     }
 
-    // One tile: MASK = the tile has fewer than 16 live rows (only the last
-    // tile of a sequence); full tiles take the branch-free path.
+    // Hand the slot back (this warp has read what it needs) and, on the leader,
+    // refill it with tile k + DEPTH.  Called exactly once per tile: by the
+    // one-head path as soon as its rows are in registers, otherwise after the tile.
+    bool refill_ok = true;
+    auto release = [&]() {
+      __syncwarp();
+      if (HS > 1 && lane == 0) mbar_arrive(empty0 + 8 * slot);
+      if (leader && k + DEPTH < nst) refill_ok = issue(k + DEPTH);
+    };
+
     auto compute_tile = [&](auto mask_tag) {
       constexpr bool MASK = decltype(mask_tag)::value;
       if constexpr (G == 1) {
-        // ---- one query head: every lane keeps the logits of its row group ----
+        // ---- one query head.  kG1Release: 2 = the lane's K and V rows go to
+        // registers first and the slot is refilled before any arithmetic; 1 = V
+        // goes to registers and the slot is refilled after QK; 0 = after the tile.
+        uint4 kr[C::RL], vr[C::RL];
+        if constexpr (kG1Release >= 1) {
+#pragma unroll
+          for (int i = 0; i < C::RL; ++i) {
+            const int row = i * C::RPI + rgp;
+            if (!MASK || row < rows) {
+              if constexpr (kG1Release == 2)
+                kr[i] = *reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16);
+              vr[i] = *reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16);
+            }
+          }
+        }
+        if constexpr (kG1Release == 2) release();
+        // every lane keeps the logits of its row group
         float x[C::RL];
 #pragma unroll
         for (int i = 0; i < C::RL; ++i) {
@@ -555,10 +563,14 @@ paged_decode_kernel(const DecodeArgs a) {
           x[i] = 0.f;
           if (!MASK || row < rows) {
             float kf[C::VEC];
-            E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
+            if constexpr (kG1Release == 2)
+              E::unpack(kr[i], kf);
+            else
+              E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
             x[i] = dot_vec<C::VEC>(qv[0], kf);
           }
         }
+        if constexpr (kG1Release == 1) release();
 #pragma unroll
         for (int off = C::LPR / 2; off >= 1; off >>= 1)
 #pragma unroll
@@ -584,7 +596,10 @@ paged_decode_kernel(const DecodeArgs a) {
           l_run += p;
           if (!MASK || row < rows) {
             float vf[C::VEC];
-            E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
+            if constexpr (kG1Release >= 1)
+              E::unpack(vr[i], vf);
+            else
+              E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
             axpy_vec<C::VEC>(p, vf, o[0]);
           }
         }
@@ -678,8 +693,16 @@ paged_decode_kernel(const DecodeArgs a) {
     } else {
       compute_tile(std::true_type{});
     }
-    __syncwarp();
-    if (k + DEPTH < nst) issue(k + DEPTH);
+    // the one-head path may have released the slot inside compute_tile already
+    if (G > 1 || kG1Release == 0 || (flags & kBad)) {
+      __syncwarp();
+      if (HS > 1 && lane == 0) mbar_arrive(empty0 + 8 * slot);
+      if (leader && k + DEPTH < nst) refill_ok = issue(k + DEPTH);
+    }
+    if (!refill_ok) {
+      bail_out(k + 1);
+      return;
+    }
 
     // ---- end of a piece: write the output or a partial -------------------------
     if (flags & kLast) {
@@ -701,7 +724,8 @@ paged_decode_kernel(const DecodeArgs a) {
       const long long item_a = s_start[s] + static_cast<long long>(kvh) * nb;
       const long long ra = rg.of(item_a);
       const long long rb = rg.of(item_a + nb - 1);
-      const size_t orow = (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D;
+      const size_t orow =
+          (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * GT + hoff) * D;
       if (ra == rb) {
         // the whole (seq, kv head) was this piece: normalise and store
 #pragma unroll
@@ -718,7 +742,7 @@ paged_decode_kernel(const DecodeArgs a) {
       } else {
         const long long r = rg.of(lo + k);
         const long long sl = piece_slot(rg, r, item_a);
-        float* wo = a.ws_o + sl * G * D;
+        float* wo = a.ws_o + (sl * GT + hoff) * D;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           if (h % C::RPI != rgp) continue;
@@ -727,11 +751,11 @@ paged_decode_kernel(const DecodeArgs a) {
             *reinterpret_cast<float4*>(wo + h * D + dl * C::VEC + e) =
                 make_float4(o[h][e], o[h][e + 1], o[h][e + 2], o[h][e + 3]);
         }
-        if (lane < G) a.ws_ml[sl * G + lane] = make_float2(m_run, bad ? -1.f : lsum);
+        if (lane < G) a.ws_ml[sl * GT + hoff + lane] = make_float2(m_run, bad ? -1.f : lsum);
         const bool heavy = (rb - ra + 1) * G > kFuseMaxValues;
         if (heavy) {
           // many pieces: the merge pass combines them; the first piece lists the item
-          if (r == ra && lane == 0) {
+          if (r == ra && lane == 0 && half == 0) {
             const int idx = atomicAdd(a.heavy, 1);
             a.heavy_list[idx] = s * Hkv + kvh;
           }
@@ -739,7 +763,7 @@ paged_decode_kernel(const DecodeArgs a) {
           __threadfence();
           __syncwarp();
           int prev = 0;
-          int* cnt = a.counters + static_cast<size_t>(s) * Hkv + kvh;
+          int* cnt = a.counters + (static_cast<size_t>(s) * Hkv + kvh) * 2 + half;
           if (lane == 0) prev = atomicAdd(cnt, 1);
           prev = __shfl_sync(kFull, prev, 0);
           if (prev == static_cast<int>(rb - ra)) {
@@ -752,7 +776,7 @@ paged_decode_kernel(const DecodeArgs a) {
               bool any_bad = false;
               for (long long rr = ra; rr <= rb; ++rr) {
                 const long long ss = piece_slot(rg, rr, item_a);
-                const float2 ml = __ldcg(a.ws_ml + ss * G + h);
+                const float2 ml = __ldcg(a.ws_ml + ss * GT + hoff + h);
                 any_bad |= ml.y < 0.f;
                 M = fmaxf(M, ml.x);
               }
@@ -762,10 +786,10 @@ paged_decode_kernel(const DecodeArgs a) {
               for (int e = 0; e < C::VEC; ++e) acc[e] = 0.f;
               for (long long rr = ra; rr <= rb; ++rr) {
                 const long long ss = piece_slot(rg, rr, item_a);
-                const float2 ml = __ldcg(a.ws_ml + ss * G + h);
+                const float2 ml = __ldcg(a.ws_ml + ss * GT + hoff + h);
                 const float w = exp2f(ml.x - M);
                 L += w * ml.y;
-                const float* po = a.ws_o + ss * G * D + h * D + dl * C::VEC;
+                const float* po = a.ws_o + (ss * GT + hoff + h) * D + dl * C::VEC;
 #pragma unroll
                 for (int e = 0; e < C::VEC; e += 4) {
                   const float4 t4 = __ldcg(reinterpret_cast<const float4*>(po + e));

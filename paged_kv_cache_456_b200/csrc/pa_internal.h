@@ -31,7 +31,8 @@ struct DecodeArgs {
   int len_cap;       // longest valid context: min(max_context_len, max_blocks_per_seq * 16)
   int part_blocks;   // most blocks one partial covers (0 = balanced share)
   float scale_log2;  // scale * log2(e)
-  int* counters;     // [num_seqs * num_kv_heads] pieces finished, zero between calls
+  int* counters;     // [num_seqs * num_kv_heads * 2] pieces finished per (item, head half),
+                     // zero between calls
   int* seq_start;    // [num_seqs + 1] first tile of each sequence (written for the merge pass)
   int* heavy;        // [2]: items listed for the merge pass, merge CTAs done (zero between calls)
   int* heavy_list;   // [num_seqs * num_kv_heads] (seq * Hkv + kv head) of those items
@@ -49,8 +50,9 @@ struct DecodeKernelInfo {
   const void* fn;   // the __global__ function
   const void* merge_fn;  // the merge pass for the same element type / shape
   int warps;        // warps per CTA
-  int depth;        // ring slots per warp
-  int warp_bytes;   // dynamic shared memory per warp
+  int workers;      // work streams per CTA (warps / head split)
+  int depth;        // ring slots per worker
+  int cta_bytes;    // dynamic shared memory per CTA, without the per-sequence arrays
 };
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);

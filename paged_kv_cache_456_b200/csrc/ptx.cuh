@@ -97,21 +97,4 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       : "memory");
 }
 
-// Ask the bulk-copy engine to bring `bytes` (multiple of 16, 16-byte aligned)
-// of global memory into L2 ahead of use; nothing is written anywhere else.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// 16-byte asynchronous copy global -> shared, bypassing L1 (cp.async.cg).
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-// Arrive on the mbarrier once all of this thread's earlier cp.async copies
-// have landed (the arrival counts against the barrier's expected count).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
 }  // namespace pa
