@@ -76,7 +76,7 @@ struct DecodePlan {
   long long ranges = 0;      // most ranges the device can form
   int sms = 0;
   // workspace layout; everything before zero_bytes must be zero on entry
-  size_t heavy_off = 0;      // [2] ints: merge-pass item count, merge CTAs done
+  size_t heavy_off = 0;      // [4] ints: merge-pass items, merge CTAs done, chunks, workers done
   size_t list_off = 0;       // [S*Hkv] ints: items for the merge pass
   size_t counters_off = 0;   // [S*Hkv*2] ints
   size_t zero_bytes = 0;
@@ -151,6 +151,7 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   const long long by_work = (tiles_max + p->kernel.workers - 1) / p->kernel.workers;
   p->grid = static_cast<int>(by_work < resident ? (by_work > 0 ? by_work : 1) : resident);
   const long long workers = static_cast<long long>(p->grid) * p->kernel.workers;
+  // static ranges (at most) plus tail chunks (at most), as the kernel cuts them
   long long ranges = workers;
   if (partition_size > 0) {
     const long long per = workers * (partition_size / pa::kBlockSize);
@@ -158,13 +159,15 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     ranges = workers * (rounds > 1 ? rounds : 1);
   }
   if (ranges > tiles_max) ranges = tiles_max > 0 ? tiles_max : 1;
+  const long long cs = pa::chunk_tiles(partition_size / pa::kBlockSize);
+  ranges += (pa::tail_tiles(tiles_max, workers) + cs - 1) / cs + 1;
   p->ranges = ranges;
   p->sms = dev.sms;
   const size_t slots = 2 * static_cast<size_t>(ranges);
   const size_t items = static_cast<size_t>(num_seqs) * num_kv_heads;
   // zero-on-entry fields first: the merge pass's count/done pair, the piece counters
   p->heavy_off = 0;
-  p->counters_off = 2 * sizeof(int);
+  p->counters_off = 4 * sizeof(int);
   p->zero_bytes = pa::decode_zero_prefix_bytes(num_seqs, num_kv_heads);
   p->list_off = p->zero_bytes;
   p->seq_start_off = round_up(p->list_off + items * sizeof(int), 16);
@@ -177,7 +180,7 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 }  // namespace
 
 size_t pa::decode_zero_prefix_bytes(int num_seqs, int num_kv_heads) {
-  return 2 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
+  return 4 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
 }
 
 extern "C" {

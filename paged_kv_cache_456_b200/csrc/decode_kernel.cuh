@@ -44,7 +44,7 @@
 namespace pa {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kMaxOwnRanges = 8;  // range starts a warp keeps in shared memory
+constexpr int kMaxOwnRanges = 4;  // range starts a warp keeps in shared memory
 
 // -- element conversion ---------------------------------------------------------
 template <typename T>
@@ -169,7 +169,8 @@ struct DecodeCfg {
   static constexpr int BND = (kMaxOwnRanges + 1) * 8;
   static constexpr int AUX = XS + ALPHA + BND;        // per warp
   static constexpr int BAR_OFF = DEPTH * SLOT;         // full[DEPTH], empty[DEPTH]
-  static constexpr int AUX_OFF = BAR_OFF + 2 * DEPTH * 8;
+  static constexpr int DESC_OFF = BAR_OFF + 2 * DEPTH * 8;  // one descriptor per slot
+  static constexpr int AUX_OFF = DESC_OFF + DEPTH * 16;
   static constexpr int WORKER_BYTES = ((AUX_OFF + HS * AUX + 127) / 128) * 128;
   static constexpr int CTA_BYTES = (WARPS / HS) * WORKER_BYTES;
   // QK is done CH rows at a time; V = CH*G partial dots are reduce-scattered
@@ -191,12 +192,22 @@ struct DecodeCfg {
 
 // -- per-warp ranges of the global tile order ------------------------------------
 struct Ranges {
-  long long W;  // tiles in total
-  long long R;  // ranges (each non-empty: R <= W)
-  __device__ __forceinline__ long long start(long long r) const { return r * W / R; }
-  __device__ __forceinline__ long long of(long long x) const { return ((x + 1) * R - 1) / W; }
+  long long W;   // tiles in total
+  long long Ws;  // the static part [0, Ws) is cut into Rs ranges, one or more per worker
+  long long Rs;
+  long long CS;  // the rest [Ws, W) is cut into chunks of CS tiles, claimed at run time
+  long long R;   // all ranges: Rs static + ceil((W - Ws) / CS) chunks
+  __device__ __forceinline__ long long start(long long r) const {
+    if (r <= Rs) return Rs ? r * Ws / Rs : 0;
+    const long long x = Ws + (r - Rs) * CS;
+    return x < W ? x : W;
+  }
+  __device__ __forceinline__ long long of(long long x) const {
+    return x < Ws ? ((x + 1) * Rs - 1) / Ws : Rs + (x - Ws) / CS;
+  }
   __device__ __forceinline__ bool is_start(long long x) const {
-    return x <= 0 || x >= W || start(of(x)) == x;
+    if (x <= 0 || x >= W) return true;
+    return x < Ws ? start(of(x)) == x : (x - Ws) % CS == 0;
   }
 };
 
@@ -206,7 +217,7 @@ struct OwnRanges {
   const long long* b;  // b[0] = first tile of the warp ... b[n] = one past its last
   int n;               // ranges owned; 0 = more than kMaxOwnRanges (fall back to division)
   __device__ __forceinline__ bool is_start(long long x, const Ranges& rg) const {
-    if (n == 0) return rg.is_start(x);
+    if (n == 0 || x < b[0] || x > b[n]) return rg.is_start(x);
     int l = 0, u = n;
     while (l < u) {
       const int m = (l + u) >> 1;
@@ -216,16 +227,25 @@ struct OwnRanges {
   }
 };
 
-// The cut of W tiles over `workers` warps: one range per warp, or more so
-// that no range exceeds part_blocks tiles (part_blocks = 0: no bound).
+// The cut of W tiles: the first part into static ranges (one per worker, or
+// more so that none exceeds part_blocks tiles), the last part (tail_tiles)
+// into chunks of chunk_tiles that workers claim as they run out of static
+// work, so that slower SMs end up with less of it.
+constexpr int kClaimAhead = 4;  // positions the leader keeps assigned beyond its refill point
+
 __device__ __forceinline__ Ranges make_ranges(long long W, long long workers, int part_blocks) {
-  long long R = workers;
+  Ranges rg;
+  rg.W = W;
+  rg.CS = chunk_tiles(part_blocks);
+  rg.Ws = W - tail_tiles(W, workers);
+  long long Rs = workers;
   if (part_blocks > 0) {
     const long long per = workers * part_blocks;
-    R = workers * max(1LL, (W + per - 1) / per);
+    Rs = workers * max(1LL, (rg.Ws + per - 1) / per);
   }
-  if (R > W) R = W;
-  return Ranges{W, R};
+  rg.Rs = Rs < rg.Ws ? Rs : rg.Ws;
+  rg.R = rg.Rs + (W - rg.Ws + rg.CS - 1) / rg.CS;
+  return rg;
 }
 
 // Partial-result slot of the piece of item [item_a, ...) that lies in range r.
@@ -234,19 +254,21 @@ __device__ __forceinline__ long long piece_slot(const Ranges& rg, long long r, l
 }
 
 // One tile of a warp's stream, as 3 words (kept one per lane, 32 tiles per batch).
-struct StageDesc {
+struct __align__(16) StageDesc {
   int phys;  // physical block id (0 if bad)
   int seq;
   int meta;  // kv head (bits 0-15) | live rows (16-20) | flags
+  int g;     // tile index in the global order
 };
 constexpr int kFirst = 1 << 24;  // first tile of a piece: reset state, fetch q
 constexpr int kLast = 1 << 25;   // last tile of a piece: finish it
 constexpr int kBad = 1 << 26;    // block-table entry out of range
+constexpr int kEnd = 1 << 27;    // no more tiles: the partner warp stops
 
 __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
                                                const int* s_len, const Ranges& rg,
                                                const OwnRanges& own, const DecodeArgs& a) {
-  StageDesc d{0, 0, 0};
+  StageDesc d{0, 0, 0, 0};
   if (g >= hi) return d;
   // largest s with s_start[s] <= g (sequences without blocks share their start)
   int lo = 0, up = a.num_seqs - 1;
@@ -274,6 +296,7 @@ __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const 
   d.phys = phys;
   d.seq = s;
   d.meta = kvh | (rows << 16) | flags;
+  d.g = static_cast<int>(g);
   return d;
 }
 
@@ -284,6 +307,7 @@ __device__ __forceinline__ StageDesc pick_desc(const StageDesc& A, const StageDe
   d.phys = __shfl_sync(kFull, in_a ? A.phys : B.phys, src);
   d.seq = __shfl_sync(kFull, in_a ? A.seq : B.seq, src);
   d.meta = __shfl_sync(kFull, in_a ? A.meta : B.meta, src);
+  d.g = __shfl_sync(kFull, in_a ? A.g : B.g, src);
   return d;
 }
 
@@ -410,9 +434,8 @@ paged_decode_kernel(const DecodeArgs a) {
   const long long NWK = static_cast<long long>(gridDim.x) * WORKERS;
   const Ranges rg = make_ranges(W, NWK, a.part_blocks);
   const long long gw = static_cast<long long>(blockIdx.x) * WORKERS + warp / HS;
-  const long long r0 = gw * rg.R / NWK;
-  const long long r1 = (gw + 1) * rg.R / NWK;
-  if (r0 >= r1) return;  // more workers than ranges
+  const long long r0 = gw * rg.Rs / NWK;  // this worker's static ranges [r0, r1)
+  const long long r1 = (gw + 1) * rg.Rs / NWK;
 
   long long* bnd = reinterpret_cast<long long*>(aux + C::XS + C::ALPHA);
   OwnRanges own{bnd, r1 - r0 <= kMaxOwnRanges ? static_cast<int>(r1 - r0) : 0};
@@ -426,9 +449,9 @@ paged_decode_kernel(const DecodeArgs a) {
     lo = rg.start(r0);
     hi = rg.start(r1);
   }
-  const int nst = static_cast<int>(hi - lo);
   float* xs = reinterpret_cast<float*>(aux);
   float* alpha_s = reinterpret_cast<float*>(aux + C::XS);
+  StageDesc* ring_desc = reinterpret_cast<StageDesc*>(wkbase + C::DESC_OFF);
 
   const int dl = lane % C::LPR;  // which 16 bytes of a row
   const int rgp = lane / C::LPR; // which row group
@@ -439,22 +462,55 @@ paged_decode_kernel(const DecodeArgs a) {
   const int imask = perm >> C::LG;
   const int hmask = perm & (G - 1);
 
-  StageDesc A = make_desc(lo + lane, hi, s_start, s_len, rg, own, a);
-  StageDesc B = make_desc(lo + 32 + lane, hi, s_start, s_len, rg, own, a);
+  // ---- the leader's stream: positions 0, 1, ... are its static tiles [lo, hi)
+  // followed by the chunks it claims; descriptors of positions [base, base+64)
+  // are held one per lane in A and B.
+  const int n0 = static_cast<int>(hi - lo);
+  int known = n0;                      // positions with a tile assigned
+  bool no_more = rg.R == rg.Rs;        // no chunks left to claim
+  auto static_desc = [&](int p) -> StageDesc {
+    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, rg, own, a) : StageDesc{0, 0, 0, 0};
+  };
+  StageDesc A{0, 0, 0, 0}, B{0, 0, 0, 0};
   int base = 0;
+  if (leader) {
+    A = static_desc(lane);
+    B = static_desc(32 + lane);
+  }
+  // claim the next chunk of the tail and give its tiles the next positions
+  auto claim = [&]() {
+    int c = 0;
+    if (lane == 0) c = atomicAdd(a.heavy + 2, 1);
+    c = __shfl_sync(kFull, c, 0);
+    if (c >= rg.R - rg.Rs) {
+      no_more = true;
+      return;
+    }
+    const long long g0 = rg.Ws + static_cast<long long>(c) * rg.CS;
+    const int len = static_cast<int>(rg.CS < W - g0 ? rg.CS : W - g0);
+    const int pa = base + lane, pb = base + 32 + lane;
+    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, rg, own, a);
+    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, rg, own, a);
+    known += len;
+  };
+  auto top_up = [&](int frontier) {
+    while (!no_more && known - frontier < kClaimAhead) claim();
+  };
 
   // Leader: fill ring slot j % DEPTH with tile j (K and V rows, plus the q rows
-  // of all GT heads on a piece start), once every warp has released the slot.
-  auto issue = [&](int j) -> bool {
-    const StageDesc e = pick_desc(A, B, j - base);
+  // of all GT heads on a piece start) -- or with the end marker -- once every
+  // warp has released the slot.  The slot's descriptor goes with it.
+  auto issue = [&](int j, bool end_marker) -> bool {
+    const StageDesc e = end_marker ? StageDesc{0, 0, kEnd, 0} : pick_desc(A, B, j - base);
     const int slot = j % DEPTH;
     if (HS > 1 && j >= DEPTH) {
       if (!__all_sync(kFull, mbar_wait_bounded(empty0 + 8 * slot, ((j / DEPTH) - 1) & 1)))
         return false;
     }
     if (lane == 0) {
+      ring_desc[slot] = e;
       const uint32_t bar = full0 + 8 * slot;
-      if (e.meta & kBad) {
+      if (e.meta & (kBad | kEnd)) {
         mbar_arrive(bar);  // nothing to fetch; complete the phase
       } else {
         const int kvh = e.meta & 0xffff;
@@ -477,30 +533,46 @@ paged_decode_kernel(const DecodeArgs a) {
     }
     return true;
   };
+  // Leader, after consuming position k: keep positions assigned ahead and
+  // refill the ring with position k + DEPTH (or the end marker, once).
+  auto advance = [&](int k) -> bool {
+    top_up(k + DEPTH + 1);
+    const int j = k + DEPTH;
+    if (j < known) return issue(j, false);
+    if (HS > 1 && j == known && no_more) return issue(j, true);
+    return true;
+  };
 
   // A bounded wait ran out: flag it, let this warp's copies in flight land, leave.
   auto bail_out = [&](int k) {
     if (lane == 0 && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
     if (leader)
-      for (int j = k; j < nst && j < k + DEPTH; ++j)
+      for (int j = k; j < known && j < k + DEPTH; ++j)
         mbar_wait_bounded(full0 + 8 * (j % DEPTH), (j / DEPTH) & 1);
   };
 
-  if (leader)
-    for (int j = 0; j < DEPTH && j < nst; ++j) issue(j);
+  if (leader) {
+    top_up(DEPTH);
+    for (int j = 0; j < DEPTH; ++j) {
+      if (j < known) issue(j, false);
+      else if (HS > 1 && j == known && no_more) issue(j, true);
+    }
+  }
 
   float qv[G][C::VEC];
   float o[G][C::VEC];
   float m_run = -INFINITY, l_run = 0.f;
   bool poisoned = false;
 
-  for (int k = 0; k < nst; ++k) {
-    const StageDesc d = pick_desc(A, B, k - base);
+  for (int k = 0;; ++k) {
+    if (leader && k >= known) break;  // (the partner warp stops at the end marker)
     const int slot = k % DEPTH;
     if (!__all_sync(kFull, mbar_wait_bounded(full0 + 8 * slot, (k / DEPTH) & 1))) {
       bail_out(k);
       return;
     }
+    const StageDesc d = ring_desc[slot];
+    if (d.meta & kEnd) break;
     const int flags = d.meta;
     const int kvh = d.meta & 0xffff;
     const int rows = (d.meta >> 16) & 31;
@@ -527,13 +599,13 @@ paged_decode_kernel(const DecodeArgs a) {
     }
 
     // Hand the slot back (this warp has read what it needs) and, on the leader,
-    // refill it with tile k + DEPTH.  Called exactly once per tile: by the
+    // refill it with position k + DEPTH.  Called exactly once per tile: by the
     // one-head path as soon as its rows are in registers, otherwise after the tile.
     bool refill_ok = true;
     auto release = [&]() {
       __syncwarp();
       if (HS > 1 && lane == 0) mbar_arrive(empty0 + 8 * slot);
-      if (leader && k + DEPTH < nst) refill_ok = issue(k + DEPTH);
+      if (leader) refill_ok = advance(k);
     };
 
     auto compute_tile = [&](auto mask_tag) {
@@ -694,11 +766,7 @@ paged_decode_kernel(const DecodeArgs a) {
       compute_tile(std::true_type{});
     }
     // the one-head path may have released the slot inside compute_tile already
-    if (G > 1 || kG1Release == 0 || (flags & kBad)) {
-      __syncwarp();
-      if (HS > 1 && lane == 0) mbar_arrive(empty0 + 8 * slot);
-      if (leader && k + DEPTH < nst) refill_ok = issue(k + DEPTH);
-    }
+    if (G > 1 || kG1Release == 0 || (flags & kBad)) release();
     if (!refill_ok) {
       bail_out(k + 1);
       return;
@@ -740,7 +808,7 @@ paged_decode_kernel(const DecodeArgs a) {
               E::pack(r);
         }
       } else {
-        const long long r = rg.of(lo + k);
+        const long long r = rg.of(d.g);
         const long long sl = piece_slot(rg, r, item_a);
         float* wo = a.ws_o + (sl * GT + hoff) * D;
 #pragma unroll
@@ -811,10 +879,17 @@ paged_decode_kernel(const DecodeArgs a) {
       }
     }
 
-    if (k - base == 31) {
+    if (leader && k - base == 31) {
       A = B;
       base += 32;
-      B = make_desc(lo + base + 32 + lane, hi, s_start, s_len, rg, own, a);
+      B = static_desc(base + 32 + lane);
+    }
+  }
+  // the last worker out resets the chunk counter for the next call
+  if (leader && lane == 0) {
+    if (atomicAdd(a.heavy + 3, 1) == static_cast<int>(NWK) - 1) {
+      a.heavy[2] = 0;
+      a.heavy[3] = 0;
     }
   }
 }

@@ -16,6 +16,25 @@ constexpr int kErrSlot = 4;
 constexpr int kErrPair = 8;
 constexpr int kErrTimeout = 16;
 
+// Work schedule: the last 1/kTailDiv of the tiles is handed out at run time
+// in chunks of kChunkTiles (0 = everything static).
+#ifndef PA_TAIL_DIV
+#define PA_TAIL_DIV 0
+#endif
+#ifndef PA_CHUNK_TILES
+#define PA_CHUNK_TILES 2
+#endif
+constexpr int kTailDiv = PA_TAIL_DIV;
+constexpr int kChunkTiles = PA_CHUNK_TILES;
+
+__host__ __device__ inline long long chunk_tiles(int part_blocks) {
+  return part_blocks > 0 && part_blocks < kChunkTiles ? part_blocks : kChunkTiles;
+}
+// tiles of the claimed tail; only used when every worker can get a chunk
+__host__ __device__ inline long long tail_tiles(long long W, long long workers) {
+  return (kTailDiv > 0 && W / kTailDiv >= workers) ? W / kTailDiv : 0;
+}
+
 struct DecodeArgs {
   void* out;
   const void* q;
@@ -34,7 +53,8 @@ struct DecodeArgs {
   int* counters;     // [num_seqs * num_kv_heads * 2] pieces finished per (item, head half),
                      // zero between calls
   int* seq_start;    // [num_seqs + 1] first tile of each sequence (written for the merge pass)
-  int* heavy;        // [2]: items listed for the merge pass, merge CTAs done (zero between calls)
+  int* heavy;        // [4]: items listed for the merge pass, merge CTAs done, tail chunks
+                     // claimed, decode workers done (all zero between calls)
   int* heavy_list;   // [num_seqs * num_kv_heads] (seq * Hkv + kv head) of those items
   float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
   float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
