@@ -51,6 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="7b")
     ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--append", choices=("fused", "separate"), default="fused",
+                    help="slot write of the new tokens fused into decode (one call) or as its "
+                         "own launch before it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=None)
     ap.add_argument("--num-blocks", type=int, default=None,
@@ -68,10 +71,16 @@ def measured_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the decode kernel's code with comments and blank space removed,
+    so that a comment edit does not orphan recorded counters."""
+    import re
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            code = f.read()
+        code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
+        code = re.sub(r"//[^\n]*", " ", code)
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 
@@ -89,8 +98,11 @@ def recorded_traffic(workload: str):
     return entry.get("dram_bytes_per_launch")
 
 
-def step_bytes(w) -> int:
-    return w.decode_bytes() + w.reshape_bytes() + w.copy_bytes()
+def step_bytes(w, fused: bool = False) -> int:
+    """Algorithmic bytes of one step.  Fused, the new rows are read once (as
+    decode's live tokens) and only their two cache writes add."""
+    append = w.append_bytes() if fused else w.reshape_bytes()
+    return w.decode_bytes() + append + w.copy_bytes()
 
 
 # ---------------------------------------------------------------------------
@@ -158,10 +170,11 @@ def sub_workload(w, k: int):
         slot_mapping_compact=None if w.slot_mapping_compact is None else w.slot_mapping_compact[:k])
 
 
-def oracle_sample(w, budget_s: float, repeat: bool = False):
+def oracle_sample(w, budget_s: float, repeat: bool = False, fused: bool = True):
     """Time the oracle's whole step on the first k sequences of the workload,
     k grown until one pass takes about budget_s (or all sequences are in);
     with ``repeat``, whole passes are then repeated until budget_s is spent.
+    Bytes follow the GPU arm's accounting (``fused``: see step_bytes).
     Returns (GB/s, seconds per pass, k, bytes per pass, threads)."""
     import oracle
 
@@ -180,7 +193,7 @@ def oracle_sample(w, budget_s: float, repeat: bool = False):
             oracle.workload_step(ws)
             passes += 1
         dt = (time.perf_counter() - t0) / passes
-    nbytes = step_bytes(ws)
+    nbytes = step_bytes(ws, fused)
     return nbytes / dt / 1e9, dt, k, nbytes, oracle.num_threads()
 
 
@@ -192,7 +205,8 @@ def run_reference(args, rank: int, world: int):
     w = build_workload(args.workload, seed=args.seed, num_blocks=args.num_blocks)
     steps, warm = args.steps, args.warmup
     per_step_budget = max(0.05, 150.0 / max(1, steps + warm))
-    _, dt, k, nbytes, threads = oracle_sample(w, per_step_budget)
+    _, dt, k, nbytes, threads = oracle_sample(w, per_step_budget,
+                                              fused=args.append == "fused")
     ws = sub_workload(w, k)
     for _ in range(warm):
         oracle.workload_step(ws)
@@ -254,19 +268,27 @@ def run_ours(args, rank: int, world: int):
     cfg = ops.launch_config(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
                             w.max_context_len, ps, tdt)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    launches_per_step = 1 + ("key" in t) + ("block_mapping" in t)
+    fused = "key" in t and args.append == "fused"
+    # decode is two kernels (the attention pass and the merge pass behind it)
+    launches_per_step = 2 + ("key" in t and not fused) + ("block_mapping" in t)
 
     def step(ev_mid=None):
         if "block_mapping" in t:
             ops.copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err_flag=err)
-        if "key" in t:
+        if "key" in t and not fused:
             ops.reshape_and_cache(t["key"], t["value"], t["k_cache"], t["v_cache"],
                                   t["slot_mapping"], err_flag=err)
         if ev_mid is not None:
             ev_mid.record(stream)
-        ops.decode(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                   t["context_lens"], scale=w.scale, max_context_len=w.max_context_len,
-                   workspace=ws, partition_size=ps, err_flag=err)
+        if fused:
+            ops.decode_append(t["out"], t["q"], t["key_seq"], t["value_seq"], t["k_cache"],
+                              t["v_cache"], t["block_tables"], t["context_lens"], scale=w.scale,
+                              max_context_len=w.max_context_len, workspace=ws,
+                              partition_size=ps, err_flag=err)
+        else:
+            ops.decode(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                       t["context_lens"], scale=w.scale, max_context_len=w.max_context_len,
+                       workspace=ws, partition_size=ps, err_flag=err)
 
     for _ in range(max(3, args.warmup)):
         flush.fill_(1)
@@ -296,7 +318,7 @@ def run_ours(args, rank: int, world: int):
         raise RuntimeError(f"device error flag {err.item()} during the benchmark")
 
     # end to end through the public API: pinned host inputs in, output back
-    e2e = end_to_end(w, t, ws, ps, dev, stream, K, args.warmup)
+    e2e = end_to_end(w, t, ws, ps, dev, stream, K, args.warmup, fused)
 
     total_t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -306,11 +328,12 @@ def run_ours(args, rank: int, world: int):
         e2e["ms"] = float(e2e_t.item())
     max_ms = float(total_t.item())
 
-    nbytes = step_bytes(w)
+    nbytes = step_bytes(w, fused)
     peak, peak_kind = measured_peaks()
     value = world * nbytes * K / (max_ms * 1e-3) / 1e9
     dec_avg = statistics.mean(dec_ms)
-    achieved = w.decode_bytes() / (dec_avg * 1e-3) / 1e9
+    dec_bytes = w.decode_bytes() + (w.append_bytes() if fused else 0)
+    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
     traffic = recorded_traffic(w.name)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -319,11 +342,12 @@ def run_ours(args, rank: int, world: int):
         w.dtype == "bf16" else "f32", "data": "synthetic", "config": workload_config(w),
         "pct_of_peak": round(100 * value / world / peak, 2),
         "seq_steps_per_s": round(world * w.num_seqs * K / (max_ms * 1e-3), 1),
+        "append": ("fused into decode" if fused else "separate launch") if "key" in t else "none",
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "kernel": "paged_decode_kernel",
                      "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
-                     "algorithmic_bytes_per_launch": w.decode_bytes(),
+                     "algorithmic_bytes_per_launch": dec_bytes,
                      "launch_ms_mean": round(dec_avg, 5),
                      "launch_ms_median": round(statistics.median(dec_ms), 5)},
         "e2e": {"value": round(world * nbytes * K / (e2e["ms"] * 1e-3) / 1e9, 2), "unit": "GB/s",
@@ -334,7 +358,7 @@ def run_ours(args, rank: int, world: int):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, dt, k, nb, threads = oracle_sample(w, budget_s=10.0, repeat=True)
+        gbs, dt, k, nb, threads = oracle_sample(w, budget_s=10.0, repeat=True, fused=fused)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
                                 "kind": "oracle",
                                 "sample": f"first {k} of {w.num_seqs} sequences of the {w.name} "
@@ -343,7 +367,7 @@ def run_ours(args, rank: int, world: int):
         print(json.dumps(line), flush=True)
 
 
-def end_to_end(w, t, ws, ps, dev, stream, K, warmup):
+def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused):
     """The step through the public API with the step's inputs in pinned host
     memory: H2D copies of q, the new K/V, slot ids, block tables and lengths,
     the kernels, and the D2H copy of the output, all inside the timed region.
@@ -351,8 +375,8 @@ def end_to_end(w, t, ws, ps, dev, stream, K, warmup):
     import torch
     from paged_kv_cache_456_b200 import ops
 
-    names = [n for n in ("q", "key", "value", "slot_mapping", "block_tables", "context_lens",
-                         "block_mapping") if n in t]
+    step_inputs = ("q", "key_seq", "value_seq") if fused else ("q", "key", "value", "slot_mapping")
+    names = [n for n in step_inputs + ("block_tables", "context_lens", "block_mapping") if n in t]
     host = {n: t[n].cpu().pin_memory() for n in names}
     out_h = torch.empty(t["out"].shape, dtype=t["out"].dtype).pin_memory()
     dv = {n: torch.empty_like(t[n]) for n in names}
@@ -368,9 +392,15 @@ def end_to_end(w, t, ws, ps, dev, stream, K, warmup):
         if "key" in dv:
             ops.reshape_and_cache(dv["key"], dv["value"], t["k_cache"], t["v_cache"],
                                   dv["slot_mapping"], err_flag=err)
-        ops.decode(t["out"], dv["q"], t["k_cache"], t["v_cache"], dv["block_tables"],
-                   dv["context_lens"], scale=w.scale, max_context_len=w.max_context_len,
-                   workspace=ws, partition_size=ps, err_flag=err)
+        if fused:
+            ops.decode_append(t["out"], dv["q"], dv["key_seq"], dv["value_seq"], t["k_cache"],
+                              t["v_cache"], dv["block_tables"], dv["context_lens"], scale=w.scale,
+                              max_context_len=w.max_context_len, workspace=ws,
+                              partition_size=ps, err_flag=err)
+        else:
+            ops.decode(t["out"], dv["q"], t["k_cache"], t["v_cache"], dv["block_tables"],
+                       dv["context_lens"], scale=w.scale, max_context_len=w.max_context_len,
+                       workspace=ws, partition_size=ps, err_flag=err)
         out_h.copy_(t["out"], non_blocking=True)
 
     for _ in range(max(3, warmup)):

@@ -3,14 +3,14 @@
  * B200 (sm_100a), with the two cache-maintenance operations that feed it.
  *
  * The key/value cache of every sequence is cut into fixed-size blocks of
- * block_size token slots (16, "typically 16 tokens per block"), and a
- * per-sequence block table maps the sequence's logical block j to a physical
- * block id in one shared pool (skandtandon.pages.dev day-9 post, section
- * "Idea 1: PagedAttention"; "What vLLM Is and Why It Exists", section "The
- * idea vLLM started from: pages").  The decode kernel reads a sequence's
- * cached keys and values "from blocks scattered anywhere in the tensor,
- * following the block table" (same section), so its result is ordinary
- * attention over the sequence's tokens.
+ * block_size token slots (16, the size the pages give as the usual one), and
+ * a per-sequence block table maps the sequence's logical block j to a
+ * physical block id in one shared pool (skandtandon.pages.dev day-9 post,
+ * section "Idea 1: PagedAttention"; "What vLLM Is and Why It Exists",
+ * section "The idea vLLM started from: pages").  The decode kernel finds
+ * each of a sequence's cached keys and values through the block table,
+ * wherever in the pool its block lies (same section), so its result is
+ * ordinary attention over the sequence's tokens.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -168,10 +168,10 @@ pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const
 /* ------------------------------------------------------------------------
  * Slot write (reshape_and_cache)
  * ------------------------------------------------------------------------
- * Writes each step's new key/value rows into the cache: the cache "grows ...
- * as the model generates new tokens" ("vLLM Solved the Wrong Bottleneck...",
- * section "Paged Attention"), one new token per request per step ("What vLLM
- * Is and Why It Exists", section "A picture").  For every token t and KV
+ * Writes each step's new key/value rows into the cache: the cache gets
+ * longer with every generated token ("vLLM Solved the Wrong Bottleneck...",
+ * section "Paged Attention"), and every request gains one token per step
+ * ("What vLLM Is and Why It Exists", section "A picture").  For every token t and KV
  * head h:
  *     slot = slot_mapping[t];  if slot < 0: skip (padding)
  *     k_cache[slot / block_size][h][slot % block_size][:] = key[t][h][:]
@@ -187,10 +187,47 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
                                pa_dtype dtype, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Fused slot write + decode attention
+ * ------------------------------------------------------------------------
+ * One decode step in one call: each sequence's newest key/value row (one new
+ * token per request per step, "What vLLM Is and Why It Exists", section "A
+ * picture"; the cache grows by that token, "vLLM Solved the Wrong
+ * Bottleneck...", section "Paged Attention") is written to its slot AND used
+ * by the attention of the same step.  For every sequence s with
+ * n = context_lens[s] >= 1 (n counts the new token) and KV head h, with
+ * slot = block_tables[s][(n-1) / block_size] * block_size + (n-1) % block_size:
+ *     k_cache[slot / block_size][h][slot % block_size][:] = key[s][h][:]
+ *     v_cache[...same...]                                 = value[s][h][:]
+ *     out[s] = pa_decode's result over positions 0..n-1
+ * The result is that of pa_reshape_and_cache with those slots followed by
+ * pa_decode, bit for bit: the kernel takes the newest row from key/value
+ * (not from the cache) and writes it back from shared memory, so the step
+ * costs one launch pair instead of two and never re-reads the row it wrote.
+ *
+ *   key, value  device, [num_seqs][num_kv_heads][head_dim], 16-byte aligned.
+ *   Every other argument, the workspace rule and the supported shapes are
+ *   pa_decode's.
+ * A sequence with n == 0 writes nothing and gets out = 0.  A sequence whose
+ * n is out of range (PA_ERRBIT_CONTEXT_LEN) or whose last block-table entry
+ * is out of range (PA_ERRBIT_BLOCK_ID) writes nothing.  The block receiving
+ * the new row must belong to that sequence alone (copy-on-write done
+ * beforehand, as pa_copy_blocks does): a block another sequence of the same
+ * call also reads races with the write.
+ */
+pa_status pa_decode_append(void *out, const void *q, const void *key, const void *value,
+                           void *k_cache, void *v_cache, const int32_t *block_tables,
+                           const int32_t *context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size,
+                           int max_blocks_per_seq, int num_blocks, int max_context_len,
+                           float scale, int partition_size, pa_dtype dtype, void *workspace,
+                           size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
  * Block copy-on-write (copy_blocks)
  * ------------------------------------------------------------------------
- * "When a shared block needs to diverge, only the changed block is copied"
- * (day-9 post, section "Idea 1: PagedAttention").  For each pair p of
+ * A block shared by several sequences is duplicated, alone, at the moment
+ * one of them must change it (day-9 post, section "Idea 1: PagedAttention",
+ * copy-on-write).  For each pair p of
  * block_mapping (int32 [num_pairs][2] = {src, dst}), the whole physical
  * block src -- all KV heads, all block_size slots -- is copied to dst, in
  * k_cache and in v_cache.  A bit-exact copy.  The dst ids must be distinct

@@ -7,11 +7,12 @@
  *
  * What it computes (each function cites the passage it follows):
  *
- *   Paged attention reads a request's cached keys and values "from blocks
- *   scattered anywhere in the tensor, following the block table" ("What vLLM
- *   Is and Why It Exists", section "The idea vLLM started from: pages"); it
- *   stores "continuous keys and values in non-contiguous memory space" ("vLLM
- *   Solved the Wrong Bottleneck...", section "Paged Attention").  Paging only
+ *   Paged attention looks up each cached key and value of a request through
+ *   its block table, whatever pool position the block holds ("What vLLM Is
+ *   and Why It Exists", section "The idea vLLM started from: pages"); keys
+ *   and values that are consecutive in the sequence need not be consecutive
+ *   in memory ("vLLM Solved the Wrong Bottleneck...", section "Paged
+ *   Attention").  Paging only
  *   changes where the bytes live, so the result is ordinary softmax
  *   attention of one query token over the n cached tokens, written here as
  *   its definition:
@@ -22,8 +23,8 @@
  *
  *   where token i of sequence s lives in physical block
  *   block_tables[s][i / block_size] at offset i % block_size (day-9 post,
- *   section "Idea 1: PagedAttention": "a block table maps logical blocks to
- *   physical GPU memory blocks").
+ *   section "Idea 1: PagedAttention": the block table takes a logical block
+ *   number to a physical block of GPU memory).
  *
  * Readings where the pages are silent (listed with the rest of the design):
  *   - cache layout [num_blocks][num_kv_heads][block_size][head_dim];
@@ -247,9 +248,9 @@ int oracle_paged_decode_partitioned(double *out, const void *q, const void *k_ca
 /*
  * Slot write: each step's new key/value of token t, for every KV head, goes
  * to the cache slot slot_mapping[t] = block * block_size + offset.  The cache
- * "grows ... as the model generates new tokens" ("vLLM Solved the Wrong
- * Bottleneck...", section "Paged Attention"), one new token per request per
- * step ("What vLLM Is and Why It Exists", section "A picture").  A pure byte
+ * gets longer with every generated token ("vLLM Solved the Wrong
+ * Bottleneck...", section "Paged Attention"), and every request gains one
+ * token per step ("What vLLM Is and Why It Exists", section "A picture").  A pure byte
  * copy: key/value are [num_tokens][num_kv_heads][head_dim].
  */
 int oracle_reshape_and_cache(void *k_cache, void *v_cache, const void *key, const void *value,
@@ -278,8 +279,8 @@ int oracle_reshape_and_cache(void *k_cache, void *v_cache, const void *key, cons
 }
 
 /*
- * Copy-on-write: "when a shared block needs to diverge, only the changed
- * block is copied" (day-9 post, section "Idea 1: PagedAttention").  For each
+ * Copy-on-write: a shared block is duplicated, alone, when one of its
+ * sharers must change it (day-9 post, section "Idea 1: PagedAttention").  For each
  * pair (src, dst) of block_mapping ([num_pairs][2]) the whole physical block
  * src (all KV heads, all slots) is copied to dst, in K and in V.
  */

@@ -14,7 +14,7 @@ of the GPU path (block tables, slot mappings and copy-on-write pairs).
   Solved the Wrong Bottleneck...", section "Paged Attention").
 * Physical blocks may sit anywhere in the pool; the free list is a random
   permutation so consecutive logical blocks land on scattered physical ones
-  (day-9 post, "Idea 1": blocks "can be scattered anywhere in memory").
+  (day-9 post, "Idea 1": a sequence's blocks need not be adjacent).
 * Two sequences with a common prefix share physical blocks, and a shared block
   that must diverge is copied alone (copy-on-write) (day-9 post, "Idea 1",
   bullets "Sharing" and "Copy-on-write").  The pages name no reference count;

@@ -231,12 +231,16 @@ pa_status pa_decode_launch_config(int num_seqs, int num_q_heads, int num_kv_head
   return PA_OK;
 }
 
-pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
-                    int partition_size, pa_dtype dtype, void* workspace, size_t workspace_bytes,
-                    int32_t* err_flag, void* stream) {
+namespace {
+
+// pa_decode and pa_decode_append: key/value null = plain decode.
+pa_status decode_impl(void* out, const void* q, const void* key, const void* value,
+                      const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_seqs, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                      int num_blocks, int max_context_len, float scale, int partition_size,
+                      pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                      int32_t* err_flag, void* stream) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -260,6 +264,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   pa::DecodeArgs args;
   args.out = out;
   args.q = q;
+  args.key = key;
+  args.value = value;
   args.k_cache = k_cache;
   args.v_cache = v_cache;
   args.block_tables = block_tables;
@@ -303,6 +309,35 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   cfg.numAttrs = 1;
   return cudaLaunchKernelExC(&cfg, p.kernel.merge_fn, mparams) == cudaSuccess ? PA_OK
                                                                                : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                    int partition_size, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    int32_t* err_flag, void* stream) {
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens,
+                     num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     max_blocks_per_seq, num_blocks, max_context_len, scale, partition_size,
+                     dtype, workspace, workspace_bytes, err_flag, stream);
+}
+
+pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value,
+                           void* k_cache, void* v_cache, const int32_t* block_tables,
+                           const int32_t* context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size,
+                           int max_blocks_per_seq, int num_blocks, int max_context_len,
+                           float scale, int partition_size, pa_dtype dtype, void* workspace,
+                           size_t workspace_bytes, int32_t* err_flag, void* stream) {
+  if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value)))
+    return PA_ERR_INVALID_ARG;
+  return decode_impl(out, q, key, value, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, max_context_len, scale, partition_size, dtype, workspace,
+                     workspace_bytes, err_flag, stream);
 }
 
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

@@ -2,32 +2,39 @@
 //
 // What it computes: for every sequence s and query head h, softmax attention
 // of q[s][h] over the context_lens[s] cached tokens, each token found through
-// the sequence's block table ("What vLLM Is and Why It Exists", section "The
-// idea vLLM started from: pages": attention reads a request's cache "from
-// blocks scattered anywhere in the tensor, following the block table").
+// the sequence's block table, wherever in the pool its block lies ("What vLLM
+// Is and Why It Exists", section "The idea vLLM started from: pages").
 //
 // How (B200 design):
 //  * Work unit = one (sequence, KV head, block) tile: 16 tokens x head_dim,
 //    contiguous in the cache, read once for all G = Hq/Hkv query heads that
 //    share the KV head.  All units are laid end to end in (seq, kv head,
-//    block) order and cut into equal contiguous ranges, one or more per warp
-//    of a persistent grid (as many CTAs as fit on the 148 SMs): every warp
-//    gets the same number of tiles however skewed the context lengths are.
-//  * Each warp streams its tiles through a private ring of DEPTH shared-memory
-//    slots with the 1-D bulk-copy engine (cp.async.bulk, one mbarrier per
-//    slot, completion counted in bytes).  Only the live rows of a partial last
-//    block are fetched.  Block-table entries for the next 32-64 tiles are
-//    loaded one per lane well ahead of use.
+//    block) order and cut into equal contiguous ranges, one or more per
+//    worker of a persistent grid (as many CTAs as fit on the 148 SMs): every
+//    worker gets the same number of tiles however skewed the lengths are.
+//    A worker is one warp, or HS = 2 warps that split the G query heads of
+//    a tile between them when G = 8.
+//  * Each worker streams its tiles through a ring of DEPTH shared-memory
+//    slots filled by its leader warp with the 1-D bulk-copy engine
+//    (cp.async.bulk, a "full" mbarrier per slot completed by byte count, an
+//    "empty" mbarrier per slot when two warps share it).  Only the live rows
+//    of a partial last block are fetched.  Block-table entries for the next
+//    32-64 tiles are loaded one per lane well ahead of use, and each slot's
+//    descriptor travels with it through shared memory.
+//  * Fused slot write (when key/value are given): the newest row of each
+//    (sequence, KV head) is fetched from key/value instead of the cache, and
+//    the leader writes it from shared memory to its cache slot.
 //  * Arithmetic is fp32 on the CUDA cores (a one-token query is a
 //    bandwidth-bound gather, not a dense contraction): lanes split head_dim
 //    16 bytes at a time, partial dot products are combined by a butterfly
 //    reduce-scatter of warp shuffles, the softmax is online (base 2, rescaled
 //    only when the running max grows by more than 2^8), and P.V accumulates
 //    in registers.
-//  * A sequence cut by a range boundary leaves partial results (m, l, o) in
-//    the workspace; the warp that finishes the last piece of a (seq, kv head)
-//    merges them by log-sum-exp and writes the output (a counter per (seq,
-//    kv head), no waiting, so nothing can hang).
+//  * A (seq, kv head) cut by a range boundary leaves partial results (m, l,
+//    o) in the workspace.  With few pieces, the warp that finishes the last
+//    piece merges them by log-sum-exp (a counter per item, no waiting, so
+//    nothing can hang); items with many pieces go to a list that a second,
+//    programmatically dependent kernel merges with all its threads.
 //  * Device-side index checks skip bad items and set err_flag bits; every
 //    wait is bounded.
 #pragma once
@@ -264,6 +271,7 @@ constexpr int kFirst = 1 << 24;  // first tile of a piece: reset state, fetch q
 constexpr int kLast = 1 << 25;   // last tile of a piece: finish it
 constexpr int kBad = 1 << 26;    // block-table entry out of range
 constexpr int kEnd = 1 << 27;    // no more tiles: the partner warp stops
+constexpr int kAppend = 1 << 28; // fused append: the tile's last live row is the new token
 
 __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
                                                const int* s_len, const Ranges& rg,
@@ -293,6 +301,7 @@ __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const 
     if (a.err_flag) atomicOr(a.err_flag, kErrBlockId);
   }
   const int rows = min(kBlockSize, n - blk * kBlockSize);
+  if (a.key && blk == nb - 1 && !(flags & kBad)) flags |= kAppend;
   d.phys = phys;
   d.seq = s;
   d.meta = kvh | (rows << 16) | flags;
@@ -521,8 +530,18 @@ paged_decode_kernel(const DecodeArgs a) {
         const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, 2 * kv_bytes + (with_q ? C::QB : 0));
-        bulk_copy_g2s(dst, static_cast<const char*>(a.k_cache) + off, kv_bytes, bar);
-        bulk_copy_g2s(dst + C::TILE, static_cast<const char*>(a.v_cache) + off, kv_bytes, bar);
+        // with a fused append the last live row comes from key/value, not the cache
+        const uint32_t cached = (e.meta & kAppend) ? kv_bytes - C::ROW : kv_bytes;
+        if (cached) {
+          bulk_copy_g2s(dst, static_cast<const char*>(a.k_cache) + off, cached, bar);
+          bulk_copy_g2s(dst + C::TILE, static_cast<const char*>(a.v_cache) + off, cached, bar);
+        }
+        if (e.meta & kAppend) {
+          const size_t src = (static_cast<size_t>(e.seq) * Hkv + kvh) * C::ROW;
+          bulk_copy_g2s(dst + cached, static_cast<const char*>(a.key) + src, C::ROW, bar);
+          bulk_copy_g2s(dst + C::TILE + cached, static_cast<const char*>(a.value) + src, C::ROW,
+                        bar);
+        }
         if (with_q)
           bulk_copy_g2s(dst + 2 * C::TILE,
                         static_cast<const char*>(a.q) +
@@ -573,6 +592,19 @@ paged_decode_kernel(const DecodeArgs a) {
     }
     const StageDesc d = ring_desc[slot];
     if (d.meta & kEnd) break;
+    if ((d.meta & kAppend) && leader) {
+      // fused append: the new token's row, now in shared memory, goes to its cache slot
+      const int nrow = ((d.meta >> 16) & 31) - 1;
+      const size_t off = (static_cast<size_t>(d.phys) * Hkv + (d.meta & 0xffff)) * C::TILE +
+                         static_cast<size_t>(nrow) * C::ROW;
+      const unsigned char* sk = wkbase + slot * C::SLOT + nrow * C::ROW;
+      for (int c = lane; c < C::ROW / 16; c += 32) {
+        *reinterpret_cast<uint4*>(static_cast<char*>(const_cast<void*>(a.k_cache)) + off + 16 * c) =
+            *reinterpret_cast<const uint4*>(sk + 16 * c);
+        *reinterpret_cast<uint4*>(static_cast<char*>(const_cast<void*>(a.v_cache)) + off + 16 * c) =
+            *reinterpret_cast<const uint4*>(sk + C::TILE + 16 * c);
+      }
+    }
     const int flags = d.meta;
     const int kvh = d.meta & 0xffff;
     const int rows = (d.meta >> 16) & 31;

@@ -38,6 +38,8 @@ __host__ __device__ inline long long tail_tiles(long long W, long long workers) 
 struct DecodeArgs {
   void* out;
   const void* q;
+  const void* key;    // fused append: [num_seqs][num_kv_heads][head_dim] newest token of each
+  const void* value;  // sequence (position context_lens[s] - 1), or null for plain decode
   const void* k_cache;
   const void* v_cache;
   const int32_t* block_tables;

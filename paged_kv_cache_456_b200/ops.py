@@ -27,8 +27,8 @@ ERRBIT_PAIR = 8
 ERRBIT_TIMEOUT = 16
 
 EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_init",
-            "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_reshape_and_cache",
-            "pa_copy_blocks")
+            "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_decode_append",
+            "pa_reshape_and_cache", "pa_copy_blocks")
 
 # size of the library's fixed scratch array used by pa_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -65,6 +65,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode.restype = i
     lib.pa_decode_noalloc.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, vp]
+    lib.pa_decode_append.restype = i
+    lib.pa_decode_append.argtypes = [vp] * 8 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode_noalloc.restype = i
     lib.pa_reshape_and_cache.argtypes = [vp] * 5 + [i] * 6 + [vp, vp]
     lib.pa_reshape_and_cache.restype = i
@@ -154,6 +156,24 @@ def decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
         S, Hq, Hkv, D, bs, block_tables.shape[1], N, int(max_context_len), float(scale),
         int(partition_size), _dtype_code(q), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream)), "pa_decode")
+    return out
+
+
+def decode_append(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor, value: torch.Tensor,
+                  k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                  context_lens: torch.Tensor, *, scale: float, max_context_len: int,
+                  workspace: torch.Tensor, partition_size: int = 0,
+                  err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Write each sequence's newest ``key``/``value`` row ``[S][Hkv][D]`` into its
+    cache slot and decode over it in the same launch; see ``pa_decode_append``."""
+    S, Hq, D = q.shape
+    N, Hkv, bs, _ = k_cache.shape
+    _check(library().pa_decode_append(
+        _ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        int(max_context_len), float(scale), int(partition_size), _dtype_code(q), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream)),
+        "pa_decode_append")
     return out
 
 

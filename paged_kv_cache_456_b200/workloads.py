@@ -182,6 +182,26 @@ class Workload:
         row = self.num_kv_heads * self.head_dim * self.elem_bytes
         return 4 * t * row + 8 * t   # key+value read, two cache writes, slot ids
 
+    def append_bytes(self) -> int:
+        """The slot write when it is fused into decode: the new rows are read
+        as part of decode_bytes' live tokens, so only the two cache writes add."""
+        if self.new_key is None:
+            return 0
+        return 2 * self.new_key.shape[0] * self.num_kv_heads * self.head_dim * self.elem_bytes
+
+    def new_rows_per_sequence(self):
+        """new_key/new_value as [num_seqs][Hkv][D] (zeros where context_lens
+        is 0), the layout of the fused slot write + decode."""
+        if self.new_key is None:
+            return None, None
+        live = np.nonzero(self.context_lens > 0)[0]
+        shape = (self.num_seqs, self.num_kv_heads, self.head_dim)
+        k = np.zeros(shape, dtype=self.new_key.dtype)
+        v = np.zeros(shape, dtype=self.new_value.dtype)
+        k[live] = self.new_key
+        v[live] = self.new_value
+        return k, v
+
     def copy_bytes(self) -> int:
         if self.block_mapping_compact is None:
             return 0
@@ -403,6 +423,9 @@ def upload(w: Workload, device="cuda", pool: bool = True):
         out["key"] = elems(w.new_key).to(device)
         out["value"] = elems(w.new_value).to(device)
         out["slot_mapping"] = torch.from_numpy(w.slot_mapping).to(device)
+        ks, vs = w.new_rows_per_sequence()
+        out["key_seq"] = elems(ks).to(device)
+        out["value_seq"] = elems(vs).to(device)
     if w.block_mapping_compact is not None:
         out["block_mapping"] = torch.from_numpy(w.block_mapping).to(device)
     out["out"] = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=tdt, device=device)

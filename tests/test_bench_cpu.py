@@ -1,0 +1,38 @@
+"""bench.py's host side without a GPU: the reference arm (the oracle) prints
+one JSON line with the contract's keys, and the step's byte accounting."""
+import json
+
+import numpy as np
+
+import bench
+from paged_kv_cache_456_b200.workloads import build_workload
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"])
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["config"]["workload"] == "tiny"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_step_bytes_fused_and_separate():
+    w = build_workload("tiny")
+    row = w.num_kv_heads * w.head_dim * w.elem_bytes
+    live = int((w.context_lens > 0).sum())
+    assert bench.step_bytes(w, fused=False) == w.decode_bytes() + 4 * live * row + 8 * live
+    assert bench.step_bytes(w, fused=True) == w.decode_bytes() + 2 * live * row
+
+
+def test_new_rows_per_sequence_layout():
+    w = build_workload("tiny")
+    k, v = w.new_rows_per_sequence()
+    assert k.shape == (w.num_seqs, w.num_kv_heads, w.head_dim)
+    live = np.nonzero(w.context_lens > 0)[0]
+    assert np.array_equal(k[live].view(np.uint8), w.new_key.view(np.uint8))
+    assert np.array_equal(v[live].view(np.uint8), w.new_value.view(np.uint8))
