@@ -43,9 +43,11 @@ struct DeviceInfo {
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
-// (device, kernel, dynamic smem) -> resident CTAs per SM; the kernel's smem
-// attributes are set when an entry is first made.
+// (device, kernel, dynamic smem) -> resident CTAs per SM
 std::map<std::tuple<int, const void*, size_t>, int> g_occupancy;
+// (device, kernel) -> the dynamic smem limit set on it so far; it only grows,
+// so every size met before stays launchable
+std::map<std::pair<int, const void*>, size_t> g_smem_limit;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -92,19 +94,27 @@ pa_status occupancy(const pa::DecodeKernelInfo& k, size_t smem, int* occ) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
+  size_t& limit = g_smem_limit[std::make_pair(dev, k.fn)];
+  if (smem > limit) {
+    if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(k.fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
+      cudaGetLastError();  // leave no launch-time error behind for the caller
+      return PA_ERR_CUDA;
+    }
+    limit = smem;
+  }
   const auto key = std::make_tuple(dev, k.fn, smem);
   auto it = g_occupancy.find(key);
   if (it != g_occupancy.end()) {
     *occ = it->second;
     return PA_OK;
   }
-  if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, k.fn, k.warps * 32, smem) != cudaSuccess) {
+    cudaGetLastError();
     return PA_ERR_CUDA;
-  cudaFuncSetAttribute(k.fn, cudaFuncAttributePreferredSharedMemoryCarveout,
-                       cudaSharedmemCarveoutMaxShared);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, k.fn, k.warps * 32, smem) != cudaSuccess)
-    return PA_ERR_CUDA;
+  }
   g_occupancy[key] = *occ;
   return PA_OK;
 }
@@ -291,8 +301,10 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   void* params[] = {&args};
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   if (cudaLaunchKernel(p.kernel.fn, dim3(p.grid), dim3(p.kernel.warps * 32), params, p.smem,
-                       st_) != cudaSuccess)
+                       st_) != cudaSuccess) {
+    cudaGetLastError();  // a refused launch is reported here, not left for the caller
     return PA_ERR_CUDA;
+  }
   // merge pass for items split into many pieces, launched behind the decode
   // kernel with programmatic dependent launch (it waits for the decode grid)
   int workers = p.grid * p.kernel.workers;
@@ -307,8 +319,11 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, p.kernel.merge_fn, mparams) == cudaSuccess ? PA_OK
-                                                                               : PA_ERR_CUDA;
+  if (cudaLaunchKernelExC(&cfg, p.kernel.merge_fn, mparams) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
 }
 
 }  // namespace

@@ -178,6 +178,19 @@ def test_split_and_unsplit_agree():
         assert (o - outs[0]).abs().max().item() <= 2e-6
 
 
+def test_shared_memory_need_may_shrink_and_grow_again():
+    """The dynamic shared memory a launch needs grows with the batch; calls of
+    one kernel with a large, a small and again the large batch all launch."""
+    for n in (300, 2, 300, 5, 301):
+        w = random_workload(50 + n, dtype="f32", num_q_heads=3, num_kv_heads=3, head_dim=64,
+                            num_seqs=n, max_len=40)
+        ref, _ = oracle.paged_decode(w.q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens,
+                                     scale=w.scale, dtype=w.dtype)
+        t, err, _ = run_gpu(w)
+        assert err == 0
+        assert_attention_close(t["out"], ref, "f32", f"{n} sequences")
+
+
 # ---------------------------------------------------------------------------
 # device-side error contract
 # ---------------------------------------------------------------------------
