@@ -27,6 +27,9 @@ static bool fill(DecodeKernelInfo* info) {
 #ifndef PA_BF16_128_WARPS
 #define PA_BF16_128_WARPS 4
 #endif
+#ifndef PA_BF16_128_MINCTAS_G8
+#define PA_BF16_128_MINCTAS_G8 3
+#endif
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info) {
   constexpr int kD = PA_BF16_128_DEPTH, kD8 = PA_BF16_128_DEPTH_G8, kW = PA_BF16_128_WARPS;
@@ -38,7 +41,7 @@ bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info) {
     case 12801: return fill<128, 1, 1, kD, kW, 3>(info);
     case 12802: return fill<128, 2, 1, kD, kW, 3>(info);
     case 12804: return fill<128, 4, 1, kD, kW, 3>(info);
-    case 12808: return fill<128, 8, 2, kD8, kW, 3>(info);
+    case 12808: return fill<128, 8, 2, kD8, kW, PA_BF16_128_MINCTAS_G8>(info);
     default: return false;
   }
 }

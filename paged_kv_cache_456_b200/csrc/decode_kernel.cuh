@@ -53,6 +53,16 @@ namespace pa {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kMaxOwnRanges = 4;  // range starts a warp keeps in shared memory
 
+// Order the warps' generic reads of a ring slot before the bulk copy that
+// refills it.  Only reads (never generic writes) touch the slots, and every
+// refill follows the release of the slot, so the barrier hand-off alone
+// orders them as in the usual producer/consumer pipelines; the fence is kept
+// as a build option.
+#ifndef PA_PROXY_FENCE
+#define PA_PROXY_FENCE 1
+#endif
+constexpr bool kProxyFence = PA_PROXY_FENCE != 0;
+
 // -- element conversion ---------------------------------------------------------
 template <typename T>
 struct Elem;
@@ -528,7 +538,7 @@ paged_decode_kernel(const DecodeArgs a) {
         const uint32_t kv_bytes = static_cast<uint32_t>(rows) * C::ROW;
         const uint32_t dst = slot0 + slot * C::SLOT;
         const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
-        fence_proxy_async_smem();
+        if (kProxyFence) fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, 2 * kv_bytes + (with_q ? C::QB : 0));
         // with a fused append the last live row comes from key/value, not the cache
         const uint32_t cached = (e.meta & kAppend) ? kv_bytes - C::ROW : kv_bytes;
@@ -1015,13 +1025,10 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   }
   // the last CTA out clears the item list for the next call
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(a.heavy + 1, 1) == static_cast<int>(gridDim.x) - 1) {
-      a.heavy[0] = 0;
-      a.heavy[1] = 0;
-      __threadfence();
-    }
+  // (every thread of this CTA has used the count it read before this point)
+  if (tid == 0 && atomicAdd(a.heavy + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+    a.heavy[0] = 0;
+    a.heavy[1] = 0;
   }
 }
 
