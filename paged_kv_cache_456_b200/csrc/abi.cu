@@ -9,6 +9,8 @@
 #include <mutex>
 #include <tuple>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "paged_attention.h"
@@ -89,6 +91,36 @@ struct DecodePlan {
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// A cache as the 2-D bf16 tensor [rows][head_dim] read by the tensor-core
+// path in boxes of 16 rows x 64 elements (128 bytes) with the 128-byte
+// swizzle.  The encoder is a host-side driver routine, looked up once.
+pa_status encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return PA_ERR_CUDA;
+      }
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pa::kBlockSize)};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                            dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
 
 pa_status occupancy(const pa::DecodeKernelInfo& k, size_t smem, int* occ) {
   int dev = 0;
@@ -297,6 +329,14 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   args.ws_o = reinterpret_cast<float*>(ws + p.o_off);
   args.ws_ml = reinterpret_cast<float2*>(ws + p.ml_off);
   args.err_flag = err_flag;
+  if (p.kernel.tma) {
+    // tile coordinates are 32-bit: row (block * Hkv + kv head) * 16 of the 2-D view
+    const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
+    if (rows >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
+    if ((st = encode_cache_map(&args.tm_k, k_cache, rows, head_dim)) != PA_OK ||
+        (st = encode_cache_map(&args.tm_v, v_cache, rows, head_dim)) != PA_OK)
+      return st;
+  }
 
   void* params[] = {&args};
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);

@@ -13,6 +13,7 @@ static bool fill(DecodeKernelInfo* info) {
   info->workers = WARPS / HS;
   info->depth = DEPTH;
   info->cta_bytes = DecodeCfg<float, D, G / HS, G, HS, DEPTH, WARPS>::CTA_BYTES;
+  info->tma = false;
   return true;
 }
 

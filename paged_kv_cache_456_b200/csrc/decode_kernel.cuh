@@ -103,12 +103,6 @@ struct Elem<__nv_bfloat16> {
   }
 };
 
-// When the one-head path hands its ring slot back (see compute_tile).
-#ifndef PA_G1_RELEASE
-#define PA_G1_RELEASE 0
-#endif
-constexpr int kG1Release = PA_G1_RELEASE;
-
 // -- the two inner loops, on packed fp32 pairs (sm_100 FFMA2) or scalar FMAs ---
 #ifndef PA_PACKED_FMA
 #define PA_PACKED_FMA 1
@@ -170,7 +164,10 @@ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 // -- compile-time geometry --------------------------------------------------------
-template <typename T, int D, int G, int GT, int HS, int DEPTH, int WARPS>
+// MMA: the tensor-core layout of a slot -- K and V tiles as 128-byte-swizzled
+// boxes (1024-byte aligned), then q, then a staging row pair for the fused
+// slot write -- padded to a multiple of 1024 bytes.
+template <typename T, int D, int G, int GT, int HS, int DEPTH, int WARPS, bool MMA = false>
 struct DecodeCfg {
   static constexpr int EB = sizeof(T);
   static constexpr int ROW = D * EB;          // bytes of one token's row of one KV head
@@ -180,7 +177,9 @@ struct DecodeCfg {
   static constexpr int RL = kBlockSize / RPI; // rows per lane per block
   static constexpr int TILE = kBlockSize * ROW;
   static constexpr int QB = GT * ROW;         // q rows of the whole group
-  static constexpr int SLOT = 2 * TILE + QB;  // K tile, V tile, q
+  static constexpr int APP = 2 * TILE + QB;   // MMA: staging for the new K and V rows
+  static constexpr int SLOT =
+      MMA ? ((2 * TILE + QB + 2 * ROW + 1023) / 1024) * 1024 : 2 * TILE + QB;  // K, V, q (, rows)
   static constexpr int XS = kBlockSize * G * 4;
   static constexpr int ALPHA = ((G * 4 + 15) / 16) * 16;
   static constexpr int BND = (kMaxOwnRanges + 1) * 8;
@@ -188,8 +187,11 @@ struct DecodeCfg {
   static constexpr int BAR_OFF = DEPTH * SLOT;         // full[DEPTH], empty[DEPTH]
   static constexpr int DESC_OFF = BAR_OFF + 2 * DEPTH * 8;  // one descriptor per slot
   static constexpr int AUX_OFF = DESC_OFF + DEPTH * 16;
-  static constexpr int WORKER_BYTES = ((AUX_OFF + HS * AUX + 127) / 128) * 128;
-  static constexpr int CTA_BYTES = (WARPS / HS) * WORKER_BYTES;
+  static constexpr int WALIGN = MMA ? 1024 : 128;
+  static constexpr int WORKER_BYTES = ((AUX_OFF + HS * AUX + WALIGN - 1) / WALIGN) * WALIGN;
+  // (MMA: plus slack to align the dynamic shared memory base to 1024 bytes)
+  static constexpr int CTA_BYTES = (WARPS / HS) * WORKER_BYTES + (MMA ? 1024 : 0);
+  static constexpr int MT = D / 16;  // MMA: 16-wide slices of head_dim
   // QK is done CH rows at a time; V = CH*G partial dots are reduce-scattered
   // over the LPR lanes of a row, leaving NV finished logits per lane.
   static constexpr int CH = cmin(RL, LPR / G >= 1 ? LPR / G : 1);
@@ -205,6 +207,8 @@ struct DecodeCfg {
   static_assert(RPI * LPR == 32 && RL * RPI == kBlockSize, "bad lane geometry");
   static_assert(NCH * CH == RL, "bad chunking");
   static_assert(32 % G == 0 && G <= 16 && GT == G * HS, "group size");
+  static_assert(!MMA || (EB == 2 && GT == 8 && HS == 1 && D % 64 == 0),
+                "the tensor-core path takes bf16, 8 heads per KV head, one warp per worker");
 };
 
 // -- per-warp ranges of the global tile order ------------------------------------
@@ -357,11 +361,11 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[V]) {
 // worker (the leader) issues the copies; every warp waits on the slot's
 // "full" barrier and releases the slot on its "empty" barrier, which the
 // leader waits on (bounded) before refilling the slot.
-template <typename T, int D, int GT, int HS, int DEPTH, int WARPS, int MIN_CTAS>
+template <typename T, int D, int GT, int HS, int DEPTH, int WARPS, int MIN_CTAS, bool MMA = false>
 __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS)
-paged_decode_kernel(const DecodeArgs a) {
+paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int G = GT / HS;  // query heads handled by one warp
-  using C = DecodeCfg<T, D, G, GT, HS, DEPTH, WARPS>;
+  using C = DecodeCfg<T, D, G, GT, HS, DEPTH, WARPS, MMA>;
   using E = Elem<T>;
   static_assert(WARPS % HS == 0, "warps per CTA must be a multiple of the head split");
   extern __shared__ __align__(128) unsigned char smem[];
@@ -377,12 +381,14 @@ paged_decode_kernel(const DecodeArgs a) {
   const int Hkv = a.num_kv_heads;
   const int Hq = a.num_q_heads;
   constexpr int WORKERS = WARPS / HS;
-  unsigned char* wkbase = smem + (warp / HS) * C::WORKER_BYTES;
+  // the swizzled tiles of the tensor-core path need 1024-byte alignment
+  unsigned char* sbase = MMA ? smem + ((1024u - (smem_addr(smem) & 1023u)) & 1023u) : smem;
+  unsigned char* wkbase = sbase + (warp / HS) * C::WORKER_BYTES;
   unsigned char* aux = wkbase + C::AUX_OFF + half * C::AUX;
   const uint32_t slot0 = smem_addr(wkbase);
   const uint32_t full0 = smem_addr(wkbase + C::BAR_OFF);
   const uint32_t empty0 = full0 + 8 * DEPTH;
-  int* s_start = reinterpret_cast<int*>(smem + WORKERS * C::WORKER_BYTES);  // [S + 1]
+  int* s_start = reinterpret_cast<int*>(sbase + WORKERS * C::WORKER_BYTES);  // [S + 1]
   int* s_len = s_start + S + 1;                                              // [S]
 
   if (leader && lane == 0) {
@@ -538,6 +544,32 @@ paged_decode_kernel(const DecodeArgs a) {
         const uint32_t kv_bytes = static_cast<uint32_t>(rows) * C::ROW;
         const uint32_t dst = slot0 + slot * C::SLOT;
         const size_t off = (static_cast<size_t>(e.phys) * Hkv + kvh) * C::TILE;
+        if constexpr (MMA) {
+          // whole 16-row tiles through the tensor maps (rows past the end are
+          // masked or zeroed after arrival); the new rows go to the staging pair
+          const bool app = (e.meta & kAppend) != 0;
+          fence_proxy_async_smem();  // the slot may have been written (staged rows, zeroed rows)
+          mbar_arrive_expect_tx(bar, 2 * C::TILE + (with_q ? C::QB : 0) + (app ? 2 * C::ROW : 0));
+          const int y = (e.phys * Hkv + kvh) * kBlockSize;
+#pragma unroll
+          for (int hx = 0; hx < D / 64; ++hx) {
+            tma_load_2d(dst + hx * 2048, &a.tm_k, hx * 64, y, bar);
+            tma_load_2d(dst + C::TILE + hx * 2048, &a.tm_v, hx * 64, y, bar);
+          }
+          if (app) {
+            const size_t src = (static_cast<size_t>(e.seq) * Hkv + kvh) * C::ROW;
+            bulk_copy_g2s(dst + C::APP, static_cast<const char*>(a.key) + src, C::ROW, bar);
+            bulk_copy_g2s(dst + C::APP + C::ROW, static_cast<const char*>(a.value) + src, C::ROW,
+                          bar);
+          }
+          if (with_q)
+            bulk_copy_g2s(dst + 2 * C::TILE,
+                          static_cast<const char*>(a.q) +
+                              (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * GT) *
+                                  C::ROW,
+                          C::QB, bar);
+          return true;
+        }
         if (kProxyFence) fence_proxy_async_smem();
         mbar_arrive_expect_tx(bar, 2 * kv_bytes + (with_q ? C::QB : 0));
         // with a fused append the last live row comes from key/value, not the cache
@@ -592,6 +624,15 @@ paged_decode_kernel(const DecodeArgs a) {
   float o[G][C::VEC];
   float m_run = -INFINITY, l_run = 0.f;
   bool poisoned = false;
+  // tensor-core path: lane (g = lane / 4, t = lane % 4) holds q as the B
+  // operand of S^T = K q^T (heads g; head_dim pairs 2t, 2t+1 and 2t+8, 2t+9
+  // of each 16-wide slice), o^T[head_dim x heads] as C fragments (head_dim
+  // g and g + 8 of each slice; heads 2t and 2t+1), and the running max / sum
+  // of heads 2t and 2t+1 (the sums over this lane's tokens only).
+  uint32_t qb[C::MT][2];
+  float oa[C::MT][4];
+  float mh[2] = {-INFINITY, -INFINITY}, lh[2] = {0.f, 0.f};
+  const int mg = lane >> 2, mtq = lane & 3;
 
   for (int k = 0;; ++k) {
     if (leader && k >= known) break;  // (the partner warp stops at the end marker)
@@ -602,7 +643,25 @@ paged_decode_kernel(const DecodeArgs a) {
     }
     const StageDesc d = ring_desc[slot];
     if (d.meta & kEnd) break;
-    if ((d.meta & kAppend) && leader) {
+    if (MMA && (d.meta & kAppend)) {
+      // fused append: the new token's rows arrived in the staging pair; they
+      // go to their cache slot and into the swizzled tiles in place of the
+      // (stale) cache row the tensor load brought
+      const int nrow = ((d.meta >> 16) & 31) - 1;
+      const size_t off = (static_cast<size_t>(d.phys) * Hkv + (d.meta & 0xffff)) * C::TILE +
+                         static_cast<size_t>(nrow) * C::ROW;
+      unsigned char* sl = wkbase + slot * C::SLOT;
+      for (int c = lane; c < C::ROW / 16; c += 32) {
+        const uint4 kr = *reinterpret_cast<const uint4*>(sl + C::APP + 16 * c);
+        const uint4 vr = *reinterpret_cast<const uint4*>(sl + C::APP + C::ROW + 16 * c);
+        *reinterpret_cast<uint4*>(static_cast<char*>(const_cast<void*>(a.k_cache)) + off + 16 * c) = kr;
+        *reinterpret_cast<uint4*>(static_cast<char*>(const_cast<void*>(a.v_cache)) + off + 16 * c) = vr;
+        const int so = (c >> 3) * 2048 + nrow * 128 + (((c & 7) ^ (nrow & 7)) << 4);
+        *reinterpret_cast<uint4*>(sl + so) = kr;
+        *reinterpret_cast<uint4*>(sl + C::TILE + so) = vr;
+      }
+      __syncwarp();
+    } else if ((d.meta & kAppend) && leader) {
       // fused append: the new token's row, now in shared memory, goes to its cache slot
       const int nrow = ((d.meta >> 16) & 31) - 1;
       const size_t off = (static_cast<size_t>(d.phys) * Hkv + (d.meta & 0xffff)) * C::TILE +
@@ -621,7 +680,19 @@ paged_decode_kernel(const DecodeArgs a) {
     const unsigned char* pk = wkbase + slot * C::SLOT;
     const unsigned char* pv = pk + C::TILE;
 
-    if (flags & kFirst) {
+    if (MMA && (flags & kFirst)) {
+      const unsigned char* pq = pk + 2 * C::TILE + mg * C::ROW + mtq * 4;
+#pragma unroll
+      for (int ks = 0; ks < C::MT; ++ks) {
+        qb[ks][0] = *reinterpret_cast<const uint32_t*>(pq + ks * 32);
+        qb[ks][1] = *reinterpret_cast<const uint32_t*>(pq + ks * 32 + 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oa[ks][e] = 0.f;
+      }
+      mh[0] = mh[1] = -INFINITY;
+      lh[0] = lh[1] = 0.f;
+      poisoned = false;
+    } else if (flags & kFirst) {
       const unsigned char* pq = pk + 2 * C::TILE;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -641,8 +712,7 @@ paged_decode_kernel(const DecodeArgs a) {
     }
 
     // Hand the slot back (this warp has read what it needs) and, on the leader,
-    // refill it with position k + DEPTH.  Called exactly once per tile: by the
-    // one-head path as soon as its rows are in registers, otherwise after the tile.
+    // refill it with position k + DEPTH.  Called exactly once per tile, after it.
     bool refill_ok = true;
     auto release = [&]() {
       __syncwarp();
@@ -652,24 +722,81 @@ paged_decode_kernel(const DecodeArgs a) {
 
     auto compute_tile = [&](auto mask_tag) {
       constexpr bool MASK = decltype(mask_tag)::value;
-      if constexpr (G == 1) {
-        // ---- one query head.  kG1Release: 2 = the lane's K and V rows go to
-        // registers first and the slot is refilled before any arithmetic; 1 = V
-        // goes to registers and the slot is refilled after QK; 0 = after the tile.
-        uint4 kr[C::RL], vr[C::RL];
-        if constexpr (kG1Release >= 1) {
+      if constexpr (MMA) {
+        // ---- 8 heads on the tensor cores: S^T = K q^T, online softmax on the
+        // fragments, o^T += V^T P^T.  Rows past the end of a partial tile:
+        // their logits are masked and their V rows zeroed (a stale or NaN row
+        // times a zero weight would still poison the sum).
+        if (MASK) {
+          unsigned char* vt = const_cast<unsigned char*>(pv);
+          for (int c = lane; c < (kBlockSize - rows) * (C::ROW / 16); c += 32) {
+            const int r = rows + c / (C::ROW / 16), cc = c % (C::ROW / 16);
+            *reinterpret_cast<uint4*>(vt + (cc >> 3) * 2048 + r * 128 + ((cc & 7) << 4)) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();  // before the tensor load that next refills the slot
+          __syncwarp();
+        }
+        const uint32_t kb = smem_addr(pk), vb = kb + C::TILE;
+        const int lr = lane & 7, lm = lane >> 3;  // ldmatrix: row within matrix, matrix
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int i = 0; i < C::RL; ++i) {
-            const int row = i * C::RPI + rgp;
-            if (!MASK || row < rows) {
-              if constexpr (kG1Release == 2)
-                kr[i] = *reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16);
-              vr[i] = *reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16);
+        for (int ks = 0; ks < C::MT; ++ks) {
+          // matrices: tokens 0-7 / 8-15 x head_dim ks*16 + 0-7, then + 8-15
+          const int tok = (lm & 1) * 8 + lr;
+          const int ch = ks * 2 + (lm >> 1);
+          uint32_t af[4];
+          ldmatrix_x4(kb + (ch >> 3) * 2048 + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4), af);
+          mma_bf16_16816(sc, af, qb[ks][0], qb[ks][1]);
+        }
+        // sc: tokens mg, mg, mg+8, mg+8 x heads 2t, 2t+1, 2t, 2t+1 (t = mtq)
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = mg + (e >> 1) * 8;
+          x[e] = (!MASK || tok < rows) ? sc[e] * a.scale_log2 : -INFINITY;
+        }
+        float mx[2] = {fmaxf(x[0], x[2]), fmaxf(x[1], x[3])};
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx[0] = fmaxf(mx[0], __shfl_xor_sync(kFull, mx[0], off));
+          mx[1] = fmaxf(mx[1], __shfl_xor_sync(kFull, mx[1], off));
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (mx[j] > mh[j] + kRescaleThreshold) {
+            const float al = exp2f(mh[j] - mx[j]);
+            mh[j] = mx[j];
+            lh[j] *= al;
+#pragma unroll
+            for (int mt = 0; mt < C::MT; ++mt) {
+              oa[mt][j] *= al;
+              oa[mt][j + 2] *= al;
             }
           }
         }
-        if constexpr (kG1Release == 2) release();
-        // every lane keeps the logits of its row group
+        __syncwarp();
+        const __nv_bfloat162 p01 =
+            __floats2bfloat162_rn(exp2f(x[0] - mh[0]), exp2f(x[1] - mh[1]));
+        const __nv_bfloat162 p23 =
+            __floats2bfloat162_rn(exp2f(x[2] - mh[0]), exp2f(x[3] - mh[1]));
+        // the sums take the weights as rounded for the product
+        lh[0] += __low2float(p01) + __low2float(p23);
+        lh[1] += __high2float(p01) + __high2float(p23);
+        const uint32_t b0 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&p01));
+        const uint32_t b1 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&p23));
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          // matrices (transposed on load): tokens 0-7 x head_dim mt*16 + 0-7 /
+          // + 8-15, then tokens 8-15 x the same
+          const int tok = (lm >> 1) * 8 + lr;
+          const int ch = mt * 2 + (lm & 1);
+          uint32_t af[4];
+          ldmatrix_x4_trans(vb + (ch >> 3) * 2048 + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4), af);
+          mma_bf16_16816(oa[mt], af, b0, b1);
+        }
+      } else if constexpr (G == 1) {
+        // ---- one query head: every lane keeps the logits of its row group
         float x[C::RL];
 #pragma unroll
         for (int i = 0; i < C::RL; ++i) {
@@ -677,14 +804,10 @@ paged_decode_kernel(const DecodeArgs a) {
           x[i] = 0.f;
           if (!MASK || row < rows) {
             float kf[C::VEC];
-            if constexpr (kG1Release == 2)
-              E::unpack(kr[i], kf);
-            else
-              E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
+            E::unpack(*reinterpret_cast<const uint4*>(pk + row * C::ROW + dl * 16), kf);
             x[i] = dot_vec<C::VEC>(qv[0], kf);
           }
         }
-        if constexpr (kG1Release == 1) release();
 #pragma unroll
         for (int off = C::LPR / 2; off >= 1; off >>= 1)
 #pragma unroll
@@ -710,10 +833,7 @@ paged_decode_kernel(const DecodeArgs a) {
           l_run += p;
           if (!MASK || row < rows) {
             float vf[C::VEC];
-            if constexpr (kG1Release >= 1)
-              E::unpack(vr[i], vf);
-            else
-              E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
+            E::unpack(*reinterpret_cast<const uint4*>(pv + row * C::ROW + dl * 16), vf);
             axpy_vec<C::VEC>(p, vf, o[0]);
           }
         }
@@ -807,15 +927,58 @@ paged_decode_kernel(const DecodeArgs a) {
     } else {
       compute_tile(std::true_type{});
     }
-    // the one-head path may have released the slot inside compute_tile already
-    if (G > 1 || kG1Release == 0 || (flags & kBad)) release();
+    release();
     if (!refill_ok) {
       bail_out(k + 1);
       return;
     }
 
     // ---- end of a piece: write the output or a partial -------------------------
-    if (flags & kLast) {
+    if (MMA && (flags & kLast)) {
+      float lt[2] = {lh[0], lh[1]};
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        lt[0] += __shfl_xor_sync(kFull, lt[0], off);
+        lt[1] += __shfl_xor_sync(kFull, lt[1], off);
+      }
+      const bool bad = __any_sync(kFull, poisoned);
+      const int s = d.seq;
+      const int nb = (s_len[s] + kBlockSize - 1) / kBlockSize;
+      const long long item_a = s_start[s] + static_cast<long long>(kvh) * nb;
+      const long long ra = rg.of(item_a);
+      const long long rb = rg.of(item_a + nb - 1);
+      const int h0 = 2 * mtq;  // this lane's heads h0, h0 + 1; head_dim mg, mg + 8 of each slice
+      if (ra == rb) {
+        // the whole (seq, kv head) was this piece: normalise and store
+        T* dst = static_cast<T*>(a.out) +
+                 (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * GT + h0) * D + mg;
+        const float i0 = bad ? 0.f : 1.f / lt[0], i1 = bad ? 0.f : 1.f / lt[1];
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          dst[mt * 16] = static_cast<T>(oa[mt][0] * i0);
+          dst[D + mt * 16] = static_cast<T>(oa[mt][1] * i1);
+          dst[mt * 16 + 8] = static_cast<T>(oa[mt][2] * i0);
+          dst[D + mt * 16 + 8] = static_cast<T>(oa[mt][3] * i1);
+        }
+      } else {
+        // a partial; every split item of this path is merged by the merge pass
+        const long long r = rg.of(d.g);
+        const long long sl = piece_slot(rg, r, item_a);
+        float* wo = a.ws_o + (sl * GT + h0) * D + mg;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          wo[mt * 16] = oa[mt][0];
+          wo[D + mt * 16] = oa[mt][1];
+          wo[mt * 16 + 8] = oa[mt][2];
+          wo[D + mt * 16 + 8] = oa[mt][3];
+        }
+        if (mg == 0) {
+          a.ws_ml[sl * GT + h0] = make_float2(mh[0], bad ? -1.f : lt[0]);
+          a.ws_ml[sl * GT + h0 + 1] = make_float2(mh[1], bad ? -1.f : lt[1]);
+        }
+        if (r == ra && lane == 0) a.heavy_list[atomicAdd(a.heavy, 1)] = s * Hkv + kvh;
+      }
+    } else if (flags & kLast) {
 #pragma unroll
       for (int off = C::LPR; off < 32; off <<= 1)
 #pragma unroll

@@ -5,6 +5,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>  // CUtensorMap (a plain 128-byte descriptor; no driver call here)
+
 namespace pa {
 
 constexpr int kBlockSize = 16;            // token slots per KV block
@@ -32,7 +34,8 @@ __host__ __device__ inline long long chunk_tiles(int part_blocks) {
 }
 // tiles of the claimed tail; only used when every worker can get a chunk
 __host__ __device__ inline long long tail_tiles(long long W, long long workers) {
-  return (kTailDiv > 0 && W / kTailDiv >= workers) ? W / kTailDiv : 0;
+  constexpr int div = kTailDiv > 0 ? kTailDiv : 1;
+  return (kTailDiv > 0 && W / div >= workers) ? W / div : 0;
 }
 
 struct DecodeArgs {
@@ -61,6 +64,10 @@ struct DecodeArgs {
   float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
   float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
   int32_t* err_flag;
+  // tensor-core path only: the caches as 2-D tensors [num_blocks * Hkv * 16][head_dim]
+  // read in boxes of 16 rows x 128 bytes with the 128-byte swizzle
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
 };
 
 // A split (seq, kv head) whose pieces x G exceed this is merged by the
@@ -75,6 +82,7 @@ struct DecodeKernelInfo {
   int workers;      // work streams per CTA (warps / head split)
   int depth;        // ring slots per worker
   int cta_bytes;    // dynamic shared memory per CTA, without the per-sequence arrays
+  bool tma;         // reads tiles through the tm_k / tm_v tensor maps
 };
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);

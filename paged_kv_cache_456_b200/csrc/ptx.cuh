@@ -1,5 +1,7 @@
-// ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, the 1-D bulk
-// copy engine (TMA, global -> shared), proxy fences and the global timer.
+// ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, the bulk copy
+// engine (TMA: 1-D copies and 2-D tiled tensor loads, global -> shared, never
+// multicast), proxy fences, the global timer, and the warp-level tensor-core
+// pieces of the grouped-head path (ldmatrix, movmatrix, mma m16n8k16 bf16).
 // Every wait on an mbarrier is bounded in time; none of these helpers traps.
 #pragma once
 
@@ -95,6 +97,51 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
           dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// 2-D tiled TMA load of one box of `tmap` at element coordinates (x, y)
+// into this CTA's shared memory, completion counted on `bar`.  x must be a
+// multiple of 16 bytes' worth of elements; `tmap` is the address of a
+// __grid_constant__ kernel parameter.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// Four 8x8 b16 matrices from shared memory; lane l gives the address of row
+// l % 8 of matrix l / 8.  `trans` delivers each matrix transposed.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// Transpose of an 8x8 b16 matrix held one 32-bit pair per lane.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// c[16x8, fp32] += a[16x16, bf16, row-major] * b[16x8, bf16, column-major]
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32"
+      " {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 }  // namespace pa
