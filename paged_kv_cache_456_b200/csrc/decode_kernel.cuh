@@ -52,6 +52,9 @@ namespace pa {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kMaxOwnRanges = 4;  // range starts a warp keeps in shared memory
+// Tensor-core path: a split item of at most this many pieces is merged by the
+// warp that finishes its last piece; more go to the merge pass.
+constexpr int kMmaFuseMaxPieces = 4;
 
 // Order the warps' generic reads of a ring slot before the bulk copy that
 // refills it.  Only reads (never generic writes) touch the slots, and every
@@ -976,7 +979,55 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           a.ws_ml[sl * GT + h0] = make_float2(mh[0], bad ? -1.f : lt[0]);
           a.ws_ml[sl * GT + h0 + 1] = make_float2(mh[1], bad ? -1.f : lt[1]);
         }
-        if (r == ra && lane == 0) a.heavy_list[atomicAdd(a.heavy, 1)] = s * Hkv + kvh;
+        if (rb - ra + 1 > kMmaFuseMaxPieces) {
+          // many pieces: the merge pass combines them; the first piece lists the item
+          if (r == ra && lane == 0) a.heavy_list[atomicAdd(a.heavy, 1)] = s * Hkv + kvh;
+        } else {
+          __threadfence();
+          __syncwarp();
+          int prev = 0;
+          int* cnt = a.counters + (static_cast<size_t>(s) * Hkv + kvh) * 2;
+          if (lane == 0) prev = atomicAdd(cnt, 1);
+          prev = __shfl_sync(kFull, prev, 0);
+          if (prev == static_cast<int>(rb - ra)) {
+            // last piece of this (seq, kv head): merge all pieces by log-sum-exp,
+            // lane l taking head_dim [DPL*l, DPL*l + DPL) of every head
+            __threadfence();
+            constexpr int DPL = D / 32;
+            T* orow = static_cast<T*>(a.out) +
+                      (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * GT) * D + lane * DPL;
+#pragma unroll 1
+            for (int h = 0; h < GT; ++h) {
+              float M = -INFINITY;
+              bool any_bad = false;
+              for (long long rr = ra; rr <= rb; ++rr) {
+                const float2 ml = __ldcg(a.ws_ml + piece_slot(rg, rr, item_a) * GT + h);
+                any_bad |= ml.y < 0.f;
+                M = fmaxf(M, ml.x);
+              }
+              float L = 0.f, acc[DPL];
+#pragma unroll
+              for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+              for (long long rr = ra; rr <= rb; ++rr) {
+                const long long ss = piece_slot(rg, rr, item_a);
+                const float2 ml = __ldcg(a.ws_ml + ss * GT + h);
+                const float w = exp2f(ml.x - M);
+                L += w * ml.y;
+                const float* po = a.ws_o + (ss * GT + h) * D + lane * DPL;
+#pragma unroll
+                for (int e = 0; e < DPL; e += 2) {
+                  const float2 t2 = __ldcg(reinterpret_cast<const float2*>(po + e));
+                  acc[e] = fmaf(w, t2.x, acc[e]);
+                  acc[e + 1] = fmaf(w, t2.y, acc[e + 1]);
+                }
+              }
+              const float inv = any_bad ? 0.f : 1.f / L;
+#pragma unroll
+              for (int e = 0; e < DPL; ++e) orow[h * D + e] = static_cast<T>(any_bad ? 0.f : acc[e] * inv);
+            }
+            if (lane == 0) *cnt = 0;  // leave the workspace zeroed for the next call
+          }
+        }
       }
     } else if (flags & kLast) {
 #pragma unroll

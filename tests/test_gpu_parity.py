@@ -191,6 +191,49 @@ def test_shared_memory_need_may_shrink_and_grow_again():
         assert_attention_close(t["out"], ref, "f32", f"{n} sequences")
 
 
+@pytest.mark.parametrize("G", [4, 8])
+def test_write_into_one_copy_moves_only_its_sequence(G):
+    """Copy-on-write isolation on the GPU: after the copies, a slot write into
+    one sequence's private copy of the last shared block changes that
+    sequence's output alone, bit for bit everywhere else."""
+    rng = np.random.default_rng(23)
+    lens = 2048 + rng.integers(1, 300, size=16)
+    w = make_workload(rng, name="cow", dtype="bf16", num_q_heads=2 * G, num_kv_heads=2,
+                      head_dim=128, context_lens=lens, num_blocks=600, prefix_tokens=2048,
+                      cow_count=8)
+    t, err, _ = run_gpu(w)
+    assert err == 0
+    out0 = t["out"].clone()
+    src, dst = (int(x) for x in w.block_mapping[0])
+    tables = w.block_tables
+    owners = [s for s in range(w.num_seqs) if dst in tables[s]]
+    assert len(owners) == 1
+    src_k = t["k_cache"][src].clone()
+    key = torch.randn(1, 2, 128, device="cuda").to(torch.bfloat16)
+    slots = torch.tensor([dst * 16 + 15], dtype=torch.int64, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.reshape_and_cache(key, -key, t["k_cache"], t["v_cache"], slots, err_flag=e)
+    ws = ops.make_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.max_context_len, 0, torch.bfloat16)
+    ops.decode(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+               scale=w.scale, max_context_len=w.max_context_len, workspace=ws, err_flag=e)
+    torch.cuda.synchronize()
+    assert e.item() == 0
+    same = (t["out"].view(torch.int16) == out0.view(torch.int16)).flatten(1).all(dim=1).cpu()
+    assert [s for s in range(w.num_seqs) if not same[s]] == owners
+    assert torch.equal(t["k_cache"][src].view(torch.int16), src_k.view(torch.int16))
+    # and the moved row is right
+    k_ref, v_ref = w.k_pool.copy(), w.v_pool.copy()
+    oracle.copy_blocks(k_ref, v_ref, w.block_mapping_compact)
+    cdst = int(w.block_mapping_compact[0][1])
+    kb = key.view(torch.int16).cpu().numpy()
+    oracle.reshape_and_cache(k_ref, v_ref, kb, (-key).view(torch.int16).cpu().numpy(),
+                             np.array([cdst * 16 + 15]))
+    ref, _ = oracle.paged_decode(w.q, k_ref, v_ref, w.tables_compact, w.context_lens,
+                                 scale=w.scale, dtype=w.dtype)
+    assert_attention_close(t["out"], ref, "bf16", "after the write into one copy")
+
+
 # ---------------------------------------------------------------------------
 # device-side error contract
 # ---------------------------------------------------------------------------

@@ -321,6 +321,32 @@ def test_workload_step_on_prefix_cow_shape():
     assert np.isnan(bad).any()
 
 
+def test_write_into_one_copy_moves_only_its_sequence():
+    """After copy-on-write, a slot write into one sequence's private copy of
+    the last shared block changes that sequence's output alone; the source
+    block and every other row stay bit-identical (day-9 post, "Idea 1",
+    copy-on-write)."""
+    rng = np.random.default_rng(22)
+    lens = 64 + rng.integers(1, 30, size=6)
+    w = make_workload(rng, name="cow", dtype="f32", num_q_heads=4, num_kv_heads=2, head_dim=64,
+                      context_lens=lens, num_blocks=100, prefix_tokens=64, cow_count=3)
+    out0, k, v, err = oracle.workload_step(w)
+    assert err == 0
+    src, dst = (int(x) for x in w.block_mapping_compact[0])
+    owners = [s for s in range(w.num_seqs) if dst in w.tables_compact[s]]
+    sharers = [s for s in range(w.num_seqs) if src in w.tables_compact[s]]
+    assert len(owners) == 1 and len(sharers) >= 1
+    src_before = (k[src].copy(), v[src].copy())
+    key = rng.standard_normal((1, 2, 64)).astype(np.float32)
+    assert oracle.reshape_and_cache(k, v, key, -key, np.array([dst * 16 + 15])) == 0
+    out1, e = oracle.paged_decode(w.q, k, v, w.tables_compact, w.context_lens, scale=w.scale,
+                                  dtype=w.dtype)
+    assert e == 0
+    changed = [s for s in range(w.num_seqs) if not np.array_equal(out0[s], out1[s])]
+    assert changed == owners
+    assert np.array_equal(k[src], src_before[0]) and np.array_equal(v[src], src_before[1])
+
+
 # ---------------------------------------------------------------------------
 # mutation checks: each plausible mistake is caught by a pin
 # ---------------------------------------------------------------------------
