@@ -52,9 +52,9 @@ namespace pa {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kMaxOwnRanges = 4;  // range starts a warp keeps in shared memory
-// Tensor-core path: a split item of at most this many pieces is merged by the
-// warp that finishes its last piece; more go to the merge pass.
-constexpr int kMmaFuseMaxPieces = 4;
+// Merge pass: an item of at most this many pieces is merged by one warp (all
+// its heads); items with more pieces get a whole CTA per head.
+constexpr int kWarpMergeMaxPieces = 8;
 
 // Order the warps' generic reads of a ring slot before the bulk copy that
 // refills it.  Only reads (never generic writes) touch the slots, and every
@@ -964,7 +964,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           dst[D + mt * 16 + 8] = static_cast<T>(oa[mt][3] * i1);
         }
       } else {
-        // a partial; every split item of this path is merged by the merge pass
+        // a partial: no fence or counter here; the merge pass, which starts once
+        // this grid has finished, combines the pieces
         const long long r = rg.of(d.g);
         const long long sl = piece_slot(rg, r, item_a);
         float* wo = a.ws_o + (sl * GT + h0) * D + mg;
@@ -979,55 +980,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           a.ws_ml[sl * GT + h0] = make_float2(mh[0], bad ? -1.f : lt[0]);
           a.ws_ml[sl * GT + h0 + 1] = make_float2(mh[1], bad ? -1.f : lt[1]);
         }
-        if (rb - ra + 1 > kMmaFuseMaxPieces) {
-          // many pieces: the merge pass combines them; the first piece lists the item
-          if (r == ra && lane == 0) a.heavy_list[atomicAdd(a.heavy, 1)] = s * Hkv + kvh;
-        } else {
-          __threadfence();
-          __syncwarp();
-          int prev = 0;
-          int* cnt = a.counters + (static_cast<size_t>(s) * Hkv + kvh) * 2;
-          if (lane == 0) prev = atomicAdd(cnt, 1);
-          prev = __shfl_sync(kFull, prev, 0);
-          if (prev == static_cast<int>(rb - ra)) {
-            // last piece of this (seq, kv head): merge all pieces by log-sum-exp,
-            // lane l taking head_dim [DPL*l, DPL*l + DPL) of every head
-            __threadfence();
-            constexpr int DPL = D / 32;
-            T* orow = static_cast<T*>(a.out) +
-                      (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * GT) * D + lane * DPL;
-#pragma unroll 1
-            for (int h = 0; h < GT; ++h) {
-              float M = -INFINITY;
-              bool any_bad = false;
-              for (long long rr = ra; rr <= rb; ++rr) {
-                const float2 ml = __ldcg(a.ws_ml + piece_slot(rg, rr, item_a) * GT + h);
-                any_bad |= ml.y < 0.f;
-                M = fmaxf(M, ml.x);
-              }
-              float L = 0.f, acc[DPL];
-#pragma unroll
-              for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-              for (long long rr = ra; rr <= rb; ++rr) {
-                const long long ss = piece_slot(rg, rr, item_a);
-                const float2 ml = __ldcg(a.ws_ml + ss * GT + h);
-                const float w = exp2f(ml.x - M);
-                L += w * ml.y;
-                const float* po = a.ws_o + (ss * GT + h) * D + lane * DPL;
-#pragma unroll
-                for (int e = 0; e < DPL; e += 2) {
-                  const float2 t2 = __ldcg(reinterpret_cast<const float2*>(po + e));
-                  acc[e] = fmaf(w, t2.x, acc[e]);
-                  acc[e + 1] = fmaf(w, t2.y, acc[e + 1]);
-                }
-              }
-              const float inv = any_bad ? 0.f : 1.f / L;
-#pragma unroll
-              for (int e = 0; e < DPL; ++e) orow[h * D + e] = static_cast<T>(any_bad ? 0.f : acc[e] * inv);
-            }
-            if (lane == 0) *cnt = 0;  // leave the workspace zeroed for the next call
-          }
-        }
+        // the merge pass combines the pieces; the first piece lists the item
+        if (r == ra && lane == 0) a.heavy_list[atomicAdd(a.heavy, 1)] = s * Hkv + kvh;
       }
     } else if (flags & kLast) {
 #pragma unroll
@@ -1150,9 +1104,10 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   }
 }
 
-// Merge pass for (seq, kv head) items split into many pieces (long contexts):
-// one CTA per (item, query head) at a time, kMergeThreads / 32 groups of lanes
-// taking every GROUPS-th piece, combined in shared memory:
+// Merge pass for the (seq, kv head) items listed by the decode kernel.  An
+// item of few pieces is merged by one warp; an item of many pieces (long
+// contexts) gets one CTA per (item, query head), kMergeThreads / 32 groups of
+// lanes taking every GROUPS-th piece, combined in shared memory:
 //     M = max_j m_j,  out = sum_j 2^(m_j - M) o_j / sum_j 2^(m_j - M) l_j.
 // Launched right behind the decode kernel with programmatic dependent launch;
 // griddepcontrol.wait returns once the decode grid has finished and its
@@ -1174,6 +1129,49 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   const long long W = __ldcg(a.seq_start + S);
   if (W > 0) {
     const Ranges rg = make_ranges(W, workers, a.part_blocks);
+    // items of few pieces: one warp each, all G heads, lane l taking head_dim
+    // [DPL*l, DPL*l + DPL)
+    for (int it = blockIdx.x * GROUPS + grp; it < count; it += gridDim.x * GROUPS) {
+      const int item = __ldcg(a.heavy_list + it);
+      const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
+      const int st = __ldcg(a.seq_start + s);
+      const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
+      const long long item_a = st + static_cast<long long>(kvh) * nb;
+      const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
+      if (rb - ra + 1 > kWarpMergeMaxPieces) continue;
+      T* orow = static_cast<T*>(a.out) +
+                (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D + lane * DPL;
+#pragma unroll 1
+      for (int hl = 0; hl < G; ++hl) {
+        float M = -INFINITY;
+        int bad = 0;
+        for (long long r = ra; r <= rb; ++r) {
+          const float2 ml = __ldcg(a.ws_ml + piece_slot(rg, r, item_a) * G + hl);
+          M = fmaxf(M, ml.x);
+          bad |= ml.y < 0.f;
+        }
+        float L = 0.f, acc[DPL];
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+        for (long long r = ra; r <= rb; ++r) {
+          const long long sl = piece_slot(rg, r, item_a);
+          const float2 ml = __ldcg(a.ws_ml + sl * G + hl);
+          const float w = exp2f(ml.x - M);
+          L = fmaf(w, ml.y, L);
+          const float* po = a.ws_o + (sl * G + hl) * D + lane * DPL;
+#pragma unroll
+          for (int d = 0; d < DPL; d += 2) {
+            const float2 t2 = __ldcg(reinterpret_cast<const float2*>(po + d));
+            acc[d] = fmaf(w, t2.x, acc[d]);
+            acc[d + 1] = fmaf(w, t2.y, acc[d + 1]);
+          }
+        }
+        const float inv = bad ? 0.f : 1.f / L;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) orow[hl * D + d] = static_cast<T>(bad ? 0.f : acc[d] * inv);
+      }
+    }
+    // items of many pieces: one CTA per (item, head)
     for (int p = blockIdx.x; p < count * G; p += gridDim.x) {
       const int item = __ldcg(a.heavy_list + p / G);
       const int hl = p % G;
@@ -1182,6 +1180,7 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
       const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
       const long long item_a = st + static_cast<long long>(kvh) * nb;
       const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
+      if (rb - ra + 1 <= kWarpMergeMaxPieces) continue;  // (the same for the whole CTA)
 
       float M = -INFINITY;
       int bad = 0;

@@ -70,9 +70,12 @@ struct DecodeArgs {
   CUtensorMap tm_v;
 };
 
-// A split (seq, kv head) whose pieces x G exceed this is merged by the
-// separate merge pass (many CTAs) instead of by one warp of the decode kernel.
-constexpr int kFuseMaxValues = 16;
+// CUDA-core path: a split (seq, kv head) whose pieces x G exceed this is merged
+// by the separate merge pass instead of by one warp of the decode kernel.
+#ifndef PA_FUSE_MAX_VALUES
+#define PA_FUSE_MAX_VALUES 16
+#endif
+constexpr int kFuseMaxValues = PA_FUSE_MAX_VALUES;
 constexpr int kMergeThreads = 256;
 
 struct DecodeKernelInfo {
