@@ -1129,8 +1129,13 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   const long long W = __ldcg(a.seq_start + S);
   if (W > 0) {
     const Ranges rg = make_ranges(W, workers, a.part_blocks);
-    // items of few pieces: one warp each, all G heads, lane l taking head_dim
-    // [DPL*l, DPL*l + DPL)
+    // items of few pieces: one warp each.  Lane l takes head l / LPH and
+    // VPL consecutive elements of it; every load of the item is issued
+    // before any is used (the partials may come from HBM).
+    constexpr int LPH = 32 / G;   // lanes per head
+    constexpr int VPL = D / LPH;  // values per lane
+    constexpr int NP = kWarpMergeMaxPieces;
+    const int hw = lane / LPH, d0 = (lane % LPH) * VPL;
     for (int it = blockIdx.x * GROUPS + grp; it < count; it += gridDim.x * GROUPS) {
       const int item = __ldcg(a.heavy_list + it);
       const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
@@ -1138,38 +1143,44 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
       const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
       const long long item_a = st + static_cast<long long>(kvh) * nb;
       const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
-      if (rb - ra + 1 > kWarpMergeMaxPieces) continue;
-      T* orow = static_cast<T*>(a.out) +
-                (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D + lane * DPL;
-#pragma unroll 1
-      for (int hl = 0; hl < G; ++hl) {
-        float M = -INFINITY;
-        int bad = 0;
-        for (long long r = ra; r <= rb; ++r) {
-          const float2 ml = __ldcg(a.ws_ml + piece_slot(rg, r, item_a) * G + hl);
-          M = fmaxf(M, ml.x);
-          bad |= ml.y < 0.f;
-        }
-        float L = 0.f, acc[DPL];
+      const int np = static_cast<int>(rb - ra + 1);
+      if (np > NP) continue;
+      long long sl[NP];
+      float2 ml[NP];
+      float M = -INFINITY;
+      int bad = 0;
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
-        for (long long r = ra; r <= rb; ++r) {
-          const long long sl = piece_slot(rg, r, item_a);
-          const float2 ml = __ldcg(a.ws_ml + sl * G + hl);
-          const float w = exp2f(ml.x - M);
-          L = fmaf(w, ml.y, L);
-          const float* po = a.ws_o + (sl * G + hl) * D + lane * DPL;
+      for (int r = 0; r < NP; ++r) {
+        sl[r] = r < np ? piece_slot(rg, ra + r, item_a) : 0;
+        ml[r] = r < np ? __ldcg(a.ws_ml + sl[r] * G + hw) : make_float2(-INFINITY, 0.f);
+      }
 #pragma unroll
-          for (int d = 0; d < DPL; d += 2) {
-            const float2 t2 = __ldcg(reinterpret_cast<const float2*>(po + d));
-            acc[d] = fmaf(w, t2.x, acc[d]);
-            acc[d + 1] = fmaf(w, t2.y, acc[d + 1]);
+      for (int r = 0; r < NP; ++r) {
+        M = fmaxf(M, ml[r].x);
+        bad |= ml[r].y < 0.f;
+      }
+      float L = 0.f, acc[VPL];
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int r = 0; r < NP; ++r) {
+        if (r < np) {
+          const float w = exp2f(ml[r].x - M);
+          L = fmaf(w, ml[r].y, L);
+          const float2* po = reinterpret_cast<const float2*>(a.ws_o + (sl[r] * G + hw) * D + d0);
+#pragma unroll
+          for (int e = 0; e < VPL / 2; ++e) {
+            const float2 t2 = __ldcg(po + e);
+            acc[2 * e] = fmaf(w, t2.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(w, t2.y, acc[2 * e + 1]);
           }
         }
-        const float inv = bad ? 0.f : 1.f / L;
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) orow[hl * D + d] = static_cast<T>(bad ? 0.f : acc[d] * inv);
       }
+      const float inv = bad ? 0.f : 1.f / L;
+      T* dst = static_cast<T*>(a.out) +
+               (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G + hw) * D + d0;
+#pragma unroll
+      for (int e = 0; e < VPL; ++e) dst[e] = static_cast<T>(bad ? 0.f : acc[e] * inv);
     }
     // items of many pieces: one CTA per (item, head)
     for (int p = blockIdx.x; p < count * G; p += gridDim.x) {
