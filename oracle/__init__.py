@@ -48,6 +48,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_paged_decode.restype = i
     lib.oracle_paged_decode_partitioned.argtypes = [p, p, p, p, p, p] + [i] * 8 + [d, i, i]
     lib.oracle_paged_decode_partitioned.restype = i
+    lib.oracle_paged_prefill.argtypes = [p, p, p, p, p, p, p] + [i] * 9 + [d, i]
+    lib.oracle_paged_prefill.restype = i
     lib.oracle_reshape_and_cache.argtypes = [p, p, p, p, p] + [i] * 6
     lib.oracle_reshape_and_cache.restype = i
     lib.oracle_copy_blocks.argtypes = [p, p, p] + [i] * 6
@@ -104,6 +106,31 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, *, scale: floa
         err = lib.oracle_paged_decode_partitioned(*args, int(partition_size))
     else:
         err = lib.oracle_paged_decode(*args)
+    return out, int(err)
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, *, scale: float,
+                  dtype: str, max_context_len: Optional[int] = None,
+                  lib: Optional[ctypes.CDLL] = None):
+    """fp64 causal attention of several query tokens per sequence, the last
+    ``Q_s = query_start[s+1] - query_start[s]`` of its ``context_lens[s]``
+    tokens.  ``q``: ``[query_start[S]][Hq][D]``; returns ``(out, err_bits)``."""
+    lib = lib or load()
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    tables = _c(block_tables, np.int32)
+    lens = _c(context_lens, np.int32)
+    qs = _c(query_start, np.int32)
+    T, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    S = lens.shape[0]
+    assert D2 == D and v_cache.shape == k_cache.shape and tables.shape[0] == S
+    assert qs.shape[0] == S + 1
+    if max_context_len is None:
+        max_context_len = int(lens.max()) if S else 0
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    err = lib.oracle_paged_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(tables),
+                                   _ptr(lens), _ptr(qs), S, T, Hq, Hkv, D, bs, tables.shape[1], N,
+                                   int(max_context_len), float(scale), _DT[dtype])
     return out, int(err)
 
 

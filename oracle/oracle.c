@@ -39,6 +39,7 @@
  *       max_blocks_per_seq * block_size)]                 (row -> zeros)
  *   4 = a slot id >= num_blocks * block_size               (token skipped)
  *   8 = a copy pair with an id outside [0, num_blocks) or src == dst (skipped)
+ *  32 = query rows of a sequence out of order or more than its length (rows -> zeros)
  *
  * Element types: 0 = IEEE fp32, 1 = bf16 (the upper 16 bits of an fp32; its
  * widening to fp32 is exact).
@@ -146,6 +147,85 @@ int oracle_paged_decode(double *out, const void *q, const void *k_cache, const v
                 o[d] /= denom;
             free(x);
         }
+    }
+    return err;
+}
+
+/*
+ * Several query tokens per sequence (a chunk of a prompt, or tokens checked
+ * together), each seeing the cache up to its own position.  The cache grows
+ * by the chunk's tokens ("vLLM Solved the Wrong Bottleneck...", section
+ * "Paged Attention") before they attend, and the chunk is the last
+ * Q = query_start[s+1] - query_start[s] of the n = context_lens[s] cached
+ * tokens, so query row j of sequence s (global row query_start[s] + j) sits
+ * at position p = n - Q + j and attends to tokens 0..p only (causal):
+ *
+ *   out[r][h][:] = sum_{i<=p} exp(x_i - m) V_i / sum_{i<=p} exp(x_i - m),
+ *   x_i = scale * q[r][h] . K_i,  m = max_{i<=p} x_i.
+ *
+ * A sequence whose query_start pair is out of order, or whose Q exceeds n,
+ * gets zero rows and error bit 32; the checks of oracle_paged_decode apply
+ * to n and the table as well.  q and out are [query_start[S]][Hq][D].
+ */
+int oracle_paged_prefill(double *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, const int32_t *context_lens,
+                         const int32_t *query_start, int num_seqs, int num_query_tokens,
+                         int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                         int max_blocks_per_seq, int num_blocks, int max_context_len,
+                         double scale, int dtype)
+{
+    const int group = num_q_heads / num_kv_heads;
+    int err = 0;
+    for (size_t i = 0; i < (size_t)num_query_tokens * num_q_heads * head_dim; ++i)
+        out[i] = 0.0;
+#pragma omp parallel for schedule(dynamic) reduction(| : err)
+    for (int s = 0; s < num_seqs; ++s) {
+        const int r0 = query_start[s], r1 = query_start[s + 1];
+        const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
+        const int n = context_lens[s];
+        if (r0 < 0 || r1 < r0 || r1 > num_query_tokens) {
+            err |= 32;
+            continue;
+        }
+        int bad = check_seq(table, n, num_blocks, block_size, max_blocks_per_seq,
+                            max_context_len);
+        if (!bad && r1 - r0 > n)
+            bad = 32;
+        if (bad) {
+            err |= bad;
+            continue;
+        }
+        const int Q = r1 - r0;
+        double *x = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        for (int j = 0; j < Q; ++j) {
+            const int p = n - Q + j;  /* position of this query token */
+            for (int h = 0; h < num_q_heads; ++h) {
+                const int g = h / group;
+                const size_t qoff = ((size_t)(r0 + j) * num_q_heads + h) * head_dim;
+                double *o = out + qoff;
+                double m = -INFINITY;
+                for (int i = 0; i <= p; ++i) {
+                    size_t ro = row_offset(table, i, g, num_kv_heads, block_size, head_dim);
+                    double dot = 0.0;
+                    for (int d = 0; d < head_dim; ++d)
+                        dot += elem(q, qoff + d, dtype) * elem(k_cache, ro + d, dtype);
+                    x[i] = scale * dot;
+                    if (x[i] > m)
+                        m = x[i];
+                }
+                double denom = 0.0;
+                for (int i = 0; i <= p; ++i) {
+                    double w = exp(x[i] - m);
+                    denom += w;
+                    size_t ro = row_offset(table, i, g, num_kv_heads, block_size, head_dim);
+                    for (int d = 0; d < head_dim; ++d)
+                        o[d] += w * elem(v_cache, ro + d, dtype);
+                }
+                for (int d = 0; d < head_dim; ++d)
+                    o[d] /= denom;
+            }
+        }
+        free(x);
     }
     return err;
 }
