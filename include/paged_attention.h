@@ -68,6 +68,8 @@ typedef enum pa_dtype {
                                      src == dst: skipped                                  */
 #define PA_ERRBIT_TIMEOUT     16  /* a bounded device wait ran out; results are invalid and
                                      the decode workspace must be re-initialised           */
+#define PA_ERRBIT_QUERY       32  /* pa_prefill: a sequence's query_start pair out of order
+                                     or more query rows than tokens: its rows written as 0 */
 
 /* Human-readable name of a status code (static storage). */
 const char *pa_status_str(pa_status status);
@@ -221,6 +223,42 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                            int max_blocks_per_seq, int num_blocks, int max_context_len,
                            float scale, int partition_size, pa_dtype dtype, void *workspace,
                            size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Several query tokens per sequence (chunked prefill, checked drafts)
+ * ------------------------------------------------------------------------
+ * A chunk of a prompt is attended to like decode tokens, each seeing the
+ * cache up to its own position.  The chunk's K/V must already be in the
+ * cache (pa_reshape_and_cache), since the cache grows by every token before
+ * it attends ("vLLM Solved the Wrong Bottleneck...", section "Paged
+ * Attention").  For sequence s with n = context_lens[s] cached tokens and
+ * Q = query_start[s+1] - query_start[s] query rows, query row j (global row
+ * r = query_start[s] + j) is the token at position p = n - Q + j:
+ *     out[r][h][:] = softmax_i(scale * q[r][h] . K_i) . V_i  over i = 0..p
+ * with K_i, V_i of KV head h / (num_q_heads / num_kv_heads), found through
+ * block_tables[s] as in pa_decode.
+ *
+ *   q, out          device, [num_query_tokens][num_q_heads][head_dim].
+ *   query_start     device int32 [num_seqs + 1], non-decreasing, from 0 to
+ *                   num_query_tokens; Q <= n for every sequence.  A
+ *                   sequence that breaks this gets zero rows and
+ *                   PA_ERRBIT_QUERY.
+ *   workspace       pa_decode_workspace_size(num_query_tokens, ...) bytes,
+ *                   zero-filled before first use, as for pa_decode.
+ *   Everything else is as in pa_decode.  Query rows are independent work
+ *   items to the decode kernel (grouped with the other query heads of their
+ *   KV head, on the tensor cores for bf16 groups of 8), so each row reads
+ *   its own prefix of the cache.  Launch-time shared memory grows with
+ *   num_query_tokens (12 bytes per row); too many rows for one SM's
+ *   shared memory returns PA_ERR_UNSUPPORTED.
+ */
+pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, const int32_t *context_lens,
+                     const int32_t *query_start, int num_seqs, int num_query_tokens,
+                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                     int partition_size, pa_dtype dtype, void *workspace,
+                     size_t workspace_bytes, int32_t *err_flag, void *stream);
 
 /* ------------------------------------------------------------------------
  * Block copy-on-write (copy_blocks)

@@ -32,6 +32,7 @@ static_assert(pa::kErrContextLen == PA_ERRBIT_CONTEXT_LEN, "error bit mismatch")
 static_assert(pa::kErrSlot == PA_ERRBIT_SLOT, "error bit mismatch");
 static_assert(pa::kErrPair == PA_ERRBIT_PAIR, "error bit mismatch");
 static_assert(pa::kErrTimeout == PA_ERRBIT_TIMEOUT, "error bit mismatch");
+static_assert(pa::kErrQuery == PA_ERRBIT_QUERY, "error bit mismatch");
 
 namespace {
 
@@ -166,8 +167,11 @@ pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, in
   return PA_OK;
 }
 
+// table_rows >= 0: several query tokens per sequence; num_seqs counts query
+// rows and the kernel also keeps their table rows and query_start on chip.
 pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                    int max_context_len, int partition_size, pa_dtype dtype, DecodePlan* p) {
+                    int max_context_len, int partition_size, pa_dtype dtype, DecodePlan* p,
+                    int table_rows = -1) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -183,7 +187,9 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 
   DeviceInfo dev;
   if ((st = device_info(&dev)) != PA_OK) return st;
-  const size_t seq_bytes = round_up((2 * static_cast<size_t>(num_seqs) + 1) * sizeof(int), 16);
+  const size_t seq_ints = 2 * static_cast<size_t>(num_seqs) + 1 +
+                          (table_rows >= 0 ? static_cast<size_t>(num_seqs) + table_rows + 1 : 0);
+  const size_t seq_bytes = round_up(seq_ints * sizeof(int), 16);
   p->smem = static_cast<size_t>(p->kernel.cta_bytes) + seq_bytes;
   if (p->smem > static_cast<size_t>(dev.smem_optin)) return PA_ERR_UNSUPPORTED;
   int occ = 0;
@@ -276,13 +282,15 @@ pa_status pa_decode_launch_config(int num_seqs, int num_q_heads, int num_kv_head
 namespace {
 
 // pa_decode and pa_decode_append: key/value null = plain decode.
+// query_start non-null: num_seqs counts query rows of table_rows sequences.
 pa_status decode_impl(void* out, const void* q, const void* key, const void* value,
                       const void* k_cache, const void* v_cache, const int32_t* block_tables,
                       const int32_t* context_lens, int num_seqs, int num_q_heads,
                       int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
                       int num_blocks, int max_context_len, float scale, int partition_size,
                       pa_dtype dtype, void* workspace, size_t workspace_bytes,
-                      int32_t* err_flag, void* stream) {
+                      int32_t* err_flag, void* stream, const int32_t* query_start = nullptr,
+                      int table_rows = -1) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -294,11 +302,12 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
     return PA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID_ARG;
+  if (query_start && table_rows <= 0) return PA_ERR_INVALID_ARG;
   if (static_cast<long long>(num_seqs) * num_kv_heads * max_blocks_per_seq >= (1LL << 31))
     return PA_ERR_UNSUPPORTED;
   DecodePlan p;
   if ((st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                      partition_size, dtype, &p)) != PA_OK)
+                      partition_size, dtype, &p, query_start ? table_rows : -1)) != PA_OK)
     return st;
   if (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace))
     return PA_ERR_WORKSPACE;
@@ -329,6 +338,8 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   args.ws_o = reinterpret_cast<float*>(ws + p.o_off);
   args.ws_ml = reinterpret_cast<float2*>(ws + p.ml_off);
   args.err_flag = err_flag;
+  args.query_start = query_start;
+  args.num_table_rows = query_start ? table_rows : num_seqs;
   if (p.kernel.tma) {
     // tile coordinates are 32-bit: row (block * Hkv + kv head) * 16 of the 2-D view
     const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
@@ -393,6 +404,22 @@ pa_status pa_decode_append(void* out, const void* q, const void* key, const void
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                      num_blocks, max_context_len, scale, partition_size, dtype, workspace,
                      workspace_bytes, err_flag, stream);
+}
+
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, const int32_t* context_lens,
+                     const int32_t* query_start, int num_seqs, int num_query_tokens,
+                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                     int partition_size, pa_dtype dtype, void* workspace,
+                     size_t workspace_bytes, int32_t* err_flag, void* stream) {
+  if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_query_tokens == 0) return PA_OK;
+  if (num_seqs == 0 || !query_start) return PA_ERR_INVALID_ARG;
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens,
+                     num_query_tokens, num_q_heads, num_kv_heads, head_dim, block_size,
+                     max_blocks_per_seq, num_blocks, max_context_len, scale, partition_size,
+                     dtype, workspace, workspace_bytes, err_flag, stream, query_start, num_seqs);
 }
 
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

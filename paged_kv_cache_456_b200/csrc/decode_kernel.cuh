@@ -291,8 +291,9 @@ constexpr int kEnd = 1 << 27;    // no more tiles: the partner warp stops
 constexpr int kAppend = 1 << 28; // fused append: the tile's last live row is the new token
 
 __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
-                                               const int* s_len, const Ranges& rg,
-                                               const OwnRanges& own, const DecodeArgs& a) {
+                                               const int* s_len, const int* s_row,
+                                               const Ranges& rg, const OwnRanges& own,
+                                               const DecodeArgs& a) {
   StageDesc d{0, 0, 0, 0};
   if (g >= hi) return d;
   // largest s with s_start[s] <= g (sequences without blocks share their start)
@@ -311,7 +312,8 @@ __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const 
   int flags = 0;
   if (g == item_a || own.is_start(g, rg)) flags |= kFirst;
   if (g + 1 == item_a + nb || own.is_start(g + 1, rg)) flags |= kLast;
-  int phys = __ldg(a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + blk);
+  const int trow = s_row ? s_row[s] : s;  // (query rows share their sequence's table)
+  int phys = __ldg(a.block_tables + static_cast<size_t>(trow) * a.max_blocks_per_seq + blk);
   if (phys < 0 || phys >= a.num_blocks) {
     flags |= kBad;
     phys = 0;
@@ -393,6 +395,10 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   const uint32_t empty0 = full0 + 8 * DEPTH;
   int* s_start = reinterpret_cast<int*>(sbase + WORKERS * C::WORKER_BYTES);  // [S + 1]
   int* s_len = s_start + S + 1;                                              // [S]
+  // several query tokens per sequence: table row of each query row, query_start
+  const bool prefill = a.query_start != nullptr;
+  int* s_row = prefill ? s_len + S : nullptr;                                // [S]
+  int* s_qs = s_len + 2 * S;                                                 // [rows + 1]
 
   if (leader && lane == 0) {
 #pragma unroll
@@ -403,6 +409,34 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     fence_barrier_init();
   }
 
+  // Tokens sequence s attends to, or minus the error bit that empties it.
+  // Decode: context_lens[s].  Several query tokens per sequence: s is a query
+  // row; its sequence (row of the block table) is found in query_start, and
+  // query j of a sequence of n tokens and Q queries sees n - Q + j + 1 tokens.
+  auto attended = [&](int s, int& row) -> int {
+    if (!prefill) {
+      row = s;
+      const int n = a.context_lens[s];
+      return (n < 0 || n > a.len_cap) ? -kErrContextLen : n;
+    }
+    int lo = 0, up = a.num_table_rows - 1;  // largest row with query_start[row] <= s
+    while (lo < up) {
+      const int mid = (lo + up + 1) >> 1;
+      if (s_qs[mid] <= s) lo = mid; else up = mid - 1;
+    }
+    row = lo;
+    const int q0 = s_qs[lo], q1 = s_qs[lo + 1];
+    if (!(q0 <= s && s < q1)) return -kErrQuery;
+    const int n = a.context_lens[lo];
+    if (n < 0 || n > a.len_cap) return -kErrContextLen;
+    if (q1 - q0 > n) return -kErrQuery;
+    return n - (q1 - q0) + (s - q0) + 1;
+  };
+  if (prefill) {
+    for (int i = tid; i <= a.num_table_rows; i += WARPS * 32) s_qs[i] = a.query_start[i];
+    __syncthreads();
+  }
+
   // ---- prologue: block counts and their prefix sums, in tiles ----------------
   {
     const int per = (S + WARPS * 32 - 1) / (WARPS * 32);
@@ -410,9 +444,11 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     const int s1 = min(S, s0 + per);
     int local = 0;
     for (int s = s0; s < s1; ++s) {
-      int n = a.context_lens[s];
-      if (n < 0 || n > a.len_cap) n = 0;
+      int row;
+      int n = attended(s, row);
+      if (n < 0) n = 0;
       s_len[s] = n;
+      if (prefill) s_row[s] = row;
       local += (n + kBlockSize - 1) / kBlockSize;
     }
     int incl = local;
@@ -443,8 +479,9 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   for (int s = blockIdx.x; s < S; s += gridDim.x) {
     if (s_len[s] != 0) continue;
     if (tid == 0 && a.err_flag) {
-      const int n = a.context_lens[s];
-      if (n < 0 || n > a.len_cap) atomicOr(a.err_flag, kErrContextLen);
+      int row;
+      const int n = attended(s, row);
+      if (n < 0) atomicOr(a.err_flag, -n);
     }
     uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(a.out) +
                                           static_cast<size_t>(s) * Hq * C::ROW);
@@ -497,7 +534,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   int known = n0;                      // positions with a tile assigned
   bool no_more = rg.R == rg.Rs;        // no chunks left to claim
   auto static_desc = [&](int p) -> StageDesc {
-    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, rg, own, a) : StageDesc{0, 0, 0, 0};
+    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, s_row, rg, own, a) : StageDesc{0, 0, 0, 0};
   };
   StageDesc A{0, 0, 0, 0}, B{0, 0, 0, 0};
   int base = 0;
@@ -517,8 +554,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     const long long g0 = rg.Ws + static_cast<long long>(c) * rg.CS;
     const int len = static_cast<int>(rg.CS < W - g0 ? rg.CS : W - g0);
     const int pa = base + lane, pb = base + 32 + lane;
-    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, rg, own, a);
-    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, rg, own, a);
+    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, s_row, rg, own, a);
+    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, s_row, rg, own, a);
     known += len;
   };
   auto top_up = [&](int frontier) {

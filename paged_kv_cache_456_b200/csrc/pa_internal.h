@@ -17,6 +17,7 @@ constexpr int kErrContextLen = 2;
 constexpr int kErrSlot = 4;
 constexpr int kErrPair = 8;
 constexpr int kErrTimeout = 16;
+constexpr int kErrQuery = 32;
 
 // Work schedule: the last 1/kTailDiv of the tiles is handed out at run time
 // in chunks of kChunkTiles (0 = everything static).
@@ -64,6 +65,11 @@ struct DecodeArgs {
   float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
   float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
   int32_t* err_flag;
+  // several query tokens per sequence (null for decode): the kernel's
+  // "sequences" are then the num_seqs query rows, each attending causally;
+  // query_start[num_table_rows + 1] maps them to the block-table rows
+  const int32_t* query_start;
+  int num_table_rows;
   // tensor-core path only: the caches as 2-D tensors [num_blocks * Hkv * 16][head_dim]
   // read in boxes of 16 rows x 128 bytes with the 128-byte swizzle
   CUtensorMap tm_k;

@@ -25,10 +25,11 @@ ERRBIT_CONTEXT_LEN = 2
 ERRBIT_SLOT = 4
 ERRBIT_PAIR = 8
 ERRBIT_TIMEOUT = 16
+ERRBIT_QUERY = 32
 
 EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_init",
             "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_decode_append",
-            "pa_reshape_and_cache", "pa_copy_blocks")
+            "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks")
 
 # size of the library's fixed scratch array used by pa_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -65,6 +66,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode.restype = i
     lib.pa_decode_noalloc.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, vp]
+    lib.pa_prefill.restype = i
+    lib.pa_prefill.argtypes = [vp] * 7 + [i] * 9 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode_append.restype = i
     lib.pa_decode_append.argtypes = [vp] * 8 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode_noalloc.restype = i
@@ -174,6 +177,24 @@ def decode_append(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor, value: 
         int(max_context_len), float(scale), int(partition_size), _dtype_code(q), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream)),
         "pa_decode_append")
+    return out
+
+
+def prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+            block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor, *,
+            scale: float, max_context_len: int, workspace: torch.Tensor, partition_size: int = 0,
+            err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Causal attention of ``q`` ``[T][Hq][D]``, the last ``query_start[s+1] -
+    query_start[s]`` tokens of each sequence, into ``out``; see ``pa_prefill``.
+    The workspace is sized for ``T`` query rows (``make_workspace(T, ...)``)."""
+    T, Hq, D = q.shape
+    N, Hkv, bs, _ = k_cache.shape
+    _check(library().pa_prefill(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        _ptr(query_start), block_tables.shape[0], T, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        int(max_context_len), float(scale), int(partition_size), _dtype_code(q),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err_flag),
+        _stream(stream)), "pa_prefill")
     return out
 
 

@@ -95,6 +95,17 @@ def test_fused_append_rejects_bad_arguments_on_the_host(lib):
     assert call(key=None, value=None, S=0) == ops.PA_OK            # nothing to do
 
 
+def test_prefill_rejects_bad_arguments_on_the_host(lib):
+    def call(qs=P(16), S=2, T=5, Hq=8):
+        return lib.pa_prefill(P(16), P(16), P(16), P(16), P(16), P(16), qs, S, T, Hq, 2, 128, 16,
+                              4, 10, 64, 0.1, 0, ops.PA_BF16, P(16), 1 << 20, None, None)
+    assert call(qs=None) == ops.PA_ERR_INVALID_ARG
+    assert call(S=0) == ops.PA_ERR_INVALID_ARG           # query rows but no sequence
+    assert call(T=-1) == ops.PA_ERR_INVALID_ARG
+    assert call(Hq=6) == ops.PA_ERR_UNSUPPORTED          # group 3
+    assert call(qs=None, T=0) == ops.PA_OK               # nothing to do
+
+
 def test_workspace_queries_validate_first(lib):
     n = ctypes.c_size_t(0)
     assert lib.pa_decode_workspace_size(2, 8, 2, 96, 64, 0, ops.PA_BF16, ctypes.byref(n)) == \

@@ -1,0 +1,97 @@
+"""Several query tokens per sequence (pa_prefill) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_456_b200 import ops
+from paged_kv_cache_456_b200.workloads import upload
+
+from tests.test_gpu_parity import SHAPES, assert_attention_close
+from tests.test_oracle_prefill import prefill_case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_cache_456_b200 import build
+    build.build()
+    ops.library()
+
+
+def run_prefill(w, q, qs, psize=0, t=None, qs_dev=None):
+    t = t if t is not None else upload(w)
+    tdt = t["q"].dtype
+    qd = torch.from_numpy(np.ascontiguousarray(q))
+    qd = (qd.view(torch.bfloat16) if w.dtype == "bf16" else qd).cuda()
+    out = torch.full(qd.shape, 7.0, dtype=tdt, device="cuda")
+    qs_dev = qs_dev if qs_dev is not None else torch.from_numpy(qs).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = ops.make_workspace(qd.shape[0], w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.max_context_len, psize, tdt)
+    ops.prefill(out, qd, t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"], qs_dev,
+                scale=w.scale, max_context_len=w.max_context_len, workspace=ws,
+                partition_size=psize, err_flag=err)
+    torch.cuda.synchronize()
+    return out, int(err.item()), t
+
+
+@pytest.mark.parametrize("dtype,D,G", SHAPES, ids=lambda x: str(x))
+@pytest.mark.parametrize("psize", [0, 16, 512])
+def test_prefill_matches_the_oracle(dtype, D, G, psize):
+    hkv = 2
+    w, q, qs = prefill_case(300 + D + G, dtype=dtype, num_q_heads=hkv * G, num_kv_heads=hkv,
+                            head_dim=D, lens=(40, 17, 1, 700, 33, 16),
+                            queries=(5, 17, 1, 40, 0, 16))
+    ref, oerr = oracle.paged_prefill(q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens, qs,
+                                     scale=w.scale, dtype=w.dtype)
+    out, err, _ = run_prefill(w, q, qs, psize)
+    assert err == 0 and oerr == 0
+    assert_attention_close(out, ref, dtype, f"prefill {dtype} D{D} G{G} P{psize}")
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_one_query_per_sequence_is_decode_bit_for_bit(G):
+    w, q, qs = prefill_case(5, dtype="bf16", num_q_heads=2 * G, num_kv_heads=2, head_dim=128,
+                            lens=(40, 17, 300, 64), queries=(1, 1, 1, 1))
+    out, err, t = run_prefill(w, q, qs)
+    assert err == 0
+    ws = ops.make_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.max_context_len, 0, torch.bfloat16)
+    dec = torch.empty_like(out)
+    qd = torch.from_numpy(np.ascontiguousarray(q)).view(torch.bfloat16).cuda()
+    ops.decode(dec, qd, t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+               scale=w.scale, max_context_len=w.max_context_len, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), dec.view(torch.int16))
+
+
+def test_long_chunks_of_a_large_batch():
+    """8 sequences of ~1-2K tokens, each with a 64-token chunk: 512 query rows."""
+    rng = np.random.default_rng(6)
+    lens = tuple(int(x) for x in rng.integers(900, 2100, size=8))
+    for G in (1, 8):
+        w, q, qs = prefill_case(7 + G, dtype="bf16", num_q_heads=4 * G, num_kv_heads=4,
+                                head_dim=128, lens=lens, queries=(64,) * 8)
+        ref, _ = oracle.paged_prefill(q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens, qs,
+                                      scale=w.scale, dtype=w.dtype)
+        out, err, _ = run_prefill(w, q, qs)
+        assert err == 0
+        assert_attention_close(out, ref, "bf16", f"chunks of 64, G{G}")
+
+
+def test_bad_query_rows_zero_that_sequence_only():
+    w, q, qs = prefill_case(8, dtype="f32", lens=(40, 17, 30), queries=(5, 9, 3))
+    bad = qs.copy()
+    bad[2] = bad[1] + 18                # 18 rows for a 17-token sequence
+    bad[3] = bad[2] + 3
+    q2 = np.resize(q, (int(bad[-1]),) + q.shape[1:])
+    ref, oerr = oracle.paged_prefill(q2, w.k_pool, w.v_pool, w.tables_compact, w.context_lens,
+                                     bad, scale=w.scale, dtype=w.dtype)
+    out, err, _ = run_prefill(w, q2, bad)
+    assert err == ops.ERRBIT_QUERY == oerr
+    assert (out[5:23] == 0).all()
+    assert_attention_close(out, ref, "f32", "rows around the bad sequence")
