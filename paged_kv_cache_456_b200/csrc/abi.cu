@@ -81,8 +81,8 @@ struct DecodePlan {
   long long ranges = 0;      // most ranges the device can form
   int sms = 0;
   // workspace layout; everything before zero_bytes must be zero on entry
-  size_t heavy_off = 0;      // [4] ints: merge-pass items, merge CTAs done, chunks, workers done
-  size_t list_off = 0;       // [S*Hkv] ints: items for the merge pass
+  size_t heavy_off = 0;      // [8] ints: merge-pass counts, merge CTAs done, chunks, workers done
+  size_t list_off = 0;       // 2 x [S*Hkv] ints: items for the merge pass (many, few pieces)
   size_t counters_off = 0;   // [S*Hkv*2] ints
   size_t zero_bytes = 0;
   size_t seq_start_off = 0;  // [S + 1] ints
@@ -215,10 +215,10 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   const size_t items = static_cast<size_t>(num_seqs) * num_kv_heads;
   // zero-on-entry fields first: the merge pass's count/done pair, the piece counters
   p->heavy_off = 0;
-  p->counters_off = 4 * sizeof(int);
+  p->counters_off = 8 * sizeof(int);
   p->zero_bytes = pa::decode_zero_prefix_bytes(num_seqs, num_kv_heads);
   p->list_off = p->zero_bytes;
-  p->seq_start_off = round_up(p->list_off + items * sizeof(int), 16);
+  p->seq_start_off = round_up(p->list_off + 2 * items * sizeof(int), 16);
   p->o_off = round_up(p->seq_start_off + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
   p->ml_off = round_up(p->o_off + slots * group * head_dim * sizeof(float), 256);
   p->ws_bytes = round_up(p->ml_off + slots * group * 2 * sizeof(float), 256);
@@ -228,7 +228,7 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 }  // namespace
 
 size_t pa::decode_zero_prefix_bytes(int num_seqs, int num_kv_heads) {
-  return 4 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
+  return 8 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
 }
 
 extern "C" {
@@ -335,6 +335,7 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   args.seq_start = reinterpret_cast<int*>(ws + p.seq_start_off);
   args.heavy = reinterpret_cast<int*>(ws + p.heavy_off);
   args.heavy_list = reinterpret_cast<int*>(ws + p.list_off);
+  args.light_list = args.heavy_list + static_cast<size_t>(num_seqs) * num_kv_heads;
   args.ws_o = reinterpret_cast<float*>(ws + p.o_off);
   args.ws_ml = reinterpret_cast<float2*>(ws + p.ml_off);
   args.err_flag = err_flag;

@@ -517,6 +517,14 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   float* xs = reinterpret_cast<float*>(aux);
   float* alpha_s = reinterpret_cast<float*>(aux + C::XS);
   StageDesc* ring_desc = reinterpret_cast<StageDesc*>(wkbase + C::DESC_OFF);
+  // an item for the merge pass: few pieces go to its one-warp list, more to
+  // its one-CTA-per-head list
+  auto list_for_merge = [&](long long pieces, int item) {
+    if (pieces <= kWarpMergeMaxPieces)
+      a.light_list[atomicAdd(a.heavy + 4, 1)] = item;
+    else
+      a.heavy_list[atomicAdd(a.heavy, 1)] = item;
+  };
 
   const int dl = lane % C::LPR;  // which 16 bytes of a row
   const int rgp = lane / C::LPR; // which row group
@@ -1018,7 +1026,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           a.ws_ml[sl * GT + h0 + 1] = make_float2(mh[1], bad ? -1.f : lt[1]);
         }
         // the merge pass combines the pieces; the first piece lists the item
-        if (r == ra && lane == 0) a.heavy_list[atomicAdd(a.heavy, 1)] = s * Hkv + kvh;
+        if (r == ra && lane == 0) list_for_merge(rb - ra + 1, s * Hkv + kvh);
       }
     } else if (flags & kLast) {
 #pragma unroll
@@ -1071,8 +1079,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
         if (heavy) {
           // many pieces: the merge pass combines them; the first piece lists the item
           if (r == ra && lane == 0 && half == 0) {
-            const int idx = atomicAdd(a.heavy, 1);
-            a.heavy_list[idx] = s * Hkv + kvh;
+            list_for_merge(rb - ra + 1, s * Hkv + kvh);
           }
         } else {
           __threadfence();
@@ -1162,7 +1169,8 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
 
   const int tid = threadIdx.x, grp = tid >> 5, lane = tid & 31;
   const int S = a.num_seqs, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
-  const int count = __ldcg(a.heavy);
+  const int count = __ldcg(a.heavy);        // items of many pieces
+  const int light = __ldcg(a.heavy + 4);    // items of few pieces
   const long long W = __ldcg(a.seq_start + S);
   if (W > 0) {
     const Ranges rg = make_ranges(W, workers, a.part_blocks);
@@ -1173,15 +1181,14 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
     constexpr int VPL = D / LPH;  // values per lane
     constexpr int NP = kWarpMergeMaxPieces;
     const int hw = lane / LPH, d0 = (lane % LPH) * VPL;
-    for (int it = blockIdx.x * GROUPS + grp; it < count; it += gridDim.x * GROUPS) {
-      const int item = __ldcg(a.heavy_list + it);
+    for (int it = blockIdx.x * GROUPS + grp; it < light; it += gridDim.x * GROUPS) {
+      const int item = __ldcg(a.light_list + it);
       const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
       const int st = __ldcg(a.seq_start + s);
       const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
       const long long item_a = st + static_cast<long long>(kvh) * nb;
       const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
-      const int np = static_cast<int>(rb - ra + 1);
-      if (np > NP) continue;
+      const int np = static_cast<int>(rb - ra + 1);  // (at most NP: listed so)
       long long sl[NP];
       float2 ml[NP];
       float M = -INFINITY;
@@ -1228,7 +1235,6 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
       const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
       const long long item_a = st + static_cast<long long>(kvh) * nb;
       const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
-      if (rb - ra + 1 <= kWarpMergeMaxPieces) continue;  // (the same for the whole CTA)
 
       float M = -INFINITY;
       int bad = 0;
@@ -1290,6 +1296,7 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   if (tid == 0 && atomicAdd(a.heavy + 1, 1) == static_cast<int>(gridDim.x) - 1) {
     a.heavy[0] = 0;
     a.heavy[1] = 0;
+    a.heavy[4] = 0;
   }
 }
 

@@ -59,9 +59,11 @@ struct DecodeArgs {
   int* counters;     // [num_seqs * num_kv_heads * 2] pieces finished per (item, head half),
                      // zero between calls
   int* seq_start;    // [num_seqs + 1] first tile of each sequence (written for the merge pass)
-  int* heavy;        // [4]: items listed for the merge pass, merge CTAs done, tail chunks
-                     // claimed, decode workers done (all zero between calls)
-  int* heavy_list;   // [num_seqs * num_kv_heads] (seq * Hkv + kv head) of those items
+  int* heavy;        // [8]: items of many pieces listed for the merge pass, merge CTAs
+                     // done, tail chunks claimed, decode workers done, items of few
+                     // pieces listed (all zero between calls)
+  int* heavy_list;   // [num_seqs * num_kv_heads] (seq * Hkv + kv head) of many-piece items
+  int* light_list;   // [num_seqs * num_kv_heads] the same for items of few pieces
   float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
   float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
   int32_t* err_flag;
