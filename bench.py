@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention: effective KV HBM GB/s (% of B200 peak); seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = ("paged_kv_cache_456_b200/csrc/decode_kernel.cuh",
                   "paged_kv_cache_456_b200/csrc/decode_bf16.cu",
@@ -64,13 +65,14 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-def measured_peaks():
+def measured_peaks(key: str = "hbm_gbs"):
+    fallback = {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}[key]
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d[key]), "measured"
     except (OSError, KeyError, ValueError):
-        return FALLBACK_HBM_GBS, "fallback"
+        return fallback, "fallback"
 
 
 def kernel_source_hash() -> str:
@@ -166,6 +168,12 @@ class ClockSampler:
 def sub_workload(w, k: int):
     """The first k sequences of a workload (same pool, same copy pairs)."""
     import dataclasses
+    if w.query_start is not None:
+        r = int(w.query_start[k])
+        return dataclasses.replace(
+            w, context_lens=w.context_lens[:k], tables_compact=w.tables_compact[:k], q=w.q[:r],
+            query_start=w.query_start[:k + 1], new_key=w.new_key[:r], new_value=w.new_value[:r],
+            slot_mapping_compact=w.slot_mapping_compact[:r])
     return dataclasses.replace(
         w, context_lens=w.context_lens[:k], tables_compact=w.tables_compact[:k], q=w.q[:k],
         new_key=None if w.new_key is None else w.new_key[:k],
@@ -267,9 +275,11 @@ def run_ours(args, rank: int, world: int):
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     tdt = t["q"].dtype
     ps = w.partition_size
-    ws = ops.make_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+    prefill = "query_start" in t     # several query tokens per sequence
+    rows = t["q"].shape[0]            # query rows: one per sequence in decode
+    ws = ops.make_workspace(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
                             w.max_context_len, ps, tdt, device=dev)
-    cfg = ops.launch_config(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+    cfg = ops.launch_config(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
                             w.max_context_len, ps, tdt)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     evict = torch.ones(128 << 20, dtype=torch.int32, device=dev)   # 512 MiB, read only
@@ -277,7 +287,7 @@ def run_ours(args, rank: int, world: int):
     def flush_l2():
         flush.fill_(1)
         evict.sum()     # the read pushes the dirty lines of the write out of L2
-    fused = "key" in t and args.append == "fused"
+    fused = "key" in t and args.append == "fused" and not prefill
     # decode is two kernels (the attention pass and the merge pass behind it)
     launches_per_step = 2 + ("key" in t and not fused) + ("block_mapping" in t)
 
@@ -289,7 +299,12 @@ def run_ours(args, rank: int, world: int):
                                   t["slot_mapping"], err_flag=err)
         if ev_mid is not None:
             ev_mid.record(stream)
-        if fused:
+        if prefill:
+            ops.prefill(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                        t["context_lens"], t["query_start"], scale=w.scale,
+                        max_context_len=w.max_context_len, workspace=ws, partition_size=ps,
+                        err_flag=err)
+        elif fused:
             ops.decode_append(t["out"], t["q"], t["key_seq"], t["value_seq"], t["k_cache"],
                               t["v_cache"], t["block_tables"], t["context_lens"], scale=w.scale,
                               max_context_len=w.max_context_len, workspace=ws,
@@ -366,6 +381,18 @@ def run_ours(args, rank: int, world: int):
         "launch": cfg,
         "clocks": clocks.summary(),
     }
+    if prefill:
+        # many query rows re-read their sequence's prefix (from L2): the attention
+        # kernel is set against the tensor roofline, by its attention FLOPs
+        fl = w.attention_flops()
+        tpk, tkind = measured_peaks("bf16_tflops")
+        tf = fl / (dec_avg * 1e-3) / 1e12
+        line["roofline"].update({"bound": "tensor", "achieved": round(tf, 2), "peak": tpk,
+                                 "unit": "TFLOP/s", "frac": round(tf / tpk, 4),
+                                 "peak_source": f"{tkind} bf16_tflops (burst cuBLAS GEMM)",
+                                 "algorithmic_flops_per_launch": fl,
+                                 "hbm_view_gbs": round(achieved, 2)})
+        line["query_rows"] = rows
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, dt, k, nb, threads = oracle_sample(w, budget_s=10.0, repeat=True, fused=fused)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
@@ -388,7 +415,8 @@ def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused):
     from paged_kv_cache_456_b200 import ops
 
     step_inputs = ("q", "key_seq", "value_seq") if fused else ("q", "key", "value", "slot_mapping")
-    names = [n for n in step_inputs + ("block_tables", "context_lens", "block_mapping") if n in t]
+    names = [n for n in step_inputs + ("block_tables", "context_lens", "block_mapping",
+                                       "query_start") if n in t]
     # one pinned staging buffer holding every input, 256-byte aligned pieces
     offs, size = {}, 0
     for n in names:
@@ -428,7 +456,12 @@ def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused):
         if "key" in d:
             ops.reshape_and_cache(d["key"], d["value"], t["k_cache"], t["v_cache"],
                                   d["slot_mapping"], err_flag=err, stream=stream)
-        if fused:
+        if "query_start" in d:
+            ops.prefill(out[b], d["q"], t["k_cache"], t["v_cache"], d["block_tables"],
+                        d["context_lens"], d["query_start"], scale=w.scale,
+                        max_context_len=w.max_context_len, workspace=ws, partition_size=ps,
+                        err_flag=err, stream=stream)
+        elif fused:
             ops.decode_append(out[b], d["q"], d["key_seq"], d["value_seq"], t["k_cache"],
                               t["v_cache"], d["block_tables"], d["context_lens"], scale=w.scale,
                               max_context_len=w.max_context_len, workspace=ws,

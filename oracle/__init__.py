@@ -170,6 +170,10 @@ def workload_step(w, partition_size: int = 0, lib: Optional[ctypes.CDLL] = None)
         err |= copy_blocks(k, v, w.block_mapping_compact, lib=lib)
     if w.new_key is not None:
         err |= reshape_and_cache(k, v, w.new_key, w.new_value, w.slot_mapping_compact, lib=lib)
-    out, e = paged_decode(w.q, k, v, w.tables_compact, w.context_lens, scale=w.scale,
-                          dtype=w.dtype, partition_size=partition_size, lib=lib)
+    if getattr(w, "query_start", None) is not None:
+        out, e = paged_prefill(w.q, k, v, w.tables_compact, w.context_lens, w.query_start,
+                               scale=w.scale, dtype=w.dtype, lib=lib)
+    else:
+        out, e = paged_decode(w.q, k, v, w.tables_compact, w.context_lens, scale=w.scale,
+                              dtype=w.dtype, partition_size=partition_size, lib=lib)
     return out, k, v, err | e

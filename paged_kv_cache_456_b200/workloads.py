@@ -54,7 +54,7 @@ from .block_allocator import BlockAllocator, blocks_for_tokens
 BLOCK_SIZE = 16
 BF16_NAN_BITS = np.int16(0x7FC0)
 
-WORKLOAD_NAMES = ("tiny", "7b", "gqa70b", "prefix_cow", "long")
+WORKLOAD_NAMES = ("tiny", "7b", "gqa70b", "prefix_cow", "long", "prefill")
 
 
 # ---------------------------------------------------------------------------
@@ -118,6 +118,9 @@ class Workload:
     block_mapping_compact: Optional[np.ndarray] = None  # int32 [M][2] (src, dst)
     refcount: Optional[np.ndarray] = None        # physical refcounts after the build
     block_size: int = BLOCK_SIZE
+    # several query tokens per sequence: q is then [T][Hq][D], the query rows
+    # of sequence s are query_start[s] .. query_start[s+1]-1 (its last tokens)
+    query_start: Optional[np.ndarray] = None     # int32 [S + 1]
 
     # -- shapes ------------------------------------------------------------
     @property
@@ -169,11 +172,23 @@ class Workload:
 
     # -- algorithmic byte counts --------------------------------------------
     def decode_bytes(self) -> int:
-        """K and V of every live token plus q read and out written."""
+        """K and V of every live token (once) plus q read and out written."""
         eb = self.elem_bytes
         kv = int(self.context_lens.astype(np.int64).sum()) * 2 * self.num_kv_heads * self.head_dim * eb
-        qo = 2 * self.num_seqs * self.num_q_heads * self.head_dim * eb
+        qo = 2 * self.q.shape[0] * self.num_q_heads * self.head_dim * eb
         return kv + qo
+
+    def attention_flops(self) -> int:
+        """2 FLOP per multiply-add of q.K and of p.V, over every attended token."""
+        if self.query_start is None:
+            attended = int(self.context_lens.astype(np.int64).sum())
+        else:
+            attended = 0
+            for s in range(self.num_seqs):
+                n = int(self.context_lens[s])
+                Q = int(self.query_start[s + 1] - self.query_start[s])
+                attended += Q * (n - Q) + Q * (Q + 1) // 2
+        return 4 * attended * self.num_q_heads * self.head_dim
 
     def reshape_bytes(self) -> int:
         if self.new_key is None:
@@ -375,11 +390,51 @@ def _build_named(name: str, rng: np.random.Generator, pool: Optional[int]) -> Wo
         return make_workload(rng, name=name, dtype="bf16", num_q_heads=32, num_kv_heads=8,
                              head_dim=128, context_lens=lens, num_blocks=n(4096),
                              prefix_tokens=2048, cow_count=64)
+    if name == "prefill":
+        prior = exp_lengths(rng, 16)
+        return make_prefill_workload(rng, name=name, dtype="bf16", num_q_heads=64,
+                                     num_kv_heads=8, head_dim=128, prior_lens=prior, chunk=128,
+                                     num_blocks=n(4096))
     if name == "long":
         return make_workload(rng, name=name, dtype="bf16", num_q_heads=32, num_kv_heads=8,
                              head_dim=128, context_lens=[32768] * 8, num_blocks=n(16384),
                              partition_size=512)
     raise KeyError(name)
+
+
+def make_prefill_workload(rng: np.random.Generator, *, name: str, dtype: str,
+                          num_q_heads: int, num_kv_heads: int, head_dim: int,
+                          prior_lens: Sequence[int], chunk: int, num_blocks: int) -> Workload:
+    """Each sequence holds ``prior_lens[s]`` tokens and takes a chunk of
+    ``chunk`` more: the chunk's K/V is returned as new rows with their slots
+    (NaN in the pool until the slot write) and its ``chunk`` query rows attend
+    causally."""
+    prior = np.asarray(prior_lens, dtype=np.int32)
+    lens = prior + chunk
+    w = make_workload(rng, name=name, dtype=dtype, num_q_heads=num_q_heads,
+                      num_kv_heads=num_kv_heads, head_dim=head_dim, context_lens=lens,
+                      num_blocks=num_blocks)
+    S, T = len(lens), len(lens) * chunk
+    qs = (np.arange(S + 1) * chunk).astype(np.int32)
+    q32 = rng.standard_normal((T, num_q_heads, head_dim), dtype=np.float32)
+    q = _cast(q32, dtype)
+    slots = np.empty(T, dtype=np.int64)
+    new_key = np.empty((T, num_kv_heads, head_dim), dtype=w.k_pool.dtype)
+    new_value = np.empty_like(new_key)
+    nanv = _nan_value(dtype)
+    for s in range(S):
+        for j in range(chunk):
+            pos = int(lens[s]) - chunk + j
+            b, off = divmod(pos, BLOCK_SIZE)
+            c = int(w.tables_compact[s, b])
+            r = s * chunk + j
+            slots[r] = c * BLOCK_SIZE + off
+            new_key[r] = w.k_pool[c, :, off, :]
+            new_value[r] = w.v_pool[c, :, off, :]
+            w.k_pool[c, :, off, :] = nanv
+            w.v_pool[c, :, off, :] = nanv
+    return dataclasses.replace(w, q=q, query_start=qs, new_key=new_key, new_value=new_value,
+                               slot_mapping_compact=slots)
 
 
 def random_workload(seed: int, *, dtype: str = "bf16", num_seqs: int = 3,
@@ -417,16 +472,19 @@ def upload(w: Workload, device="cuda", pool: bool = True):
             full[idx] = elems(src).to(device)
             out[key] = full
     out["q"] = elems(w.q).to(device)
+    if w.query_start is not None:
+        out["query_start"] = torch.from_numpy(w.query_start).to(device)
     out["block_tables"] = torch.from_numpy(w.block_tables).to(device)
     out["context_lens"] = torch.from_numpy(w.context_lens).to(device)
     if w.new_key is not None:
         out["key"] = elems(w.new_key).to(device)
         out["value"] = elems(w.new_value).to(device)
         out["slot_mapping"] = torch.from_numpy(w.slot_mapping).to(device)
-        ks, vs = w.new_rows_per_sequence()
-        out["key_seq"] = elems(ks).to(device)
-        out["value_seq"] = elems(vs).to(device)
+        if w.query_start is None:
+            ks, vs = w.new_rows_per_sequence()
+            out["key_seq"] = elems(ks).to(device)
+            out["value_seq"] = elems(vs).to(device)
     if w.block_mapping_compact is not None:
         out["block_mapping"] = torch.from_numpy(w.block_mapping).to(device)
-    out["out"] = torch.empty((w.num_seqs, w.num_q_heads, w.head_dim), dtype=tdt, device=device)
+    out["out"] = torch.empty((w.q.shape[0], w.num_q_heads, w.head_dim), dtype=tdt, device=device)
     return out

@@ -95,3 +95,22 @@ def test_bad_query_rows_zero_that_sequence_only():
     assert err == ops.ERRBIT_QUERY == oerr
     assert (out[5:23] == 0).all()
     assert_attention_close(out, ref, "f32", "rows around the bad sequence")
+
+
+def test_prefill_workload_step():
+    """The benchmark's prefill step: the chunks' slot write, then pa_prefill."""
+    from paged_kv_cache_456_b200.workloads import build_workload
+    w = build_workload("prefill")
+    t = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.reshape_and_cache(t["key"], t["value"], t["k_cache"], t["v_cache"], t["slot_mapping"],
+                          err_flag=err)
+    ws = ops.make_workspace(t["q"].shape[0], w.num_q_heads, w.num_kv_heads, w.head_dim,
+                            w.max_context_len, 0, torch.bfloat16)
+    ops.prefill(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                t["context_lens"], t["query_start"], scale=w.scale,
+                max_context_len=w.max_context_len, workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    ref, _, _, oerr = oracle.workload_step(w)
+    assert err.item() == 0 and oerr == 0
+    assert_attention_close(t["out"], ref, "bf16", "prefill workload")

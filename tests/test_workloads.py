@@ -79,3 +79,21 @@ def test_lengths_of_the_big_workloads(name):
     idx = {"7b": 1, "gqa70b": 2}[name]
     lens = exp_lengths(np.random.default_rng(idx + 1), {"7b": 64, "gqa70b": 256}[name])
     assert lens.min() >= 100 and lens.max() <= 4096
+
+
+def test_prefill_workload_structure():
+    from paged_kv_cache_456_b200.workloads import bf16_bits_to_f32
+    w = build_workload("prefill")
+    S, T = w.num_seqs, w.q.shape[0]
+    assert (np.diff(w.query_start) == 128).all() and w.query_start[-1] == T == 128 * S
+    assert w.new_key.shape == (T, w.num_kv_heads, w.head_dim)
+    # the chunk's slots are the last 128 positions of each sequence, NaN until written
+    for s in (0, S - 1):
+        n = int(w.context_lens[s])
+        for j in (0, 127):
+            r = int(w.query_start[s]) + j
+            b, off = divmod(n - 128 + j, 16)
+            assert w.slot_mapping_compact[r] == int(w.tables_compact[s, b]) * 16 + off
+            assert np.isnan(bf16_bits_to_f32(w.k_pool[int(w.tables_compact[s, b]), :, off])).all()
+    assert w.attention_flops() == 4 * w.num_q_heads * w.head_dim * sum(
+        128 * (int(n) - 128) + 128 * 129 // 2 for n in w.context_lens)
