@@ -39,13 +39,13 @@ static bool fill(DecodeKernelInfo* info) {
 #define PA_G8_MMA 1
 #endif
 #ifndef PA_MMA_DEPTH
-#define PA_MMA_DEPTH 2
+#define PA_MMA_DEPTH 3
 #endif
 #ifndef PA_MMA_WARPS
-#define PA_MMA_WARPS 4
+#define PA_MMA_WARPS 2
 #endif
 #ifndef PA_MMA_MINCTAS
-#define PA_MMA_MINCTAS 2
+#define PA_MMA_MINCTAS 3
 #endif
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info) {

@@ -1171,16 +1171,15 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   const int S = a.num_seqs, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
   const int count = __ldcg(a.heavy);        // items of many pieces
   const int light = __ldcg(a.heavy + 4);    // items of few pieces
+  if (count == 0 && light == 0) return;     // nothing listed, nothing to reset
   const long long W = __ldcg(a.seq_start + S);
   if (W > 0) {
     const Ranges rg = make_ranges(W, workers, a.part_blocks);
-    // items of few pieces: one warp each.  Lane l takes head l / LPH and
-    // VPL consecutive elements of it; every load of the item is issued
-    // before any is used (the partials may come from HBM).
-    constexpr int LPH = 32 / G;   // lanes per head
-    constexpr int VPL = D / LPH;  // values per lane
+    // items of few pieces: one warp each.  Lane l takes head_dim
+    // [DPL*l, DPL*l + DPL) of every head, so each load and store of the warp
+    // is contiguous, and all of an item's loads are in flight together.
     constexpr int NP = kWarpMergeMaxPieces;
-    const int hw = lane / LPH, d0 = (lane % LPH) * VPL;
+    using VecF = typename std::conditional<DPL == 4, float4, float2>::type;
     for (int it = blockIdx.x * GROUPS + grp; it < light; it += gridDim.x * GROUPS) {
       const int item = __ldcg(a.light_list + it);
       const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
@@ -1190,41 +1189,54 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
       const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
       const int np = static_cast<int>(rb - ra + 1);  // (at most NP: listed so)
       long long sl[NP];
-      float2 ml[NP];
-      float M = -INFINITY;
-      int bad = 0;
 #pragma unroll
-      for (int r = 0; r < NP; ++r) {
-        sl[r] = r < np ? piece_slot(rg, ra + r, item_a) : 0;
-        ml[r] = r < np ? __ldcg(a.ws_ml + sl[r] * G + hw) : make_float2(-INFINITY, 0.f);
-      }
+      for (int r = 0; r < NP; ++r) sl[r] = r < np ? piece_slot(rg, ra + r, item_a) : 0;
+      float M[G];
+      int bad = 0;  // bit h: head h poisoned
 #pragma unroll
-      for (int r = 0; r < NP; ++r) {
-        M = fmaxf(M, ml[r].x);
-        bad |= ml[r].y < 0.f;
-      }
-      float L = 0.f, acc[VPL];
-#pragma unroll
-      for (int e = 0; e < VPL; ++e) acc[e] = 0.f;
+      for (int h = 0; h < G; ++h) M[h] = -INFINITY;
 #pragma unroll
       for (int r = 0; r < NP; ++r) {
         if (r < np) {
-          const float w = exp2f(ml[r].x - M);
-          L = fmaf(w, ml[r].y, L);
-          const float2* po = reinterpret_cast<const float2*>(a.ws_o + (sl[r] * G + hw) * D + d0);
 #pragma unroll
-          for (int e = 0; e < VPL / 2; ++e) {
-            const float2 t2 = __ldcg(po + e);
-            acc[2 * e] = fmaf(w, t2.x, acc[2 * e]);
-            acc[2 * e + 1] = fmaf(w, t2.y, acc[2 * e + 1]);
+          for (int h = 0; h < G; ++h) {
+            const float2 ml = __ldcg(a.ws_ml + sl[r] * G + h);
+            M[h] = fmaxf(M[h], ml.x);
+            bad |= (ml.y < 0.f) << h;
           }
         }
       }
-      const float inv = bad ? 0.f : 1.f / L;
-      T* dst = static_cast<T*>(a.out) +
-               (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G + hw) * D + d0;
+      float L[G], acc[G][DPL];
 #pragma unroll
-      for (int e = 0; e < VPL; ++e) dst[e] = static_cast<T>(bad ? 0.f : acc[e] * inv);
+      for (int h = 0; h < G; ++h) {
+        L[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < NP; ++r) {
+        if (r < np) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float2 ml = __ldcg(a.ws_ml + sl[r] * G + h);
+            const VecF t = __ldcg(reinterpret_cast<const VecF*>(a.ws_o + (sl[r] * G + h) * D) + lane);
+            const float w = exp2f(ml.x - M[h]);
+            L[h] = fmaf(w, ml.y, L[h]);
+            const float* tv = reinterpret_cast<const float*>(&t);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(w, tv[e], acc[h][e]);
+          }
+        }
+      }
+      T* dst = static_cast<T*>(a.out) +
+               (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D + lane * DPL;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const bool hb = (bad >> h) & 1;
+        const float inv = hb ? 0.f : 1.f / L[h];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) dst[h * D + e] = static_cast<T>(hb ? 0.f : acc[h][e] * inv);
+      }
     }
     // items of many pieces: one CTA per (item, head)
     for (int p = blockIdx.x; p < count * G; p += gridDim.x) {

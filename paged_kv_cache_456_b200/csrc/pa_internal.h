@@ -79,9 +79,12 @@ struct DecodeArgs {
 };
 
 // CUDA-core path: a split (seq, kv head) whose pieces x G exceed this is merged
-// by the separate merge pass instead of by one warp of the decode kernel.
+// by the separate merge pass instead of by the warp of the decode kernel that
+// finishes its last piece.  0 (the default, measured faster since the merge
+// pass takes one warp per item): every split goes to the merge pass, and the
+// decode kernel needs no fence or counter per piece.
 #ifndef PA_FUSE_MAX_VALUES
-#define PA_FUSE_MAX_VALUES 16
+#define PA_FUSE_MAX_VALUES 0
 #endif
 constexpr int kFuseMaxValues = PA_FUSE_MAX_VALUES;
 constexpr int kMergeThreads = 256;
