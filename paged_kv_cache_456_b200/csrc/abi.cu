@@ -82,10 +82,9 @@ struct DecodePlan {
   int sms = 0;
   // workspace layout; everything before zero_bytes must be zero on entry
   size_t heavy_off = 0;      // [8] ints: merge-pass counts, merge CTAs done, chunks, workers done
-  size_t list_off = 0;       // 2 x [S*Hkv] ints: items for the merge pass (many, few pieces)
+  size_t list_off = 0;       // 2 x [S*Hkv] int4 records: items for the merge pass (many, few pieces)
   size_t counters_off = 0;   // [S*Hkv*2] ints
   size_t zero_bytes = 0;
-  size_t seq_start_off = 0;  // [S + 1] ints
   size_t o_off = 0;
   size_t ml_off = 0;
   size_t ws_bytes = 0;
@@ -217,9 +216,8 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   p->heavy_off = 0;
   p->counters_off = 8 * sizeof(int);
   p->zero_bytes = pa::decode_zero_prefix_bytes(num_seqs, num_kv_heads);
-  p->list_off = p->zero_bytes;
-  p->seq_start_off = round_up(p->list_off + 2 * items * sizeof(int), 16);
-  p->o_off = round_up(p->seq_start_off + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
+  p->list_off = round_up(p->zero_bytes, 16);  // (int4 records)
+  p->o_off = round_up(p->list_off + 2 * items * 4 * sizeof(int), 256);
   p->ml_off = round_up(p->o_off + slots * group * head_dim * sizeof(float), 256);
   p->ws_bytes = round_up(p->ml_off + slots * group * 2 * sizeof(float), 256);
   return PA_OK;
@@ -332,10 +330,9 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   args.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   char* ws = static_cast<char*>(workspace);
   args.counters = reinterpret_cast<int*>(ws + p.counters_off);
-  args.seq_start = reinterpret_cast<int*>(ws + p.seq_start_off);
   args.heavy = reinterpret_cast<int*>(ws + p.heavy_off);
   args.heavy_list = reinterpret_cast<int*>(ws + p.list_off);
-  args.light_list = args.heavy_list + static_cast<size_t>(num_seqs) * num_kv_heads;
+  args.light_list = args.heavy_list + 4 * static_cast<size_t>(num_seqs) * num_kv_heads;
   args.ws_o = reinterpret_cast<float*>(ws + p.o_off);
   args.ws_ml = reinterpret_cast<float2*>(ws + p.ml_off);
   args.err_flag = err_flag;

@@ -491,8 +491,6 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   // ---- this worker's share of the tiles -------------------------------------------
   // the merge pass (launched after this kernel) may start its prologue now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (blockIdx.x == 0)
-    for (int s = tid; s <= S; s += WARPS * 32) a.seq_start[s] = s_start[s];
 
   const long long W = s_start[S];
   if (W == 0) return;
@@ -517,13 +515,17 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   float* xs = reinterpret_cast<float*>(aux);
   float* alpha_s = reinterpret_cast<float*>(aux + C::XS);
   StageDesc* ring_desc = reinterpret_cast<StageDesc*>(wkbase + C::DESC_OFF);
-  // an item for the merge pass: few pieces go to its one-warp list, more to
-  // its one-CTA-per-head list
-  auto list_for_merge = [&](long long pieces, int item) {
-    if (pieces <= kWarpMergeMaxPieces)
-      a.light_list[atomicAdd(a.heavy + 4, 1)] = item;
+  // An item for the merge pass, listed by its first piece as a record
+  // {seq * Hkv + kv head, first range, pieces, partial slot of the first
+  // piece}: each later piece starts its range r, so its partial is in slot 2r.  Few pieces go to the one-warp list, more to the
+  // one-CTA-per-head list.
+  auto list_for_merge = [&](long long ra, long long rb, long long item_a, int item) {
+    const int4 rec = make_int4(item, static_cast<int>(ra), static_cast<int>(rb - ra + 1),
+                               static_cast<int>(piece_slot(rg, ra, item_a)));
+    if (rb - ra + 1 <= kWarpMergeMaxPieces)
+      reinterpret_cast<int4*>(a.light_list)[atomicAdd(a.heavy + 4, 1)] = rec;
     else
-      a.heavy_list[atomicAdd(a.heavy, 1)] = item;
+      reinterpret_cast<int4*>(a.heavy_list)[atomicAdd(a.heavy, 1)] = rec;
   };
 
   const int dl = lane % C::LPR;  // which 16 bytes of a row
@@ -1026,7 +1028,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           a.ws_ml[sl * GT + h0 + 1] = make_float2(mh[1], bad ? -1.f : lt[1]);
         }
         // the merge pass combines the pieces; the first piece lists the item
-        if (r == ra && lane == 0) list_for_merge(rb - ra + 1, s * Hkv + kvh);
+        if (r == ra && lane == 0) list_for_merge(ra, rb, item_a, s * Hkv + kvh);
       }
     } else if (flags & kLast) {
 #pragma unroll
@@ -1079,7 +1081,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
         if (heavy) {
           // many pieces: the merge pass combines them; the first piece lists the item
           if (r == ra && lane == 0 && half == 0) {
-            list_for_merge(rb - ra + 1, s * Hkv + kvh);
+            list_for_merge(ra, rb, item_a, s * Hkv + kvh);
           }
         } else {
           __threadfence();
@@ -1172,25 +1174,19 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   const int count = __ldcg(a.heavy);        // items of many pieces
   const int light = __ldcg(a.heavy + 4);    // items of few pieces
   if (count == 0 && light == 0) return;     // nothing listed, nothing to reset
-  const long long W = __ldcg(a.seq_start + S);
-  if (W > 0) {
-    const Ranges rg = make_ranges(W, workers, a.part_blocks);
+  {
     // items of few pieces: one warp each.  Lane l takes head_dim
     // [DPL*l, DPL*l + DPL) of every head, so each load and store of the warp
     // is contiguous, and all of an item's loads are in flight together.
     constexpr int NP = kWarpMergeMaxPieces;
     using VecF = typename std::conditional<DPL == 4, float4, float2>::type;
     for (int it = blockIdx.x * GROUPS + grp; it < light; it += gridDim.x * GROUPS) {
-      const int item = __ldcg(a.light_list + it);
-      const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
-      const int st = __ldcg(a.seq_start + s);
-      const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
-      const long long item_a = st + static_cast<long long>(kvh) * nb;
-      const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
-      const int np = static_cast<int>(rb - ra + 1);  // (at most NP: listed so)
+      const int4 rec = __ldcg(reinterpret_cast<const int4*>(a.light_list) + it);
+      const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
+      const int np = rec.z;  // (at most NP: listed so)
       long long sl[NP];
 #pragma unroll
-      for (int r = 0; r < NP; ++r) sl[r] = r < np ? piece_slot(rg, ra + r, item_a) : 0;
+      for (int r = 0; r < NP; ++r) sl[r] = r == 0 ? rec.w : 2 * (static_cast<long long>(rec.y) + r);
       float M[G];
       int bad = 0;  // bit h: head h poisoned
 #pragma unroll
@@ -1240,18 +1236,16 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
     }
     // items of many pieces: one CTA per (item, head)
     for (int p = blockIdx.x; p < count * G; p += gridDim.x) {
-      const int item = __ldcg(a.heavy_list + p / G);
+      const int4 rec = __ldcg(reinterpret_cast<const int4*>(a.heavy_list) + p / G);
       const int hl = p % G;
-      const int s = item / Hkv, kvh = item - (item / Hkv) * Hkv;
-      const int st = __ldcg(a.seq_start + s);
-      const int nb = (__ldcg(a.seq_start + s + 1) - st) / Hkv;
-      const long long item_a = st + static_cast<long long>(kvh) * nb;
-      const long long ra = rg.of(item_a), rb = rg.of(item_a + nb - 1);
+      const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
+      const long long ra = rec.y, rb = ra + rec.z - 1;
+      auto slot_of = [&](long long r) -> long long { return r == ra ? rec.w : 2 * r; };
 
       float M = -INFINITY;
       int bad = 0;
       for (long long r = ra + grp; r <= rb; r += GROUPS) {
-        const float2 ml = __ldcg(a.ws_ml + piece_slot(rg, r, item_a) * G + hl);
+        const float2 ml = __ldcg(a.ws_ml + slot_of(r) * G + hl);
         M = fmaxf(M, ml.x);
         bad |= ml.y < 0.f;
       }
@@ -1270,7 +1264,7 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
       for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
       float L = 0.f;
       for (long long r = ra + grp; r <= rb; r += GROUPS) {
-        const long long sl = piece_slot(rg, r, item_a);
+        const long long sl = slot_of(r);
         const float2 ml = __ldcg(a.ws_ml + sl * G + hl);
         const float w = exp2f(ml.x - M);
         L = fmaf(w, ml.y, L);

@@ -58,12 +58,12 @@ struct DecodeArgs {
   float scale_log2;  // scale * log2(e)
   int* counters;     // [num_seqs * num_kv_heads * 2] pieces finished per (item, head half),
                      // zero between calls
-  int* seq_start;    // [num_seqs + 1] first tile of each sequence (written for the merge pass)
   int* heavy;        // [8]: items of many pieces listed for the merge pass, merge CTAs
                      // done, tail chunks claimed, decode workers done, items of few
                      // pieces listed (all zero between calls)
-  int* heavy_list;   // [num_seqs * num_kv_heads] (seq * Hkv + kv head) of many-piece items
-  int* light_list;   // [num_seqs * num_kv_heads] the same for items of few pieces
+  int* heavy_list;   // [num_seqs * num_kv_heads] int4 records {seq * Hkv + kv head, first
+                     // range, pieces, first piece's slot} of many-piece items
+  int* light_list;   // the same for items of few pieces
   float* ws_o;       // [2 * ranges][G][head_dim] unnormalised partial outputs
   float2* ws_ml;     // [2 * ranges][G] (running max, sum) of each partial; sum < 0 = poisoned
   int32_t* err_flag;
