@@ -4,6 +4,7 @@
 // heads runs on the tensor cores, one warp per KV head (or, built with
 // PA_G8_MMA=0, on the CUDA cores split over two warps that share one ring).
 #include "decode_kernel.cuh"
+#include "merge_kernel.cuh"
 
 namespace pa {
 

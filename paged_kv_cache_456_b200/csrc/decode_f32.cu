@@ -2,6 +2,7 @@
 // Ring depth and warps per CTA are chosen per shape so that two or more CTAs
 // fit in an SM's shared memory with several tiles in flight per warp.
 #include "decode_kernel.cuh"
+#include "merge_kernel.cuh"
 
 namespace pa {
 

@@ -1,0 +1,172 @@
+// merge_kernel.cuh -- the second pass of split-K decode: combines the
+// partial results (m, l, o) of (sequence, KV head) items that the decode
+// kernel cut into pieces, by log-sum-exp.
+#pragma once
+
+#include <cstdint>
+#include <type_traits>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+// Merge pass for the (seq, kv head) items listed by the decode kernel.  An
+// item of few pieces is merged by one warp; an item of many pieces (long
+// contexts) gets one CTA per (item, query head), kMergeThreads / 32 groups of
+// lanes taking every GROUPS-th piece, combined in shared memory:
+//     M = max_j m_j,  out = sum_j 2^(m_j - M) o_j / sum_j 2^(m_j - M) l_j.
+// Launched right behind the decode kernel with programmatic dependent launch;
+// griddepcontrol.wait returns once the decode grid has finished and its
+// writes are visible.  The last CTA to finish resets the item list.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kMergeThreads)
+paged_decode_merge_kernel(const DecodeArgs a, int workers) {
+  constexpr int GROUPS = kMergeThreads / 32;
+  constexpr int DPL = D / 32;  // dims per lane
+  __shared__ float s_m[GROUPS];
+  __shared__ float s_l[GROUPS];
+  __shared__ int s_bad[GROUPS];
+  __shared__ __align__(16) float s_acc[GROUPS][D];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int tid = threadIdx.x, grp = tid >> 5, lane = tid & 31;
+  const int S = a.num_seqs, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
+  const int count = __ldcg(a.heavy);        // items of many pieces
+  const int light = __ldcg(a.heavy + 4);    // items of few pieces
+  if (count == 0 && light == 0) return;     // nothing listed, nothing to reset
+  {
+    // items of few pieces: one warp each.  Lane l takes head_dim
+    // [DPL*l, DPL*l + DPL) of every head, so each load and store of the warp
+    // is contiguous, and all of an item's loads are in flight together.
+    constexpr int NP = kWarpMergeMaxPieces;
+    using VecF = typename std::conditional<DPL == 4, float4, float2>::type;
+    for (int it = blockIdx.x * GROUPS + grp; it < light; it += gridDim.x * GROUPS) {
+      const int4 rec = __ldcg(reinterpret_cast<const int4*>(a.light_list) + it);
+      const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
+      const int np = rec.z;  // (at most NP: listed so)
+      long long sl[NP];
+#pragma unroll
+      for (int r = 0; r < NP; ++r) sl[r] = r == 0 ? rec.w : 2 * (static_cast<long long>(rec.y) + r);
+      float M[G];
+      int bad = 0;  // bit h: head h poisoned
+#pragma unroll
+      for (int h = 0; h < G; ++h) M[h] = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < NP; ++r) {
+        if (r < np) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float2 ml = __ldcg(a.ws_ml + sl[r] * G + h);
+            M[h] = fmaxf(M[h], ml.x);
+            bad |= (ml.y < 0.f) << h;
+          }
+        }
+      }
+      float L[G], acc[G][DPL];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        L[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < NP; ++r) {
+        if (r < np) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float2 ml = __ldcg(a.ws_ml + sl[r] * G + h);
+            const VecF t = __ldcg(reinterpret_cast<const VecF*>(a.ws_o + (sl[r] * G + h) * D) + lane);
+            const float w = exp2f(ml.x - M[h]);
+            L[h] = fmaf(w, ml.y, L[h]);
+            const float* tv = reinterpret_cast<const float*>(&t);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(w, tv[e], acc[h][e]);
+          }
+        }
+      }
+      T* dst = static_cast<T*>(a.out) +
+               (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D + lane * DPL;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const bool hb = (bad >> h) & 1;
+        const float inv = hb ? 0.f : 1.f / L[h];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) dst[h * D + e] = static_cast<T>(hb ? 0.f : acc[h][e] * inv);
+      }
+    }
+    // items of many pieces: one CTA per (item, head)
+    for (int p = blockIdx.x; p < count * G; p += gridDim.x) {
+      const int4 rec = __ldcg(reinterpret_cast<const int4*>(a.heavy_list) + p / G);
+      const int hl = p % G;
+      const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
+      const long long ra = rec.y, rb = ra + rec.z - 1;
+      auto slot_of = [&](long long r) -> long long { return r == ra ? rec.w : 2 * r; };
+
+      float M = -INFINITY;
+      int bad = 0;
+      for (long long r = ra + grp; r <= rb; r += GROUPS) {
+        const float2 ml = __ldcg(a.ws_ml + slot_of(r) * G + hl);
+        M = fmaxf(M, ml.x);
+        bad |= ml.y < 0.f;
+      }
+      if (lane == 0) {
+        s_m[grp] = M;
+        s_bad[grp] = bad;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) {
+        M = fmaxf(M, s_m[g]);
+        bad |= s_bad[g];
+      }
+      float acc[DPL];
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+      float L = 0.f;
+      for (long long r = ra + grp; r <= rb; r += GROUPS) {
+        const long long sl = slot_of(r);
+        const float2 ml = __ldcg(a.ws_ml + sl * G + hl);
+        const float w = exp2f(ml.x - M);
+        L = fmaf(w, ml.y, L);
+        const float* po = a.ws_o + (sl * G + hl) * D + lane * DPL;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, __ldcg(po + d), acc[d]);
+      }
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) s_acc[grp][lane * DPL + d] = acc[d];
+      if (lane == 0) s_l[grp] = L;
+      __syncthreads();
+      if (grp == 0) {
+        float Lt = 0.f;
+#pragma unroll
+        for (int g = 0; g < GROUPS; ++g) Lt += s_l[g];
+        float r[DPL];
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) {
+          float t = 0.f;
+#pragma unroll
+          for (int g = 0; g < GROUPS; ++g) t += s_acc[g][lane * DPL + d];
+          r[d] = bad ? 0.f : t / Lt;
+        }
+        T* dst = static_cast<T*>(a.out) +
+                 (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G + hl) * D + lane * DPL;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) dst[d] = static_cast<T>(r[d]);
+      }
+      __syncthreads();
+    }
+  }
+  // the last CTA out clears the item list for the next call
+  __syncthreads();
+  // (every thread of this CTA has used the count it read before this point)
+  if (tid == 0 && atomicAdd(a.heavy + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+    a.heavy[0] = 0;
+    a.heavy[1] = 0;
+    a.heavy[4] = 0;
+  }
+}
+
+}  // namespace pa

@@ -88,6 +88,9 @@ struct DecodeArgs {
 #endif
 constexpr int kFuseMaxValues = PA_FUSE_MAX_VALUES;
 constexpr int kMergeThreads = 256;
+// Merge pass: an item of at most this many pieces is merged by one warp (all
+// its heads); items with more pieces get a whole CTA per head.
+constexpr int kWarpMergeMaxPieces = 8;
 
 struct DecodeKernelInfo {
   const void* fn;   // the __global__ function
