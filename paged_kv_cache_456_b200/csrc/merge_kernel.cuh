@@ -34,6 +34,11 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
 
   const int tid = threadIdx.x, grp = tid >> 5, lane = tid & 31;
   const int S = a.num_seqs, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
+  // this warp's first record is read together with the counts (the list has
+  // room for S * Hkv records; one past the count is simply not used)
+  const int it0 = blockIdx.x * GROUPS + grp;
+  const int4 rec0 = it0 < S * Hkv ? __ldcg(reinterpret_cast<const int4*>(a.light_list) + it0)
+                                  : make_int4(0, 0, 0, 0);
   const int count = __ldcg(a.heavy);        // items of many pieces
   const int light = __ldcg(a.heavy + 4);    // items of few pieces
   if (count == 0 && light == 0) return;     // nothing listed, nothing to reset
@@ -43,47 +48,53 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
     // is contiguous, and all of an item's loads are in flight together.
     constexpr int NP = kWarpMergeMaxPieces;
     using VecF = typename std::conditional<DPL == 4, float4, float2>::type;
-    for (int it = blockIdx.x * GROUPS + grp; it < light; it += gridDim.x * GROUPS) {
-      const int4 rec = __ldcg(reinterpret_cast<const int4*>(a.light_list) + it);
+    for (int it = it0; it < light; it += gridDim.x * GROUPS) {
+      const int4 rec =
+          it == it0 ? rec0 : __ldcg(reinterpret_cast<const int4*>(a.light_list) + it);
       const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
       const int np = rec.z;  // (at most NP: listed so)
-      long long sl[NP];
-#pragma unroll
-      for (int r = 0; r < NP; ++r) sl[r] = r == 0 ? rec.w : 2 * (static_cast<long long>(rec.y) + r);
-      float M[G];
+      auto slot_of = [&](int r) -> long long {  // piece r's partial slot
+        return r == 0 ? rec.w : 2 * (static_cast<long long>(rec.y) + r);
+      };
+      // pieces two at a time, every load of a pair issued before any is used
+      // (one memory round trip per pair), merged with a running maximum
+      float M[G], L[G], acc[G][DPL];
       int bad = 0;  // bit h: head h poisoned
 #pragma unroll
-      for (int h = 0; h < G; ++h) M[h] = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < NP; ++r) {
-        if (r < np) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float2 ml = __ldcg(a.ws_ml + sl[r] * G + h);
-            M[h] = fmaxf(M[h], ml.x);
-            bad |= (ml.y < 0.f) << h;
-          }
-        }
-      }
-      float L[G], acc[G][DPL];
-#pragma unroll
       for (int h = 0; h < G; ++h) {
+        M[h] = -INFINITY;
         L[h] = 0.f;
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
       }
 #pragma unroll
-      for (int r = 0; r < NP; ++r) {
-        if (r < np) {
+      for (int r0 = 0; r0 < NP; r0 += 2) {
+        if (r0 < np) {
+          const bool two = r0 + 1 < np;
+          float2 ml[2][G];
+          VecF ov[2][G];
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const long long sj = slot_of(r0 + (two ? j : 0));  // (a lone last piece: twice)
+              ml[j][h] = __ldcg(a.ws_ml + sj * G + h);
+              ov[j][h] = __ldcg(reinterpret_cast<const VecF*>(a.ws_o + (sj * G + h) * D) + lane);
+            }
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float2 ml = __ldcg(a.ws_ml + sl[r] * G + h);
-            const VecF t = __ldcg(reinterpret_cast<const VecF*>(a.ws_o + (sl[r] * G + h) * D) + lane);
-            const float w = exp2f(ml.x - M[h]);
-            L[h] = fmaf(w, ml.y, L[h]);
-            const float* tv = reinterpret_cast<const float*>(&t);
+            const float2 m0 = ml[0][h], m1 = two ? ml[1][h] : make_float2(-INFINITY, 0.f);
+            bad |= ((m0.y < 0.f) | (m1.y < 0.f)) << h;
+            const float mn = fmaxf(M[h], fmaxf(m0.x, m1.x));
+            // (an empty running state, M = -inf, has nothing to scale)
+            const float sc = M[h] == -INFINITY ? 0.f : exp2f(M[h] - mn);
+            const float w0 = exp2f(m0.x - mn), w1 = two ? exp2f(m1.x - mn) : 0.f;
+            L[h] = L[h] * sc + w0 * m0.y + w1 * m1.y;
+            const float* t0 = reinterpret_cast<const float*>(&ov[0][h]);
+            const float* t1 = reinterpret_cast<const float*>(&ov[1][h]);
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(w, tv[e], acc[h][e]);
+            for (int e = 0; e < DPL; ++e) acc[h][e] = acc[h][e] * sc + w0 * t0[e] + w1 * t1[e];
+            M[h] = mn;
           }
         }
       }
