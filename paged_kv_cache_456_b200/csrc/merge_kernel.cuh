@@ -116,56 +116,75 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
       const long long ra = rec.y, rb = ra + rec.z - 1;
       auto slot_of = [&](long long r) -> long long { return r == ra ? rec.w : 2 * r; };
 
-      float M = -INFINITY;
+      // each warp takes pieces ra + grp, + GROUPS, ..., four at a time with all
+      // their loads in flight, merged with a running maximum; then the warps'
+      // (M, L, acc) are combined through shared memory
+      constexpr int CHUNK = 4;
+      float M = -INFINITY, L = 0.f, acc[DPL];
       int bad = 0;
-      for (long long r = ra + grp; r <= rb; r += GROUPS) {
-        const float2 ml = __ldcg(a.ws_ml + slot_of(r) * G + hl);
-        M = fmaxf(M, ml.x);
-        bad |= ml.y < 0.f;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+      for (long long base = ra + grp; base <= rb; base += CHUNK * GROUPS) {
+        float2 ml[CHUNK];
+        VecF ov[CHUNK];
+#pragma unroll
+        for (int j = 0; j < CHUNK; ++j) {
+          const long long r = base + j * GROUPS;
+          const long long sl = slot_of(r <= rb ? r : base);
+          ml[j] = __ldcg(a.ws_ml + sl * G + hl);
+          ov[j] = __ldcg(reinterpret_cast<const VecF*>(a.ws_o + (sl * G + hl) * D) + lane);
+          if (r > rb) ml[j] = make_float2(-INFINITY, 0.f);   // (a repeat, weighed 0)
+        }
+        float mn = M;
+#pragma unroll
+        for (int j = 0; j < CHUNK; ++j) {
+          mn = fmaxf(mn, ml[j].x);
+          bad |= ml[j].y < 0.f;
+        }
+        const float sc = M == -INFINITY ? 0.f : exp2f(M - mn);
+        L *= sc;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) acc[d] *= sc;
+#pragma unroll
+        for (int j = 0; j < CHUNK; ++j) {
+          const float w = ml[j].x == -INFINITY ? 0.f : exp2f(ml[j].x - mn);
+          L = fmaf(w, ml[j].y, L);
+          const float* t = reinterpret_cast<const float*>(&ov[j]);
+#pragma unroll
+          for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, t[d], acc[d]);
+        }
+        M = mn;
       }
       if (lane == 0) {
         s_m[grp] = M;
+        s_l[grp] = L;
         s_bad[grp] = bad;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int g = 0; g < GROUPS; ++g) {
-        M = fmaxf(M, s_m[g]);
-        bad |= s_bad[g];
-      }
-      float acc[DPL];
-#pragma unroll
-      for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
-      float L = 0.f;
-      for (long long r = ra + grp; r <= rb; r += GROUPS) {
-        const long long sl = slot_of(r);
-        const float2 ml = __ldcg(a.ws_ml + sl * G + hl);
-        const float w = exp2f(ml.x - M);
-        L = fmaf(w, ml.y, L);
-        const float* po = a.ws_o + (sl * G + hl) * D + lane * DPL;
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, __ldcg(po + d), acc[d]);
       }
 #pragma unroll
       for (int d = 0; d < DPL; ++d) s_acc[grp][lane * DPL + d] = acc[d];
-      if (lane == 0) s_l[grp] = L;
       __syncthreads();
       if (grp == 0) {
-        float Lt = 0.f;
+        float Mt = -INFINITY;
+        int bt = 0;
 #pragma unroll
-        for (int g = 0; g < GROUPS; ++g) Lt += s_l[g];
-        float r[DPL];
+        for (int g = 0; g < GROUPS; ++g) {
+          Mt = fmaxf(Mt, s_m[g]);
+          bt |= s_bad[g];
+        }
+        float Lt = 0.f, r[DPL];
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) {
-          float t = 0.f;
+        for (int d = 0; d < DPL; ++d) r[d] = 0.f;
 #pragma unroll
-          for (int g = 0; g < GROUPS; ++g) t += s_acc[g][lane * DPL + d];
-          r[d] = bad ? 0.f : t / Lt;
+        for (int g = 0; g < GROUPS; ++g) {
+          const float f = s_m[g] == -INFINITY ? 0.f : exp2f(s_m[g] - Mt);
+          Lt = fmaf(f, s_l[g], Lt);
+#pragma unroll
+          for (int d = 0; d < DPL; ++d) r[d] = fmaf(f, s_acc[g][lane * DPL + d], r[d]);
         }
         T* dst = static_cast<T*>(a.out) +
                  (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G + hl) * D + lane * DPL;
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) dst[d] = static_cast<T>(r[d]);
+        for (int d = 0; d < DPL; ++d) dst[d] = static_cast<T>(bt ? 0.f : r[d] / Lt);
       }
       __syncthreads();
     }
