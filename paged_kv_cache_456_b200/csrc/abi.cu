@@ -354,8 +354,8 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
     cudaGetLastError();  // a refused launch is reported here, not left for the caller
     return PA_ERR_CUDA;
   }
-  // merge pass for items split into many pieces, launched behind the decode
-  // kernel with programmatic dependent launch (it waits for the decode grid)
+  // merge pass for the split items, launched behind the decode kernel with
+  // programmatic dependent launch (it waits for the decode grid)
   int workers = p.grid * p.kernel.workers;
   void* mparams[] = {&args, &workers};
   cudaLaunchConfig_t cfg = {};

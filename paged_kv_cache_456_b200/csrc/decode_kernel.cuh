@@ -1138,8 +1138,9 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       B = static_desc(base + 32 + lane);
     }
   }
-  // the last worker out resets the chunk counter for the next call
-  if (leader && lane == 0) {
+  // the last worker out resets the chunk counter for the next call (only a
+  // claimed tail uses it)
+  if (kTailDiv > 0 && leader && lane == 0) {
     if (atomicAdd(a.heavy + 3, 1) == static_cast<int>(NWK) - 1) {
       a.heavy[2] = 0;
       a.heavy[3] = 0;
