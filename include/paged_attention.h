@@ -88,6 +88,10 @@ const char *pa_status_str(pa_status status);
  * Only tokens 0..n-1 are read; unused slots of a partial last block and
  * table entries past ceil(n/16) may hold anything (NaN, -1).  n == 0 gives a
  * zero row.  out is rounded once (nearest-even) to the element type.
+ * Arithmetic is fp32.  For bf16 caches with 8 query heads per KV head the
+ * dot products and the weighted sum of V run on the tensor cores (bf16
+ * operands, fp32 accumulation), the softmax weights being rounded to bf16
+ * for that sum (and for its normaliser alike).
  *
  * Arguments:
  *   out            [num_seqs][num_q_heads][head_dim]            written
