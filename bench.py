@@ -289,8 +289,12 @@ def run_ours(args, rank: int, world: int):
     ps = w.partition_size
     prefill = "query_start" in t     # several query tokens per sequence
     rows = t["q"].shape[0]            # query rows: one per sequence in decode
-    ws = ops.make_workspace(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                            w.max_context_len, ps, tdt, device=dev)
+    if prefill:
+        ws = ops.make_prefill_workspace(w.num_seqs, rows, w.num_q_heads, w.num_kv_heads,
+                                        w.head_dim, w.max_context_len, ps, tdt, device=dev)
+    else:
+        ws = ops.make_workspace(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                w.max_context_len, ps, tdt, device=dev)
     cfg = ops.launch_config(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
                             w.max_context_len, ps, tdt)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)

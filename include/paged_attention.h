@@ -245,17 +245,26 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
  *   q, out          device, [num_query_tokens][num_q_heads][head_dim].
  *   query_start     device int32 [num_seqs + 1], non-decreasing, from 0 to
  *                   num_query_tokens; Q <= n for every sequence.  A
- *                   sequence that breaks this gets zero rows and
- *                   PA_ERRBIT_QUERY.
- *   workspace       pa_decode_workspace_size(num_query_tokens, ...) bytes,
- *                   zero-filled before first use, as for pa_decode.
- *   Everything else is as in pa_decode.  Query rows are independent work
- *   items to the decode kernel (grouped with the other query heads of their
- *   KV head, on the tensor cores for bf16 groups of 8), so each row reads
- *   its own prefix of the cache.  Launch-time shared memory grows with
- *   num_query_tokens (12 bytes per row); too many rows for one SM's
- *   shared memory returns PA_ERR_UNSUPPORTED.
+ *                   sequence with Q > n gets zero rows and PA_ERRBIT_QUERY;
+ *                   query_start values out of order or outside
+ *                   [0, num_query_tokens] set PA_ERRBIT_QUERY, and rows no
+ *                   valid sequence covers may be left unwritten.
+ *   workspace       pa_prefill_workspace_size() bytes, zero-filled before
+ *                   first use (pa_decode_workspace_init), as for pa_decode.
+ *   Everything else is as in pa_decode.  Each query row is a work item of
+ *   the decode kernel over its own prefix of the cache, together with the
+ *   other query heads of its KV head.  For bf16 caches with 8 query heads
+ *   per KV head, an item is a pair of consecutive query rows of a
+ *   sequence (16 columns on the tensor cores): each K/V tile of the pair's
+ *   longer prefix is read once for both, and the earlier row masks the last
+ *   token.  Launch-time shared memory grows with num_query_tokens (12 to 20
+ *   bytes per row); too many rows for one SM's shared memory returns
+ *   PA_ERR_UNSUPPORTED.
  */
+pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_q_heads,
+                                    int num_kv_heads, int head_dim, int max_context_len,
+                                    int partition_size, pa_dtype dtype, size_t *bytes);
+
 pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, const int32_t *context_lens,
                      const int32_t *query_start, int num_seqs, int num_query_tokens,

@@ -175,9 +175,15 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
   const int group = num_q_heads / num_kv_heads;
-  const bool found = dtype == PA_BF16 ? pa::decode_kernel_bf16(head_dim, group, &p->kernel)
-                                      : pa::decode_kernel_f32(head_dim, group, &p->kernel);
+  // several query tokens per sequence: bf16 groups of 8 heads have their own
+  // kernel (groups of query rows per item); everything else shares decode's
+  bool found = table_rows >= 0 && dtype == PA_BF16 &&
+               pa::prefill_kernel_bf16(head_dim, group, &p->kernel);
+  if (!found)
+    found = dtype == PA_BF16 ? pa::decode_kernel_bf16(head_dim, group, &p->kernel)
+                             : pa::decode_kernel_f32(head_dim, group, &p->kernel);
   if (!found) return PA_ERR_UNSUPPORTED;
+  const int columns = group * p->kernel.rows_per_item;  // partial columns per item
   // tiles: must fit the kernel's 32-bit tile counter
   const long long blocks_max = (static_cast<long long>(max_context_len) + pa::kBlockSize - 1) /
                                pa::kBlockSize;
@@ -186,8 +192,12 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 
   DeviceInfo dev;
   if ((st = device_info(&dev)) != PA_OK) return st;
-  const size_t seq_ints = 2 * static_cast<size_t>(num_seqs) + 1 +
-                          (table_rows >= 0 ? static_cast<size_t>(num_seqs) + table_rows + 1 : 0);
+  size_t seq_ints = 2 * static_cast<size_t>(num_seqs) + 1;  // item starts, lengths
+  if (table_rows >= 0) {
+    seq_ints += static_cast<size_t>(num_seqs) + table_rows + 1;  // table rows, query_start
+    if (p->kernel.rows_per_item > 1)
+      seq_ints += static_cast<size_t>(num_seqs) + table_rows + 1;  // group rows, group starts
+  }
   const size_t seq_bytes = round_up(seq_ints * sizeof(int), 16);
   p->smem = static_cast<size_t>(p->kernel.cta_bytes) + seq_bytes;
   if (p->smem > static_cast<size_t>(dev.smem_optin)) return PA_ERR_UNSUPPORTED;
@@ -218,8 +228,8 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   p->zero_bytes = pa::decode_zero_prefix_bytes(num_seqs, num_kv_heads);
   p->list_off = round_up(p->zero_bytes, 16);  // (int4 records)
   p->o_off = round_up(p->list_off + 2 * items * 4 * sizeof(int), 256);
-  p->ml_off = round_up(p->o_off + slots * group * head_dim * sizeof(float), 256);
-  p->ws_bytes = round_up(p->ml_off + slots * group * 2 * sizeof(float), 256);
+  p->ml_off = round_up(p->o_off + slots * columns * head_dim * sizeof(float), 256);
+  p->ws_bytes = round_up(p->ml_off + slots * columns * 2 * sizeof(float), 256);
   return PA_OK;
 }
 
@@ -249,6 +259,34 @@ pa_status pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_hea
   DecodePlan p;
   const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
                                  partition_size, dtype, &p);
+  if (st != PA_OK) return st;
+  *bytes = p.ws_bytes;
+  return PA_OK;
+}
+
+// Items of a call with several query tokens per sequence: one per query
+// row, or -- with the grouping kernel -- at most ceil((T + (NR-1) R) / NR)
+// groups of NR rows (sum over sequences of ceil(Q_s / NR)).
+static int prefill_items(int num_seqs, int num_query_tokens, int num_q_heads, int num_kv_heads,
+                  int head_dim, pa_dtype dtype) {
+  pa::DecodeKernelInfo k{};
+  if (dtype != PA_BF16 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      !pa::prefill_kernel_bf16(head_dim, num_q_heads / num_kv_heads, &k) || k.rows_per_item <= 1)
+    return num_query_tokens;
+  const long long nr = k.rows_per_item;
+  const long long items = (num_query_tokens + (nr - 1) * static_cast<long long>(num_seqs) + nr - 1) / nr;
+  return static_cast<int>(items < num_query_tokens ? items : num_query_tokens);
+}
+
+pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_q_heads,
+                                    int num_kv_heads, int head_dim, int max_context_len,
+                                    int partition_size, pa_dtype dtype, size_t* bytes) {
+  if (!bytes || num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
+  DecodePlan p;
+  const int items = prefill_items(num_seqs, num_query_tokens, num_q_heads, num_kv_heads,
+                                  head_dim, dtype);
+  const pa_status st = make_plan(items, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                 partition_size, dtype, &p, num_seqs > 0 ? num_seqs : 1);
   if (st != PA_OK) return st;
   *bytes = p.ws_bytes;
   return PA_OK;
@@ -288,7 +326,7 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
                       int num_blocks, int max_context_len, float scale, int partition_size,
                       pa_dtype dtype, void* workspace, size_t workspace_bytes,
                       int32_t* err_flag, void* stream, const int32_t* query_start = nullptr,
-                      int table_rows = -1) {
+                      int table_rows = -1, int query_rows = 0) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -338,6 +376,7 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   args.err_flag = err_flag;
   args.query_start = query_start;
   args.num_table_rows = query_start ? table_rows : num_seqs;
+  args.num_query_rows = query_start ? query_rows : num_seqs;
   if (p.kernel.tma) {
     // tile coordinates are 32-bit: row (block * Hkv + kv head) * 16 of the 2-D view
     const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
@@ -414,10 +453,13 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
   if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
   if (num_query_tokens == 0) return PA_OK;
   if (num_seqs == 0 || !query_start) return PA_ERR_INVALID_ARG;
+  const int items = prefill_items(num_seqs, num_query_tokens, num_q_heads, num_kv_heads,
+                                  head_dim, dtype);
   return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens,
-                     num_query_tokens, num_q_heads, num_kv_heads, head_dim, block_size,
+                     items, num_q_heads, num_kv_heads, head_dim, block_size,
                      max_blocks_per_seq, num_blocks, max_context_len, scale, partition_size,
-                     dtype, workspace, workspace_bytes, err_flag, stream, query_start, num_seqs);
+                     dtype, workspace, workspace_bytes, err_flag, stream, query_start, num_seqs,
+                     num_query_tokens);
 }
 
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

@@ -8,16 +8,19 @@
 
 namespace pa {
 
-template <int D, int G, int HS, int DEPTH, int WARPS, int MIN_CTAS = 1, bool MMA = false>
+template <int D, int G, int HS, int DEPTH, int WARPS, int MIN_CTAS = 1, bool MMA = false,
+          int NR = 1>
 static bool fill(DecodeKernelInfo* info) {
   info->fn = reinterpret_cast<const void*>(
-      &paged_decode_kernel<__nv_bfloat16, D, G, HS, DEPTH, WARPS, MIN_CTAS, MMA>);
-  info->merge_fn = reinterpret_cast<const void*>(&paged_decode_merge_kernel<__nv_bfloat16, D, G>);
+      &paged_decode_kernel<__nv_bfloat16, D, G, HS, DEPTH, WARPS, MIN_CTAS, MMA, NR>);
+  info->merge_fn =
+      reinterpret_cast<const void*>(&paged_decode_merge_kernel<__nv_bfloat16, D, NR * G, G>);
   info->warps = WARPS;
   info->workers = WARPS / HS;
   info->depth = DEPTH;
-  info->cta_bytes = DecodeCfg<__nv_bfloat16, D, G / HS, G, HS, DEPTH, WARPS, MMA>::CTA_BYTES;
+  info->cta_bytes = DecodeCfg<__nv_bfloat16, D, G / HS, G, HS, DEPTH, WARPS, MMA, NR>::CTA_BYTES;
   info->tma = MMA;
+  info->rows_per_item = NR;
   return true;
 }
 
@@ -48,6 +51,27 @@ static bool fill(DecodeKernelInfo* info) {
 #ifndef PA_MMA_MINCTAS
 #define PA_MMA_MINCTAS 3
 #endif
+
+// Several query tokens per sequence with 8 heads per KV head: the
+// tensor-core kernel with groups of PA_PREFILL_ROWS query rows per item (they
+// share every K/V tile of the group's longest prefix).
+#ifndef PA_PREFILL_ROWS
+#define PA_PREFILL_ROWS 2
+#endif
+#ifndef PA_PREFILL_DEPTH
+#define PA_PREFILL_DEPTH 2
+#endif
+
+bool prefill_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info) {
+  if (!PA_G8_MMA || group != 8 || PA_PREFILL_ROWS < 2) return false;
+  switch (head_dim) {
+    case 64:
+      return fill<64, 8, 1, PA_PREFILL_DEPTH, PA_MMA_WARPS, PA_MMA_MINCTAS, true, PA_PREFILL_ROWS>(info);
+    case 128:
+      return fill<128, 8, 1, PA_PREFILL_DEPTH, PA_MMA_WARPS, PA_MMA_MINCTAS, true, PA_PREFILL_ROWS>(info);
+    default: return false;
+  }
+}
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info) {
   constexpr int kD = PA_BF16_128_DEPTH, kD8 = PA_BF16_128_DEPTH_G8, kW = PA_BF16_128_WARPS;

@@ -15,6 +15,7 @@ static bool fill(DecodeKernelInfo* info) {
   info->depth = DEPTH;
   info->cta_bytes = DecodeCfg<float, D, G / HS, G, HS, DEPTH, WARPS>::CTA_BYTES;
   info->tma = false;
+  info->rows_per_item = 1;
   return true;
 }
 

@@ -167,7 +167,8 @@ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 // MMA: the tensor-core layout of a slot -- K and V tiles as 128-byte-swizzled
 // boxes (1024-byte aligned), then q, then a staging row pair for the fused
 // slot write -- padded to a multiple of 1024 bytes.
-template <typename T, int D, int G, int GT, int HS, int DEPTH, int WARPS, bool MMA = false>
+template <typename T, int D, int G, int GT, int HS, int DEPTH, int WARPS, bool MMA = false,
+          int NR = 1>
 struct DecodeCfg {
   static constexpr int EB = sizeof(T);
   static constexpr int ROW = D * EB;          // bytes of one token's row of one KV head
@@ -176,7 +177,7 @@ struct DecodeCfg {
   static constexpr int RPI = 32 / LPR;        // rows one warp instruction covers (row groups)
   static constexpr int RL = kBlockSize / RPI; // rows per lane per block
   static constexpr int TILE = kBlockSize * ROW;
-  static constexpr int QB = GT * ROW;         // q rows of the whole group
+  static constexpr int QB = NR * GT * ROW;    // q rows of the whole group (of NR query rows)
   static constexpr int APP = 2 * TILE + QB;   // MMA: staging for the new K and V rows
   static constexpr int SLOT =
       MMA ? ((2 * TILE + QB + 2 * ROW + 1023) / 1024) * 1024 : 2 * TILE + QB;  // K, V, q (, rows)
@@ -209,6 +210,7 @@ struct DecodeCfg {
   static_assert(32 % G == 0 && G <= 16 && GT == G * HS, "group size");
   static_assert(!MMA || (EB == 2 && GT == 8 && HS == 1 && D % 64 == 0),
                 "the tensor-core path takes bf16, 8 heads per KV head, one warp per worker");
+  static_assert(NR == 1 || (MMA && NR <= 2), "several query rows per item: tensor-core path");
 };
 
 // -- per-warp ranges of the global tile order ------------------------------------
@@ -363,11 +365,15 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[V]) {
 // worker (the leader) issues the copies; every warp waits on the slot's
 // "full" barrier and releases the slot on its "empty" barrier, which the
 // leader waits on (bounded) before refilling the slot.
-template <typename T, int D, int GT, int HS, int DEPTH, int WARPS, int MIN_CTAS, bool MMA = false>
+// NR > 1 (tensor-core path, several query tokens per sequence only): an item
+// is a group of NR consecutive query rows of one sequence, whose 8 x NR
+// (row, head) columns share every K/V tile of the group's longest prefix.
+template <typename T, int D, int GT, int HS, int DEPTH, int WARPS, int MIN_CTAS, bool MMA = false,
+          int NR = 1>
 __global__ void __launch_bounds__(WARPS * 32, MIN_CTAS)
 paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int G = GT / HS;  // query heads handled by one warp
-  using C = DecodeCfg<T, D, G, GT, HS, DEPTH, WARPS, MMA>;
+  using C = DecodeCfg<T, D, G, GT, HS, DEPTH, WARPS, MMA, NR>;
   using E = Elem<T>;
   static_assert(WARPS % HS == 0, "warps per CTA must be a multiple of the head split");
   extern __shared__ __align__(128) unsigned char smem[];
@@ -396,6 +402,9 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   const bool prefill = a.query_start != nullptr;
   int* s_row = prefill ? s_len + S : nullptr;                                // [S]
   int* s_qs = s_len + 2 * S;                                                 // [rows + 1]
+  // NR > 1: first query row | (rows << 24) of each group; first group of each sequence
+  int* s_r0 = s_qs + a.num_table_rows + 1;                                   // [S]
+  int* s_gs = s_r0 + S;                                                      // [rows + 1]
 
   if (leader && lane == 0) {
 #pragma unroll
@@ -410,11 +419,34 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   // Decode: context_lens[s].  Several query tokens per sequence: s is a query
   // row; its sequence (row of the block table) is found in query_start, and
   // query j of a sequence of n tokens and Q queries sees n - Q + j + 1 tokens.
-  auto attended = [&](int s, int& row) -> int {
+  auto attended = [&](int s, int& row, int& r0nr) -> int {
     if (!prefill) {
       row = s;
+      r0nr = s | (1 << 24);
       const int n = a.context_lens[s];
       return (n < 0 || n > a.len_cap) ? -kErrContextLen : n;
+    }
+    if constexpr (NR > 1) {
+      // s is a group of up to NR consecutive query rows; it attends to the
+      // prefix of its last row
+      const int R = a.num_table_rows;
+      row = 0;
+      r0nr = 0;
+      if (s >= s_gs[R]) return 0;  // no such group (the launch sizes for the most)
+      int lo = 0, up = R - 1;      // largest sequence with s_gs[sequence] <= s
+      while (lo < up) {
+        const int mid = (lo + up + 1) >> 1;
+        if (s_gs[mid] <= s) lo = mid; else up = mid - 1;
+      }
+      row = lo;
+      const int q0 = s_qs[lo], Q = s_qs[lo + 1] - q0;
+      const int j0 = NR * (s - s_gs[lo]);
+      const int nr = min(NR, Q - j0);
+      r0nr = (q0 + j0) | (nr << 24);
+      const int n = a.context_lens[lo];
+      if (n < 0 || n > a.len_cap) return -kErrContextLen;
+      if (Q > n) return -kErrQuery;
+      return n - Q + j0 + nr;
     }
     int lo = 0, up = a.num_table_rows - 1;  // largest row with query_start[row] <= s
     while (lo < up) {
@@ -422,6 +454,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       if (s_qs[mid] <= s) lo = mid; else up = mid - 1;
     }
     row = lo;
+    r0nr = s | (1 << 24);
     const int q0 = s_qs[lo], q1 = s_qs[lo + 1];
     if (!(q0 <= s && s < q1)) return -kErrQuery;
     const int n = a.context_lens[lo];
@@ -432,6 +465,31 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   if (prefill) {
     for (int i = tid; i <= a.num_table_rows; i += WARPS * 32) s_qs[i] = a.query_start[i];
     __syncthreads();
+    if (NR > 1 && warp == 0) {
+      // groups of each sequence, ceil(Q / NR), and their prefix sums
+      const int R = a.num_table_rows;
+      int carry = 0;
+      for (int base = 0; base < R; base += 32) {
+        const int i = base + lane;
+        // a sequence's rows must lie in [0, rows of q); one that breaks this
+        // gets no group (its rows are not touched) and the error bit
+        const bool ok = i >= R || (s_qs[i] >= 0 && s_qs[i] <= s_qs[i + 1] &&
+                                   s_qs[i + 1] <= a.num_query_rows);
+        if (!ok && blockIdx.x == 0 && a.err_flag) atomicOr(a.err_flag, kErrQuery);
+        const int q = i < R && ok ? s_qs[i + 1] - s_qs[i] : 0;
+        const int ng = q > 0 ? (q + NR - 1) / NR : 0;
+        int incl = ng;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(kFull, incl, o);
+          if (lane >= o) incl += t;
+        }
+        if (i < R) s_gs[i] = carry + incl - ng;
+        carry += __shfl_sync(kFull, incl, 31);
+      }
+      if (lane == 0) s_gs[R] = carry;
+    }
+    __syncthreads();
   }
 
   // ---- prologue: block counts and their prefix sums, in tiles ----------------
@@ -441,11 +499,12 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     const int s1 = min(S, s0 + per);
     int local = 0;
     for (int s = s0; s < s1; ++s) {
-      int row;
-      int n = attended(s, row);
+      int row, r0nr;
+      int n = attended(s, row, r0nr);
       if (n < 0) n = 0;
       s_len[s] = n;
       if (prefill) s_row[s] = row;
+      if (NR > 1) s_r0[s] = r0nr;
       local += (n + kBlockSize - 1) / kBlockSize;
     }
     int incl = local;
@@ -475,14 +534,15 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   // ---- rows of empty or invalid sequences are zero --------------------------------
   for (int s = blockIdx.x; s < S; s += gridDim.x) {
     if (s_len[s] != 0) continue;
-    if (tid == 0 && a.err_flag) {
-      int row;
-      const int n = attended(s, row);
-      if (n < 0) atomicOr(a.err_flag, -n);
-    }
+    int row, r0nr;
+    const int n = attended(s, row, r0nr);
+    if (tid == 0 && a.err_flag && n < 0) atomicOr(a.err_flag, -n);
+    // (its query rows: one, or a group's; a group that does not exist has none)
+    const int nrows = NR > 1 ? (r0nr >> 24) : 1;
+    const int r0 = NR > 1 ? (r0nr & 0xffffff) : s;
     uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(a.out) +
-                                          static_cast<size_t>(s) * Hq * C::ROW);
-    for (int i = tid; i < Hq * C::ROW / 16; i += WARPS * 32) dst[i] = make_uint4(0, 0, 0, 0);
+                                          static_cast<size_t>(r0) * Hq * C::ROW);
+    for (int i = tid; i < nrows * Hq * C::ROW / 16; i += WARPS * 32) dst[i] = make_uint4(0, 0, 0, 0);
   }
 
   // ---- this worker's share of the tiles -------------------------------------------
@@ -513,11 +573,12 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   float* alpha_s = reinterpret_cast<float*>(aux + C::XS);
   StageDesc* ring_desc = reinterpret_cast<StageDesc*>(wkbase + C::DESC_OFF);
   // An item for the merge pass, listed by its first piece as a record
-  // {seq * Hkv + kv head, first range, pieces, partial slot of the first
-  // piece}: each later piece starts its range r, so its partial is in slot 2r.  Few pieces go to the one-warp list, more to the
+  // {first out row * Hkv + kv head, first range, pieces | (out rows << 24),
+  // partial slot of the first piece}: each later piece starts its range r, so
+  // its partial is in slot 2r.  Few pieces go to the one-warp list, more to the
   // one-CTA-per-head list.
-  auto list_for_merge = [&](long long ra, long long rb, long long item_a, int item) {
-    const int4 rec = make_int4(item, static_cast<int>(ra), static_cast<int>(rb - ra + 1),
+  auto list_for_merge = [&](long long ra, long long rb, long long item_a, int item, int nr = 1) {
+    const int4 rec = make_int4(item, static_cast<int>(ra), static_cast<int>(rb - ra + 1) | (nr << 24),
                                static_cast<int>(piece_slot(rg, ra, item_a)));
     if (rb - ra + 1 <= kWarpMergeMaxPieces)
       reinterpret_cast<int4*>(a.light_list)[atomicAdd(a.heavy + 4, 1)] = rec;
@@ -596,7 +657,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           // masked or zeroed after arrival); the new rows go to the staging pair
           const bool app = (e.meta & kAppend) != 0;
           fence_proxy_async_smem();  // the slot may have been written (staged rows, zeroed rows)
-          mbar_arrive_expect_tx(bar, 2 * C::TILE + (with_q ? C::QB : 0) + (app ? 2 * C::ROW : 0));
+          const int q_rows = !with_q ? 0 : NR > 1 ? (s_r0[e.seq] >> 24) : 1;
+          mbar_arrive_expect_tx(bar, 2 * C::TILE + q_rows * GT * C::ROW + (app ? 2 * C::ROW : 0));
           const int y = (e.phys * Hkv + kvh) * kBlockSize;
 #pragma unroll
           for (int hx = 0; hx < D / 64; ++hx) {
@@ -609,12 +671,17 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
             bulk_copy_g2s(dst + C::APP + C::ROW, static_cast<const char*>(a.value) + src, C::ROW,
                           bar);
           }
-          if (with_q)
-            bulk_copy_g2s(dst + 2 * C::TILE,
-                          static_cast<const char*>(a.q) +
-                              (static_cast<size_t>(e.seq) * Hq + static_cast<size_t>(kvh) * GT) *
-                                  C::ROW,
-                          C::QB, bar);
+          if (with_q) {
+            // the q rows of the item's query rows (one, or a group's)
+            const int r0nr = NR > 1 ? s_r0[e.seq] : (e.seq | (1 << 24));
+            const int r0 = r0nr & 0xffffff, nr = r0nr >> 24;
+            for (int j = 0; j < nr; ++j)
+              bulk_copy_g2s(dst + 2 * C::TILE + j * GT * C::ROW,
+                            static_cast<const char*>(a.q) +
+                                (static_cast<size_t>(r0 + j) * Hq + static_cast<size_t>(kvh) * GT) *
+                                    C::ROW,
+                            GT * C::ROW, bar);
+          }
           return true;
         }
         if (kProxyFence) fence_proxy_async_smem();
@@ -675,10 +742,13 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   // operand of S^T = K q^T (heads g; head_dim pairs 2t, 2t+1 and 2t+8, 2t+9
   // of each 16-wide slice), o^T[head_dim x heads] as C fragments (head_dim
   // g and g + 8 of each slice; heads 2t and 2t+1), and the running max / sum
-  // of heads 2t and 2t+1 (the sums over this lane's tokens only).
-  uint32_t qb[C::MT][2];
-  float oa[C::MT][4];
-  float mh[2] = {-INFINITY, -INFINITY}, lh[2] = {0.f, 0.f};
+  // of heads 2t and 2t+1 (the sums over this lane's tokens only) -- one set
+  // per query row of the item (NR).
+  uint32_t qb[NR][C::MT][2];
+  float oa[NR][C::MT][4];
+  float mh[NR][2], lh[NR][2];
+#pragma unroll
+  for (int j = 0; j < NR; ++j) mh[j][0] = mh[j][1] = -INFINITY, lh[j][0] = lh[j][1] = 0.f;
   const int mg = lane >> 2, mtq = lane & 3;
 
   for (int k = 0;; ++k) {
@@ -728,16 +798,20 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     const unsigned char* pv = pk + C::TILE;
 
     if (MMA && (flags & kFirst)) {
-      const unsigned char* pq = pk + 2 * C::TILE + mg * C::ROW + mtq * 4;
 #pragma unroll
-      for (int ks = 0; ks < C::MT; ++ks) {
-        qb[ks][0] = *reinterpret_cast<const uint32_t*>(pq + ks * 32);
-        qb[ks][1] = *reinterpret_cast<const uint32_t*>(pq + ks * 32 + 16);
+      for (int j = 0; j < NR; ++j) {
+        // (a group's missing second row reads stale q; its columns are masked)
+        const unsigned char* pq = pk + 2 * C::TILE + (j * GT + mg) * C::ROW + mtq * 4;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) oa[ks][e] = 0.f;
+        for (int ks = 0; ks < C::MT; ++ks) {
+          qb[j][ks][0] = *reinterpret_cast<const uint32_t*>(pq + ks * 32);
+          qb[j][ks][1] = *reinterpret_cast<const uint32_t*>(pq + ks * 32 + 16);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) oa[j][ks][e] = 0.f;
+        }
+        mh[j][0] = mh[j][1] = -INFINITY;
+        lh[j][0] = lh[j][1] = 0.f;
       }
-      mh[0] = mh[1] = -INFINITY;
-      lh[0] = lh[1] = 0.f;
       poisoned = false;
     } else if (flags & kFirst) {
       const unsigned char* pq = pk + 2 * C::TILE;
@@ -786,7 +860,22 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
         }
         const uint32_t kb = smem_addr(pk), vb = kb + C::TILE;
         const int lr = lane & 7, lm = lane >> 3;  // ldmatrix: row within matrix, matrix
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        // a group of NR query rows: row j sees token t of this tile iff
+        // t <= lim[j] (its causal limit); a missing row sees nothing
+        int lim[NR];
+        if constexpr (NR > 1) {
+          const int v = d.seq;
+          const int len = s_len[v];
+          const long long item_a =
+              s_start[v] + static_cast<long long>(kvh) * ((len + kBlockSize - 1) / kBlockSize);
+          const int tb = static_cast<int>(d.g - item_a) * kBlockSize;
+          const int nr = s_r0[v] >> 24;
+#pragma unroll
+          for (int j = 0; j < NR; ++j) lim[j] = j < nr ? len - nr + j - tb : -1;
+        }
+        float sc[NR][4];
+#pragma unroll
+        for (int j = 0; j < NR; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < C::MT; ++ks) {
           // matrices: tokens 0-7 / 8-15 x head_dim ks*16 + 0-7, then + 8-15
@@ -794,44 +883,52 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           const int ch = ks * 2 + (lm >> 1);
           uint32_t af[4];
           ldmatrix_x4(kb + (ch >> 3) * 2048 + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4), af);
-          mma_bf16_16816(sc, af, qb[ks][0], qb[ks][1]);
+#pragma unroll
+          for (int j = 0; j < NR; ++j) mma_bf16_16816(sc[j], af, qb[j][ks][0], qb[j][ks][1]);
         }
-        // sc: tokens mg, mg, mg+8, mg+8 x heads 2t, 2t+1, 2t, 2t+1 (t = mtq)
-        float x[4];
+        // sc[j]: tokens mg, mg, mg+8, mg+8 x heads 2t, 2t+1, 2t, 2t+1 (t = mtq)
+        uint32_t b0[NR], b1[NR];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int tok = mg + (e >> 1) * 8;
-          x[e] = (!MASK || tok < rows) ? sc[e] * a.scale_log2 : -INFINITY;
-        }
-        float mx[2] = {fmaxf(x[0], x[2]), fmaxf(x[1], x[3])};
+        for (int j = 0; j < NR; ++j) {
+          float x[4];
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          mx[0] = fmaxf(mx[0], __shfl_xor_sync(kFull, mx[0], off));
-          mx[1] = fmaxf(mx[1], __shfl_xor_sync(kFull, mx[1], off));
-        }
+          for (int e = 0; e < 4; ++e) {
+            const int tok = mg + (e >> 1) * 8;
+            const bool seen = NR > 1 ? tok <= lim[j] : (!MASK || tok < rows);
+            x[e] = seen ? sc[j][e] * a.scale_log2 : -INFINITY;
+          }
+          float mx[2] = {fmaxf(x[0], x[2]), fmaxf(x[1], x[3])};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (mx[j] > mh[j] + kRescaleThreshold) {
-            const float al = exp2f(mh[j] - mx[j]);
-            mh[j] = mx[j];
-            lh[j] *= al;
+          for (int off = 4; off < 32; off <<= 1) {
+            mx[0] = fmaxf(mx[0], __shfl_xor_sync(kFull, mx[0], off));
+            mx[1] = fmaxf(mx[1], __shfl_xor_sync(kFull, mx[1], off));
+          }
 #pragma unroll
-            for (int mt = 0; mt < C::MT; ++mt) {
-              oa[mt][j] *= al;
-              oa[mt][j + 2] *= al;
+          for (int c = 0; c < 2; ++c) {
+            if (mx[c] > mh[j][c] + kRescaleThreshold) {
+              const float al = exp2f(mh[j][c] - mx[c]);
+              mh[j][c] = mx[c];
+              lh[j][c] *= al;
+#pragma unroll
+              for (int mt = 0; mt < C::MT; ++mt) {
+                oa[j][mt][c] *= al;
+                oa[j][mt][c + 2] *= al;
+              }
             }
           }
+          __syncwarp();
+          // (a logit masked out weighs 0, also while its running max is still -inf)
+          auto wgt = [](float xv, float m) { return xv == -INFINITY ? 0.f : exp2f(xv - m); };
+          const __nv_bfloat162 p01 =
+              __floats2bfloat162_rn(wgt(x[0], mh[j][0]), wgt(x[1], mh[j][1]));
+          const __nv_bfloat162 p23 =
+              __floats2bfloat162_rn(wgt(x[2], mh[j][0]), wgt(x[3], mh[j][1]));
+          // the sums take the weights as rounded for the product
+          lh[j][0] += __low2float(p01) + __low2float(p23);
+          lh[j][1] += __high2float(p01) + __high2float(p23);
+          b0[j] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&p01));
+          b1[j] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&p23));
         }
-        __syncwarp();
-        const __nv_bfloat162 p01 =
-            __floats2bfloat162_rn(exp2f(x[0] - mh[0]), exp2f(x[1] - mh[1]));
-        const __nv_bfloat162 p23 =
-            __floats2bfloat162_rn(exp2f(x[2] - mh[0]), exp2f(x[3] - mh[1]));
-        // the sums take the weights as rounded for the product
-        lh[0] += __low2float(p01) + __low2float(p23);
-        lh[1] += __high2float(p01) + __high2float(p23);
-        const uint32_t b0 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&p01));
-        const uint32_t b1 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&p23));
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
           // matrices (transposed on load): tokens 0-7 x head_dim mt*16 + 0-7 /
@@ -840,7 +937,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           const int ch = mt * 2 + (lm & 1);
           uint32_t af[4];
           ldmatrix_x4_trans(vb + (ch >> 3) * 2048 + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4), af);
-          mma_bf16_16816(oa[mt], af, b0, b1);
+#pragma unroll
+          for (int j = 0; j < NR; ++j) mma_bf16_16816(oa[j][mt], af, b0[j], b1[j]);
         }
       } else if constexpr (G == 1) {
         // ---- one query head: every lane keeps the logits of its row group
@@ -982,12 +1080,6 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
 
     // ---- end of a piece: write the output or a partial -------------------------
     if (MMA && (flags & kLast)) {
-      float lt[2] = {lh[0], lh[1]};
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        lt[0] += __shfl_xor_sync(kFull, lt[0], off);
-        lt[1] += __shfl_xor_sync(kFull, lt[1], off);
-      }
       const bool bad = __any_sync(kFull, poisoned);
       const int s = d.seq;
       const int nb = (s_len[s] + kBlockSize - 1) / kBlockSize;
@@ -995,38 +1087,52 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       const long long ra = rg.of(item_a);
       const long long rb = rg.of(item_a + nb - 1);
       const int h0 = 2 * mtq;  // this lane's heads h0, h0 + 1; head_dim mg, mg + 8 of each slice
-      if (ra == rb) {
-        // the whole (seq, kv head) was this piece: normalise and store
-        T* dst = static_cast<T*>(a.out) +
-                 (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * GT + h0) * D + mg;
-        const float i0 = bad ? 0.f : 1.f / lt[0], i1 = bad ? 0.f : 1.f / lt[1];
+      // the item's query rows: out rows r0 .. r0 + nr - 1 (decode: the sequence's)
+      const int r0nr = NR > 1 ? s_r0[s] : (s | (1 << 24));
+      const int r0 = r0nr & 0xffffff, nr = r0nr >> 24;
+      const long long r = rg.of(d.g);
+      const long long sl = piece_slot(rg, r, item_a);
 #pragma unroll
-        for (int mt = 0; mt < C::MT; ++mt) {
-          dst[mt * 16] = static_cast<T>(oa[mt][0] * i0);
-          dst[D + mt * 16] = static_cast<T>(oa[mt][1] * i1);
-          dst[mt * 16 + 8] = static_cast<T>(oa[mt][2] * i0);
-          dst[D + mt * 16 + 8] = static_cast<T>(oa[mt][3] * i1);
-        }
-      } else {
-        // a partial: no fence or counter here; the merge pass, which starts once
-        // this grid has finished, combines the pieces
-        const long long r = rg.of(d.g);
-        const long long sl = piece_slot(rg, r, item_a);
-        float* wo = a.ws_o + (sl * GT + h0) * D + mg;
+      for (int j = 0; j < NR; ++j) {
+        float lt[2] = {lh[j][0], lh[j][1]};
 #pragma unroll
-        for (int mt = 0; mt < C::MT; ++mt) {
-          wo[mt * 16] = oa[mt][0];
-          wo[D + mt * 16] = oa[mt][1];
-          wo[mt * 16 + 8] = oa[mt][2];
-          wo[D + mt * 16 + 8] = oa[mt][3];
+        for (int off = 4; off < 32; off <<= 1) {
+          lt[0] += __shfl_xor_sync(kFull, lt[0], off);
+          lt[1] += __shfl_xor_sync(kFull, lt[1], off);
         }
-        if (mg == 0) {
-          a.ws_ml[sl * GT + h0] = make_float2(mh[0], bad ? -1.f : lt[0]);
-          a.ws_ml[sl * GT + h0 + 1] = make_float2(mh[1], bad ? -1.f : lt[1]);
+        if (j >= nr) continue;
+        if (ra == rb) {
+          // the whole item was this piece: normalise and store
+          T* dst = static_cast<T*>(a.out) +
+                   (static_cast<size_t>(r0 + j) * Hq + static_cast<size_t>(kvh) * GT + h0) * D + mg;
+          const float i0 = bad ? 0.f : 1.f / lt[0], i1 = bad ? 0.f : 1.f / lt[1];
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt) {
+            dst[mt * 16] = static_cast<T>(oa[j][mt][0] * i0);
+            dst[D + mt * 16] = static_cast<T>(oa[j][mt][1] * i1);
+            dst[mt * 16 + 8] = static_cast<T>(oa[j][mt][2] * i0);
+            dst[D + mt * 16 + 8] = static_cast<T>(oa[j][mt][3] * i1);
+          }
+        } else {
+          // a partial (columns j * 8 + head of the slot): no fence or counter
+          // here; the merge pass, which starts once this grid has finished,
+          // combines the pieces
+          float* wo = a.ws_o + (sl * (NR * GT) + j * GT + h0) * D + mg;
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt) {
+            wo[mt * 16] = oa[j][mt][0];
+            wo[D + mt * 16] = oa[j][mt][1];
+            wo[mt * 16 + 8] = oa[j][mt][2];
+            wo[D + mt * 16 + 8] = oa[j][mt][3];
+          }
+          if (mg == 0) {
+            a.ws_ml[sl * (NR * GT) + j * GT + h0] = make_float2(mh[j][0], bad ? -1.f : lt[0]);
+            a.ws_ml[sl * (NR * GT) + j * GT + h0 + 1] = make_float2(mh[j][1], bad ? -1.f : lt[1]);
+          }
         }
-        // the merge pass combines the pieces; the first piece lists the item
-        if (r == ra && lane == 0) list_for_merge(ra, rb, item_a, s * Hkv + kvh);
       }
+      // the merge pass combines the pieces; the first piece lists the item
+      if (ra != rb && r == ra && lane == 0) list_for_merge(ra, rb, item_a, r0 * Hkv + kvh, nr);
     } else if (flags & kLast) {
 #pragma unroll
       for (int off = C::LPR; off < 32; off <<= 1)

@@ -21,7 +21,9 @@ namespace pa {
 // Launched right behind the decode kernel with programmatic dependent launch;
 // griddepcontrol.wait returns once the decode grid has finished and its
 // writes are visible.  The last CTA to finish resets the item list.
-template <typename T, int D, int G>
+// G partial columns per item: GH query heads of a KV head for each of the
+// item's G / GH query rows (one row in decode).
+template <typename T, int D, int G, int GH = G>
 __global__ void __launch_bounds__(kMergeThreads)
 paged_decode_merge_kernel(const DecodeArgs a, int workers) {
   constexpr int GROUPS = kMergeThreads / 32;
@@ -51,8 +53,9 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
     for (int it = it0; it < light; it += gridDim.x * GROUPS) {
       const int4 rec =
           it == it0 ? rec0 : __ldcg(reinterpret_cast<const int4*>(a.light_list) + it);
-      const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
-      const int np = rec.z;  // (at most NP: listed so)
+      const int r0 = rec.x / Hkv, kvh = rec.x - r0 * Hkv;  // first out row, KV head
+      const int np = rec.z & 0xffffff;  // (at most NP: listed so)
+      const int nr = rec.z >> 24;       // out rows of the item
       auto slot_of = [&](int r) -> long long {  // piece r's partial slot
         return r == 0 ? rec.w : 2 * (static_cast<long long>(rec.y) + r);
       };
@@ -98,22 +101,27 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
           }
         }
       }
-      T* dst = static_cast<T*>(a.out) +
-               (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G) * D + lane * DPL;
+      // column h is head h % GH of out row r0 + h / GH
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const bool hb = (bad >> h) & 1;
         const float inv = hb ? 0.f : 1.f / L[h];
+        if (h / GH >= nr) continue;
+        T* dst = static_cast<T*>(a.out) +
+                 (static_cast<size_t>(r0 + h / GH) * Hq + static_cast<size_t>(kvh) * GH + h % GH) * D +
+                 lane * DPL;
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) dst[h * D + e] = static_cast<T>(hb ? 0.f : acc[h][e] * inv);
+        for (int e = 0; e < DPL; ++e) dst[e] = static_cast<T>(hb ? 0.f : acc[h][e] * inv);
       }
     }
     // items of many pieces: one CTA per (item, head)
     for (int p = blockIdx.x; p < count * G; p += gridDim.x) {
       const int4 rec = __ldcg(reinterpret_cast<const int4*>(a.heavy_list) + p / G);
       const int hl = p % G;
-      const int s = rec.x / Hkv, kvh = rec.x - s * Hkv;
-      const long long ra = rec.y, rb = ra + rec.z - 1;
+      const int r0 = rec.x / Hkv, kvh = rec.x - r0 * Hkv;  // first out row, KV head
+      const long long ra = rec.y, rb = ra + (rec.z & 0xffffff) - 1;
+      const int nr = rec.z >> 24;
+      if (hl / GH >= nr) continue;  // (the same for the whole CTA)
       auto slot_of = [&](long long r) -> long long { return r == ra ? rec.w : 2 * r; };
 
       // each warp takes pieces ra + grp, + GROUPS, ..., four at a time with all
@@ -182,7 +190,9 @@ paged_decode_merge_kernel(const DecodeArgs a, int workers) {
           for (int d = 0; d < DPL; ++d) r[d] = fmaf(f, s_acc[g][lane * DPL + d], r[d]);
         }
         T* dst = static_cast<T*>(a.out) +
-                 (static_cast<size_t>(s) * Hq + static_cast<size_t>(kvh) * G + hl) * D + lane * DPL;
+                 (static_cast<size_t>(r0 + hl / GH) * Hq + static_cast<size_t>(kvh) * GH + hl % GH) *
+                     D +
+                 lane * DPL;
 #pragma unroll
         for (int d = 0; d < DPL; ++d) dst[d] = static_cast<T>(bt ? 0.f : r[d] / Lt);
       }

@@ -72,6 +72,7 @@ struct DecodeArgs {
   // query_start[num_table_rows + 1] maps them to the block-table rows
   const int32_t* query_start;
   int num_table_rows;
+  int num_query_rows;  // rows of q and out (several query tokens per sequence)
   // tensor-core path only: the caches as 2-D tensors [num_blocks * Hkv * 16][head_dim]
   // read in boxes of 16 rows x 128 bytes with the 128-byte swizzle
   CUtensorMap tm_k;
@@ -100,9 +101,13 @@ struct DecodeKernelInfo {
   int depth;        // ring slots per worker
   int cta_bytes;    // dynamic shared memory per CTA, without the per-sequence arrays
   bool tma;         // reads tiles through the tm_k / tm_v tensor maps
+  int rows_per_item;  // query rows an item groups (several query tokens per sequence)
 };
 
 bool decode_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);
+// The kernel for several query tokens per sequence when it differs from the
+// decode one (false: use decode_kernel_*).
+bool prefill_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);
 
 // Bytes at the start of a decode workspace that must be zero when a call
 // begins (the merge-pass header and the piece counters).

@@ -29,7 +29,7 @@ ERRBIT_QUERY = 32
 
 EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_init",
             "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_decode_append",
-            "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks")
+            "pa_prefill", "pa_prefill_workspace_size", "pa_reshape_and_cache", "pa_copy_blocks")
 
 # size of the library's fixed scratch array used by pa_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -66,6 +66,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode.restype = i
     lib.pa_decode_noalloc.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, vp]
+    lib.pa_prefill_workspace_size.restype = i
+    lib.pa_prefill_workspace_size.argtypes = [i] * 8 + [ctypes.POINTER(sz)]
     lib.pa_prefill.restype = i
     lib.pa_prefill.argtypes = [vp] * 7 + [i] * 9 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode_append.restype = i
@@ -132,6 +134,19 @@ def make_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim:
     n = workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
                        partition_size, dtype)
     return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def make_prefill_workspace(num_seqs: int, num_query_tokens: int, num_q_heads: int,
+                           num_kv_heads: int, head_dim: int, max_context_len: int,
+                           partition_size: int = 0, dtype: torch.dtype = torch.bfloat16,
+                           device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size ``pa_prefill`` needs."""
+    n = ctypes.c_size_t(0)
+    _check(library().pa_prefill_workspace_size(
+        num_seqs, num_query_tokens, num_q_heads, num_kv_heads, head_dim, int(max_context_len),
+        int(partition_size), PA_BF16 if dtype == torch.bfloat16 else PA_F32, ctypes.byref(n)),
+        "pa_prefill_workspace_size")
+    return torch.zeros(max(n.value, 16), dtype=torch.uint8, device=device)
 
 
 def launch_config(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,

@@ -104,6 +104,11 @@ def test_prefill_rejects_bad_arguments_on_the_host(lib):
     assert call(T=-1) == ops.PA_ERR_INVALID_ARG
     assert call(Hq=6) == ops.PA_ERR_UNSUPPORTED          # group 3
     assert call(qs=None, T=0) == ops.PA_OK               # nothing to do
+    n = ctypes.c_size_t(0)
+    assert lib.pa_prefill_workspace_size(2, 8, 8, 2, 128, 64, 0, ops.PA_BF16, None) == \
+        ops.PA_ERR_INVALID_ARG
+    assert lib.pa_prefill_workspace_size(2, -1, 8, 2, 128, 64, 0, ops.PA_BF16,
+                                         ctypes.byref(n)) == ops.PA_ERR_INVALID_ARG
 
 
 def test_workspace_queries_validate_first(lib):
