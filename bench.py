@@ -295,8 +295,12 @@ def run_ours(args, rank: int, world: int):
     else:
         ws = ops.make_workspace(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
                                 w.max_context_len, ps, tdt, device=dev)
-    cfg = ops.launch_config(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                            w.max_context_len, ps, tdt)
+    if prefill:
+        cfg = ops.prefill_launch_config(w.num_seqs, rows, w.num_q_heads, w.num_kv_heads,
+                                        w.head_dim, w.max_context_len, ps, tdt)
+    else:
+        cfg = ops.launch_config(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                w.max_context_len, ps, tdt)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     evict = torch.ones(128 << 20, dtype=torch.int32, device=dev)   # 512 MiB, read only
 

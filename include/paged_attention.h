@@ -48,7 +48,7 @@ extern "C" {
 typedef enum pa_status {
     PA_OK = 0,
     PA_ERR_INVALID_ARG = 1,  /* a null pointer, a negative size, a misaligned buffer ... */
-    PA_ERR_UNSUPPORTED = 2,  /* a valid shape this build has no kernel for              */
+    PA_ERR_UNSUPPORTED = 2,  /* a valid shape the library has no kernel for            */
     PA_ERR_WORKSPACE = 3,    /* the decode workspace is missing or too small            */
     PA_ERR_CUDA = 4          /* the CUDA runtime refused a query or a launch            */
 } pa_status;
@@ -264,6 +264,12 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
 pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_q_heads,
                                     int num_kv_heads, int head_dim, int max_context_len,
                                     int partition_size, pa_dtype dtype, size_t *bytes);
+
+/* The launch pa_prefill would make (as pa_decode_launch_config). */
+pa_status pa_prefill_launch_config(int num_seqs, int num_query_tokens, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int max_context_len,
+                                   int partition_size, pa_dtype dtype, int *grid,
+                                   int *warps_per_cta, int *pipeline_depth, int *smem_bytes);
 
 pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, const int32_t *context_lens,

@@ -315,6 +315,24 @@ pa_status pa_decode_launch_config(int num_seqs, int num_q_heads, int num_kv_head
   return PA_OK;
 }
 
+pa_status pa_prefill_launch_config(int num_seqs, int num_query_tokens, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int max_context_len,
+                                   int partition_size, pa_dtype dtype, int* grid,
+                                   int* warps_per_cta, int* pipeline_depth, int* smem_bytes) {
+  if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
+  DecodePlan p;
+  const int items = prefill_items(num_seqs, num_query_tokens, num_q_heads, num_kv_heads,
+                                  head_dim, dtype);
+  const pa_status st = make_plan(items, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                 partition_size, dtype, &p, num_seqs > 0 ? num_seqs : 1);
+  if (st != PA_OK) return st;
+  if (grid) *grid = p.grid;
+  if (warps_per_cta) *warps_per_cta = p.kernel.warps;
+  if (pipeline_depth) *pipeline_depth = p.kernel.depth;
+  if (smem_bytes) *smem_bytes = static_cast<int>(p.smem);
+  return PA_OK;
+}
+
 namespace {
 
 // pa_decode and pa_decode_append: key/value null = plain decode.

@@ -29,7 +29,8 @@ ERRBIT_QUERY = 32
 
 EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_init",
             "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_decode_append",
-            "pa_prefill", "pa_prefill_workspace_size", "pa_reshape_and_cache", "pa_copy_blocks")
+            "pa_prefill", "pa_prefill_workspace_size", "pa_prefill_launch_config",
+            "pa_reshape_and_cache", "pa_copy_blocks")
 
 # size of the library's fixed scratch array used by pa_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -66,6 +67,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_decode.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, sz, vp, vp]
     lib.pa_decode.restype = i
     lib.pa_decode_noalloc.argtypes = [vp] * 6 + [i] * 8 + [f, i, i, vp, vp]
+    lib.pa_prefill_launch_config.restype = i
+    lib.pa_prefill_launch_config.argtypes = [i] * 8 + [ctypes.POINTER(i)] * 4
     lib.pa_prefill_workspace_size.restype = i
     lib.pa_prefill_workspace_size.argtypes = [i] * 8 + [ctypes.POINTER(sz)]
     lib.pa_prefill.restype = i
@@ -158,6 +161,20 @@ def launch_config(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: 
                                              max_context_len, partition_size, code,
                                              *[ctypes.byref(v) for v in vals]),
            "pa_decode_launch_config")
+    return dict(zip(("grid", "warps_per_cta", "pipeline_depth", "smem_bytes"),
+                    (v.value for v in vals)))
+
+
+def prefill_launch_config(num_seqs: int, num_query_tokens: int, num_q_heads: int,
+                          num_kv_heads: int, head_dim: int, max_context_len: int,
+                          partition_size: int = 0, dtype: torch.dtype = torch.bfloat16) -> dict:
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    code = PA_BF16 if dtype == torch.bfloat16 else PA_F32
+    _check(library().pa_prefill_launch_config(num_seqs, num_query_tokens, num_q_heads,
+                                              num_kv_heads, head_dim, max_context_len,
+                                              partition_size, code,
+                                              *[ctypes.byref(v) for v in vals]),
+           "pa_prefill_launch_config")
     return dict(zip(("grid", "warps_per_cta", "pipeline_depth", "smem_bytes"),
                     (v.value for v in vals)))
 
