@@ -138,6 +138,21 @@ def test_many_sequences():
     assert_attention_close(t["out"], ref, "bf16", "3000 sequences")
 
 
+def test_very_large_batch():
+    """12000 short sequences: the per-sequence arrays take most of an SM's
+    shared memory, leaving one CTA per SM."""
+    rng = np.random.default_rng(8)
+    lens = rng.integers(0, 40, size=12000)
+    w = make_workload(rng, name="huge", dtype="bf16", num_q_heads=2, num_kv_heads=2, head_dim=64,
+                      context_lens=lens, num_blocks=int(sum(-(-lens // 16))) + 10)
+    ref, _ = oracle.paged_decode(w.q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens,
+                                 scale=w.scale, dtype=w.dtype)
+    t, err, ws = run_gpu(w)
+    assert err == 0
+    assert_attention_close(t["out"], ref, "bf16", "12000 sequences")
+    assert counters_zero(w, ws)
+
+
 def test_all_empty_and_single_token():
     w = random_workload(5, dtype="f32", num_q_heads=4, num_kv_heads=4, head_dim=64, lens=[1, 1])
     t, err, _ = run_gpu(w)
