@@ -63,13 +63,6 @@ constexpr int kMaxOwnRanges = 4;  // range starts a warp keeps in shared memory
 #endif
 constexpr bool kProxyFence = PA_PROXY_FENCE != 0;
 
-// Tensor-core path, one query row per item: split the QK^T accumulation over
-// two accumulators (even / odd head_dim slices) to halve the MMA chain.
-#ifndef PA_MMA_SPLIT_ACC
-#define PA_MMA_SPLIT_ACC 1
-#endif
-constexpr bool kMmaSplitAcc = PA_MMA_SPLIT_ACC != 0;
-
 // -- element conversion ---------------------------------------------------------
 template <typename T>
 struct Elem;
@@ -880,14 +873,9 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
           for (int j = 0; j < NR; ++j) lim[j] = j < nr ? len - nr + j - tb : -1;
         }
-        // (with one row, even and odd slices of head_dim go to two accumulators:
-        // two dependent MMA chains of half the length)
-        constexpr int NA = (NR == 1 && kMmaSplitAcc) ? 2 : 1;
-        float sc[NR][4], sc2[NA][4];
+        float sc[NR][4];
 #pragma unroll
         for (int j = 0; j < NR; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-#pragma unroll
-        for (int j = 0; j < NA; ++j) sc2[j][0] = sc2[j][1] = sc2[j][2] = sc2[j][3] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < C::MT; ++ks) {
           // matrices: tokens 0-7 / 8-15 x head_dim ks*16 + 0-7, then + 8-15
@@ -895,16 +883,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           const int ch = ks * 2 + (lm >> 1);
           uint32_t af[4];
           ldmatrix_x4(kb + (ch >> 3) * 2048 + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4), af);
-          if constexpr (NA == 2) {
-            mma_bf16_16816(sc2[ks & 1], af, qb[0][ks][0], qb[0][ks][1]);
-          } else {
 #pragma unroll
-            for (int j = 0; j < NR; ++j) mma_bf16_16816(sc[j], af, qb[j][ks][0], qb[j][ks][1]);
-          }
-        }
-        if constexpr (NA == 2) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sc[0][e] = sc2[0][e] + sc2[1][e];
+          for (int j = 0; j < NR; ++j) mma_bf16_16816(sc[j], af, qb[j][ks][0], qb[j][ks][1]);
         }
         // sc[j]: tokens mg, mg, mg+8, mg+8 x heads 2t, 2t+1, 2t, 2t+1 (t = mtq)
         uint32_t b0[NR], b1[NR];
