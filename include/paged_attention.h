@@ -70,6 +70,10 @@ typedef enum pa_dtype {
                                      the decode workspace must be re-initialised           */
 #define PA_ERRBIT_QUERY       32  /* pa_prefill: a sequence's query_start pair out of order
                                      or more query rows than tokens: its rows written as 0 */
+#define PA_ERRBIT_GROUP       64  /* pa_decode_shared_prefix: a group entry that does not
+                                     match the block tables (or a sequence two groups list)
+                                     was ignored; those sequences were attended in full, so
+                                     the output is still exact                            */
 
 /* Human-readable name of a status code (static storage). */
 const char *pa_status_str(pa_status status);
@@ -278,6 +282,69 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
                      int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
                      int partition_size, pa_dtype dtype, void *workspace,
                      size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Prefix-deduplicated decode
+ * ------------------------------------------------------------------------
+ * Requests with a common prefix hold the same physical blocks for it
+ * (day-9 post, section "Idea 1: PagedAttention", sharing).  pa_decode reads
+ * such a block once per sequence; pa_decode_shared_prefix reads it once per
+ * group: a tensor-core pass computes, for every (member, query head) of a
+ * group and the group's shared blocks, the online-softmax state (running
+ * max, sum of weights, unnormalised output), and the decode kernel goes on
+ * from that state over each sequence's remaining blocks.  Attention over the
+ * union of two token sets is the log-sum-exp combination of the two, so the
+ * result is that of pa_decode (or, with key/value, pa_decode_append) up to
+ * rounding: the shared part's weights are rounded to bf16 for the product,
+ * as on the tensor-core decode path.  bf16 only (fp32 returns
+ * PA_ERR_UNSUPPORTED).
+ *
+ * The groups: group g lists its member sequences in
+ *   group_seqs[group_start[g] .. group_start[g+1])   (device int32)
+ * and shares its first group_blocks[g] logical blocks (device int32): every
+ * member's block table holds the same physical ids there, and every member
+ * has at least one token after them (16 * group_blocks[g] < n).  The pass
+ * checks both on the device; a member that fails, or a sequence that two
+ * groups list, is attended in full by the decode kernel and PA_ERRBIT_GROUP
+ * is set.  A sequence in no group is attended as by pa_decode.
+ * num_listed = group_start[num_groups]; num_groups <= 16384.
+ *
+ * pa_shared_prefix_plan finds such groups on the HOST (its pointers are
+ * host pointers, unlike every other entry point's): sequences whose first
+ * physical block is the same form a candidate group, which shares the
+ * longest run of leading blocks all its members hold, capped so that each
+ * keeps one token of its own.  Groups of one member, or sharing fewer than
+ * min_shared_blocks blocks, are dropped.  Output arrays: group_seqs and
+ * group_blocks of num_seqs entries, group_start of num_seqs + 1.  Groups are
+ * ordered by their first member, members by sequence index.
+ *
+ * Workspace: pa_shared_prefix_workspace_size() bytes, zero-filled before
+ * first use (pa_decode_workspace_init); the calls leave it ready for the
+ * next one.  Everything else is as in pa_decode / pa_decode_append.
+ */
+pa_status pa_shared_prefix_plan(const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int max_blocks_per_seq, int block_size,
+                                int min_shared_blocks, int32_t *group_seqs,
+                                int32_t *group_start, int32_t *group_blocks, int *num_groups,
+                                int *num_listed);
+
+pa_status pa_shared_prefix_workspace_size(int num_seqs, int num_listed, int num_q_heads,
+                                          int num_kv_heads, int head_dim,
+                                          int max_blocks_per_seq, int max_context_len,
+                                          int partition_size, pa_dtype dtype, size_t *bytes);
+
+/* key, value: NULL for plain decode, or both given for the fused slot write
+ * of pa_decode_append. */
+pa_status pa_decode_shared_prefix(void *out, const void *q, const void *key, const void *value,
+                                  void *k_cache, void *v_cache, const int32_t *block_tables,
+                                  const int32_t *context_lens, const int32_t *group_seqs,
+                                  const int32_t *group_start, const int32_t *group_blocks,
+                                  int num_groups, int num_listed, int num_seqs, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int num_blocks, int max_context_len,
+                                  float scale, int partition_size, pa_dtype dtype,
+                                  void *workspace, size_t workspace_bytes, int32_t *err_flag,
+                                  void *stream);
 
 /* ------------------------------------------------------------------------
  * Block copy-on-write (copy_blocks)

@@ -33,6 +33,7 @@ static_assert(pa::kErrSlot == PA_ERRBIT_SLOT, "error bit mismatch");
 static_assert(pa::kErrPair == PA_ERRBIT_PAIR, "error bit mismatch");
 static_assert(pa::kErrTimeout == PA_ERRBIT_TIMEOUT, "error bit mismatch");
 static_assert(pa::kErrQuery == PA_ERRBIT_QUERY, "error bit mismatch");
+static_assert(pa::kErrGroup == PA_ERRBIT_GROUP, "error bit mismatch");
 
 namespace {
 
@@ -168,9 +169,10 @@ pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, in
 
 // table_rows >= 0: several query tokens per sequence; num_seqs counts query
 // rows and the kernel also keeps their table rows and query_start on chip.
+// shared_prefix: the kernel keeps each sequence's block offset on chip.
 pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                     int max_context_len, int partition_size, pa_dtype dtype, DecodePlan* p,
-                    int table_rows = -1) {
+                    int table_rows = -1, bool shared_prefix = false) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -198,6 +200,7 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     if (p->kernel.rows_per_item > 1)
       seq_ints += static_cast<size_t>(num_seqs) + table_rows + 1;  // group rows, group starts
   }
+  if (shared_prefix) seq_ints += static_cast<size_t>(num_seqs);  // blocks attended already
   const size_t seq_bytes = round_up(seq_ints * sizeof(int), 16);
   p->smem = static_cast<size_t>(p->kernel.cta_bytes) + seq_bytes;
   if (p->smem > static_cast<size_t>(dev.smem_optin)) return PA_ERR_UNSUPPORTED;
@@ -344,7 +347,8 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
                       int num_blocks, int max_context_len, float scale, int partition_size,
                       pa_dtype dtype, void* workspace, size_t workspace_bytes,
                       int32_t* err_flag, void* stream, const int32_t* query_start = nullptr,
-                      int table_rows = -1, int query_rows = 0) {
+                      int table_rows = -1, int query_rows = 0,
+                      const pa::SharedPrefixLaunch* pre = nullptr) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -361,7 +365,8 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
     return PA_ERR_UNSUPPORTED;
   DecodePlan p;
   if ((st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                      partition_size, dtype, &p, query_start ? table_rows : -1)) != PA_OK)
+                      partition_size, dtype, &p, query_start ? table_rows : -1,
+                      pre != nullptr)) != PA_OK)
     return st;
   if (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace))
     return PA_ERR_WORKSPACE;
@@ -395,6 +400,9 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
   args.query_start = query_start;
   args.num_table_rows = query_start ? table_rows : num_seqs;
   args.num_query_rows = query_start ? query_rows : num_seqs;
+  args.pre_blocks = pre ? pre->pre_blocks : nullptr;
+  args.pre_o = pre ? pre->pre_o : nullptr;
+  args.pre_ml = pre ? pre->pre_ml : nullptr;
   if (p.kernel.tma) {
     // tile coordinates are 32-bit: row (block * Hkv + kv head) * 16 of the 2-D view
     const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
@@ -478,6 +486,94 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
                      max_blocks_per_seq, num_blocks, max_context_len, scale, partition_size,
                      dtype, workspace, workspace_bytes, err_flag, stream, query_start, num_seqs,
                      num_query_tokens);
+}
+
+pa_status pa_shared_prefix_workspace_size(int num_seqs, int num_listed, int num_q_heads,
+                                          int num_kv_heads, int head_dim,
+                                          int max_blocks_per_seq, int max_context_len,
+                                          int partition_size, pa_dtype dtype, size_t* bytes) {
+  if (!bytes || num_listed < 0 || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
+  if (dtype != PA_BF16) return dtype == PA_F32 ? PA_ERR_UNSUPPORTED : PA_ERR_INVALID_ARG;
+  DecodePlan p;
+  const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                 partition_size, dtype, &p, -1, true);
+  if (st != PA_OK) return st;
+  const size_t extra = pa::shared_prefix_workspace_bytes(num_seqs, num_listed, num_q_heads,
+                                                         head_dim, max_blocks_per_seq);
+  if (extra == 0) return PA_ERR_UNSUPPORTED;
+  *bytes = round_up(p.ws_bytes, 256) + extra;
+  return PA_OK;
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, const void* value,
+                                  void* k_cache, void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, const int32_t* group_seqs,
+                                  const int32_t* group_start, const int32_t* group_blocks,
+                                  int num_groups, int num_listed, int num_seqs, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int num_blocks, int max_context_len,
+                                  float scale, int partition_size, pa_dtype dtype,
+                                  void* workspace, size_t workspace_bytes, int32_t* err_flag,
+                                  void* stream) {
+  pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                    max_context_len, partition_size, dtype);
+  if (st != PA_OK) return st;
+  if (dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (num_groups < 0 || num_listed < 0 || (key == nullptr) != (value == nullptr))
+    return PA_ERR_INVALID_ARG;
+  if (max_blocks_per_seq <= 0 || num_blocks <= 0 || block_size <= 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (num_groups > 0 && (!group_seqs || !group_start || !group_blocks || num_listed == 0))
+    return PA_ERR_INVALID_ARG;
+  if (num_groups > 16384) return PA_ERR_UNSUPPORTED;  // (the pass keeps one int per group on chip)
+  if (key && (!aligned16(key) || !aligned16(value))) return PA_ERR_INVALID_ARG;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  size_t need = 0;
+  if ((st = pa_shared_prefix_workspace_size(num_seqs, num_listed, num_q_heads, num_kv_heads,
+                                            head_dim, max_blocks_per_seq, max_context_len,
+                                            partition_size, dtype, &need)) != PA_OK)
+    return st;
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+  DecodePlan p;
+  if ((st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                      partition_size, dtype, &p, -1, true)) != PA_OK)
+    return st;
+  const size_t dec_bytes = round_up(p.ws_bytes, 256);
+  pa::SharedPrefixLaunch l{};
+  l.q = q;
+  l.k_cache = k_cache;
+  l.v_cache = v_cache;
+  l.block_tables = block_tables;
+  l.context_lens = context_lens;
+  l.group_seqs = group_seqs;
+  l.group_start = group_start;
+  l.group_blocks = group_blocks;
+  l.num_groups = num_groups;
+  l.num_listed = num_listed;
+  l.num_seqs = num_seqs;
+  l.num_q_heads = num_q_heads;
+  l.num_kv_heads = num_kv_heads;
+  l.head_dim = head_dim;
+  l.max_blocks_per_seq = max_blocks_per_seq;
+  l.num_blocks = num_blocks;
+  const long long cap = static_cast<long long>(max_blocks_per_seq) * pa::kBlockSize;
+  l.len_cap = static_cast<int>(max_context_len < cap ? max_context_len : cap);
+  l.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  l.workspace = static_cast<char*>(workspace) + dec_bytes;
+  l.err_flag = err_flag;
+  if (pa::launch_shared_prefix(l, p.sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  return decode_impl(out, q, key, value, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, max_context_len, scale, partition_size, dtype, workspace,
+                     dec_bytes, err_flag, stream, nullptr, -1, 0, &l);
 }
 
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

@@ -288,11 +288,12 @@ constexpr int kLast = 1 << 25;   // last tile of a piece: finish it
 constexpr int kBad = 1 << 26;    // block-table entry out of range
 constexpr int kEnd = 1 << 27;    // no more tiles: the partner warp stops
 constexpr int kAppend = 1 << 28; // fused append: the tile's last live row is the new token
+constexpr int kPrefix = 1 << 29; // first tile of an item that continues a shared-prefix state
 
 __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
                                                const int* s_len, const int* s_row,
-                                               const Ranges& rg, const OwnRanges& own,
-                                               const DecodeArgs& a) {
+                                               const int* s_boff, const Ranges& rg,
+                                               const OwnRanges& own, const DecodeArgs& a) {
   StageDesc d{0, 0, 0, 0};
   if (g >= hi) return d;
   // largest s with s_start[s] <= g (sequences without blocks share their start)
@@ -312,7 +313,10 @@ __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const 
   if (g == item_a || own.is_start(g, rg)) flags |= kFirst;
   if (g + 1 == item_a + nb || own.is_start(g + 1, rg)) flags |= kLast;
   const int trow = s_row ? s_row[s] : s;  // (query rows share their sequence's table)
-  int phys = __ldg(a.block_tables + static_cast<size_t>(trow) * a.max_blocks_per_seq + blk);
+  // (shared-prefix decode: the sequence's first boff blocks were attended already)
+  const int boff = s_boff ? s_boff[s] : 0;
+  if (boff > 0 && g == item_a) flags |= kPrefix;
+  int phys = __ldg(a.block_tables + static_cast<size_t>(trow) * a.max_blocks_per_seq + boff + blk);
   if (phys < 0 || phys >= a.num_blocks) {
     flags |= kBad;
     phys = 0;
@@ -405,6 +409,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   // NR > 1: first query row | (rows << 24) of each group; first group of each sequence
   int* s_r0 = s_qs + a.num_table_rows + 1;                                   // [S]
   int* s_gs = s_r0 + S;                                                      // [rows + 1]
+  // shared-prefix decode: leading blocks of each sequence attended already
+  int* s_boff = (!prefill && a.pre_blocks) ? s_len + S : nullptr;            // [S]
 
   if (leader && lane == 0) {
 #pragma unroll
@@ -424,7 +430,9 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       row = s;
       r0nr = s | (1 << 24);
       const int n = a.context_lens[s];
-      return (n < 0 || n > a.len_cap) ? -kErrContextLen : n;
+      if (n < 0 || n > a.len_cap) return -kErrContextLen;
+      // (a claimed shared prefix always leaves at least one token)
+      return a.pre_blocks ? n - kBlockSize * max(a.pre_blocks[s], 0) : n;
     }
     if constexpr (NR > 1) {
       // s is a group of up to NR consecutive query rows; it attends to the
@@ -504,6 +512,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       if (n < 0) n = 0;
       s_len[s] = n;
       if (prefill) s_row[s] = row;
+      if (s_boff) s_boff[s] = n > 0 ? max(a.pre_blocks[s], 0) : 0;
       if (NR > 1) s_r0[s] = r0nr;
       local += (n + kBlockSize - 1) / kBlockSize;
     }
@@ -602,7 +611,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   int known = n0;                      // positions with a tile assigned
   bool no_more = rg.R == rg.Rs;        // no chunks left to claim
   auto static_desc = [&](int p) -> StageDesc {
-    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, s_row, rg, own, a) : StageDesc{0, 0, 0, 0};
+    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, s_row, s_boff, rg, own, a) : StageDesc{0, 0, 0, 0};
   };
   StageDesc A{0, 0, 0, 0}, B{0, 0, 0, 0};
   int base = 0;
@@ -622,8 +631,8 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     const long long g0 = rg.Ws + static_cast<long long>(c) * rg.CS;
     const int len = static_cast<int>(rg.CS < W - g0 ? rg.CS : W - g0);
     const int pa = base + lane, pb = base + 32 + lane;
-    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, s_row, rg, own, a);
-    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, s_row, rg, own, a);
+    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, s_row, s_boff, rg, own, a);
+    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, s_row, s_boff, rg, own, a);
     known += len;
   };
   auto top_up = [&](int frontier) {
@@ -812,6 +821,24 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
         mh[j][0] = mh[j][1] = -INFINITY;
         lh[j][0] = lh[j][1] = 0.f;
       }
+      if (NR == 1 && (flags & kPrefix)) {
+        // continue from the shared-prefix state: this lane's heads 2t, 2t+1,
+        // head_dim g, g + 8 of each slice; the sums go to one lane per head
+        const size_t hb = static_cast<size_t>(d.seq) * Hq + static_cast<size_t>(kvh) * GT + 2 * mtq;
+        const float2 m0 = a.pre_ml[hb], m1 = a.pre_ml[hb + 1];
+        mh[0][0] = m0.x;
+        mh[0][1] = m1.x;
+        lh[0][0] = mg == 0 ? m0.y : 0.f;
+        lh[0][1] = mg == 0 ? m1.y : 0.f;
+        const float* po = a.pre_o + hb * D + mg;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          oa[0][mt][0] = po[mt * 16];
+          oa[0][mt][1] = po[D + mt * 16];
+          oa[0][mt][2] = po[mt * 16 + 8];
+          oa[0][mt][3] = po[D + mt * 16 + 8];
+        }
+      }
       poisoned = false;
     } else if (flags & kFirst) {
       const unsigned char* pq = pk + 2 * C::TILE;
@@ -829,6 +856,29 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       }
       m_run = -INFINITY;
       l_run = 0.f;
+      if (flags & kPrefix) {
+        // continue from the shared-prefix state.  The final reductions add
+        // o over row groups and l over the lanes that share a head, so both
+        // start in one of them; the running max is per head (per warp at G = 1).
+        const size_t hb = static_cast<size_t>(d.seq) * Hq + static_cast<size_t>(kvh) * GT + hoff;
+        const float2 ml = a.pre_ml[hb + hs];
+        m_run = ml.x;
+        l_run = (G == 1 ? rgp == 0 : lane < G) ? ml.y : 0.f;
+        if (rgp == 0) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float* po = a.pre_o + (hb + h) * D + dl * C::VEC;
+#pragma unroll
+            for (int e = 0; e < C::VEC; e += 4) {
+              const float4 t4 = *reinterpret_cast<const float4*>(po + e);
+              o[h][e] = t4.x;
+              o[h][e + 1] = t4.y;
+              o[h][e + 2] = t4.z;
+              o[h][e + 3] = t4.w;
+            }
+          }
+        }
+      }
       poisoned = false;
     }
 

@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include <cuda.h>  // CUtensorMap (a plain 128-byte descriptor; no driver call here)
+#include <cuda_runtime.h>
 
 namespace pa {
 
@@ -18,6 +19,7 @@ constexpr int kErrSlot = 4;
 constexpr int kErrPair = 8;
 constexpr int kErrTimeout = 16;
 constexpr int kErrQuery = 32;
+constexpr int kErrGroup = 64;
 
 // Work schedule: the last 1/kTailDiv of the tiles is handed out at run time
 // in chunks of kChunkTiles (0 = everything static).
@@ -73,6 +75,14 @@ struct DecodeArgs {
   const int32_t* query_start;
   int num_table_rows;
   int num_query_rows;  // rows of q and out (several query tokens per sequence)
+  // shared-prefix decode (all null otherwise): per sequence the number of
+  // leading blocks the shared-prefix pass attended to (> 0; 0 or less: none),
+  // and that pass's state per (sequence, query head): the unnormalised output
+  // and (running max in log2 units, sum of weights).  The kernel then attends
+  // to the remaining blocks only, starting from that state.
+  const int32_t* pre_blocks;  // [num_seqs]
+  const float* pre_o;         // [num_seqs][num_q_heads][head_dim]
+  const float2* pre_ml;       // [num_seqs][num_q_heads]
   // tensor-core path only: the caches as 2-D tensors [num_blocks * Hkv * 16][head_dim]
   // read in boxes of 16 rows x 128 bytes with the 128-byte swizzle
   CUtensorMap tm_k;
@@ -113,5 +123,39 @@ bool prefill_kernel_bf16(int head_dim, int group, DecodeKernelInfo* info);
 // begins (the merge-pass header and the piece counters).
 size_t decode_zero_prefix_bytes(int num_seqs, int num_kv_heads);
 bool decode_kernel_f32(int head_dim, int group, DecodeKernelInfo* info);
+
+// The shared-prefix pass of deduplicated decode (shared_prefix.cu).
+struct SharedPrefixLaunch {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* group_seqs;    // [num_listed] member sequences, group by group
+  const int32_t* group_start;   // [num_groups + 1] offsets into group_seqs
+  const int32_t* group_blocks;  // [num_groups] leading blocks the members share
+  int num_groups;
+  int num_listed;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int len_cap;
+  float scale_log2;
+  void* workspace;              // shared_prefix_workspace_bytes(...) bytes, zero on first use
+  int32_t* err_flag;
+  // outputs for the decode kernel (inside the workspace)
+  int32_t* pre_blocks;
+  float* pre_o;
+  float2* pre_ml;
+};
+// Bytes of the pass's workspace region; 0 if the shape is unsupported.
+size_t shared_prefix_workspace_bytes(int num_seqs, int num_listed, int num_q_heads,
+                                     int head_dim, int max_blocks_per_seq);
+// Fills pre_blocks / pre_o / pre_ml of `l` from its workspace and launches the
+// pass; returns cudaSuccess or the launch error.
+cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_t stream);
 
 }  // namespace pa

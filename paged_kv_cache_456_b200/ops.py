@@ -9,8 +9,10 @@ from __future__ import annotations
 
 import ctypes
 import os
+from dataclasses import dataclass
 from typing import Optional
 
+import numpy as np
 import torch
 
 # PA_LIBRARY selects another build of the library (e.g. a tuning variant)
@@ -26,11 +28,13 @@ ERRBIT_SLOT = 4
 ERRBIT_PAIR = 8
 ERRBIT_TIMEOUT = 16
 ERRBIT_QUERY = 32
+ERRBIT_GROUP = 64
 
 EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_init",
             "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_decode_append",
             "pa_prefill", "pa_prefill_workspace_size", "pa_prefill_launch_config",
-            "pa_reshape_and_cache", "pa_copy_blocks")
+            "pa_reshape_and_cache", "pa_copy_blocks", "pa_shared_prefix_plan",
+            "pa_shared_prefix_workspace_size", "pa_decode_shared_prefix")
 
 # size of the library's fixed scratch array used by pa_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -80,6 +84,13 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pa_reshape_and_cache.restype = i
     lib.pa_copy_blocks.argtypes = [vp] * 3 + [i] * 6 + [vp, vp]
     lib.pa_copy_blocks.restype = i
+    ip = ctypes.POINTER(i)
+    lib.pa_shared_prefix_plan.argtypes = [vp, vp] + [i] * 4 + [vp, vp, vp, ip, ip]
+    lib.pa_shared_prefix_plan.restype = i
+    lib.pa_shared_prefix_workspace_size.argtypes = [i] * 9 + [ctypes.POINTER(sz)]
+    lib.pa_shared_prefix_workspace_size.restype = i
+    lib.pa_decode_shared_prefix.argtypes = [vp] * 11 + [i] * 10 + [f, i, i, vp, sz, vp, vp]
+    lib.pa_decode_shared_prefix.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -267,3 +278,95 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: tor
     _check(library().pa_copy_blocks(
         _ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), block_mapping.shape[0], Hkv, D, bs, N,
         _dtype_code(k_cache), _ptr(err_flag), _stream(stream)), "pa_copy_blocks")
+
+
+# ---------------------------------------------------------------------------
+# prefix-deduplicated decode
+# ---------------------------------------------------------------------------
+@dataclass
+class SharedPrefixGroups:
+    """Groups of sequences that share their leading blocks (``pa_shared_prefix_plan``):
+    group g's members are ``seqs[start[g]:start[g+1]]`` and share ``blocks[g]`` blocks."""
+    seqs: np.ndarray
+    start: np.ndarray
+    blocks: np.ndarray
+
+    @property
+    def num_groups(self) -> int:
+        return len(self.blocks)
+
+    @property
+    def num_listed(self) -> int:
+        return len(self.seqs)
+
+    def to(self, device="cuda"):
+        """(seqs, start, blocks) as int32 device tensors."""
+        return tuple(torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+                     for a in (self.seqs, self.start, self.blocks))
+
+
+def shared_prefix_plan(block_tables: np.ndarray, context_lens: np.ndarray,
+                       min_shared_blocks: int = 1) -> SharedPrefixGroups:
+    """Find the groups on the host (the library's planner; no device needed)."""
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S = int(cl.shape[0])
+    if bt.ndim != 2 or bt.shape[0] != S:
+        raise ValueError("block_tables must be [num_seqs][max_blocks_per_seq]")
+    seqs = np.zeros(max(S, 1), dtype=np.int32)
+    start = np.zeros(S + 1, dtype=np.int32)
+    blocks = np.zeros(max(S, 1), dtype=np.int32)
+    ng, nl = ctypes.c_int(0), ctypes.c_int(0)
+    vp = ctypes.c_void_p
+    _check(library().pa_shared_prefix_plan(
+        vp(bt.ctypes.data), vp(cl.ctypes.data), S, int(bt.shape[1]), 16, int(min_shared_blocks),
+        vp(seqs.ctypes.data), vp(start.ctypes.data), vp(blocks.ctypes.data), ctypes.byref(ng),
+        ctypes.byref(nl)), "pa_shared_prefix_plan")
+    return SharedPrefixGroups(seqs[:nl.value].copy(), start[:ng.value + 1].copy(),
+                              blocks[:ng.value].copy())
+
+
+def shared_prefix_workspace_size(num_seqs: int, num_listed: int, num_q_heads: int,
+                                 num_kv_heads: int, head_dim: int, max_blocks_per_seq: int,
+                                 max_context_len: int, partition_size: int = 0,
+                                 dtype: torch.dtype = torch.bfloat16) -> int:
+    out = ctypes.c_size_t(0)
+    _check(library().pa_shared_prefix_workspace_size(
+        num_seqs, num_listed, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+        int(max_context_len), int(partition_size),
+        PA_BF16 if dtype == torch.bfloat16 else PA_F32, ctypes.byref(out)),
+        "pa_shared_prefix_workspace_size")
+    return int(out.value)
+
+
+def make_shared_prefix_workspace(num_seqs: int, num_listed: int, num_q_heads: int,
+                                 num_kv_heads: int, head_dim: int, max_blocks_per_seq: int,
+                                 max_context_len: int, partition_size: int = 0,
+                                 dtype: torch.dtype = torch.bfloat16, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size ``pa_decode_shared_prefix`` needs."""
+    n = shared_prefix_workspace_size(num_seqs, num_listed, num_q_heads, num_kv_heads, head_dim,
+                                     max_blocks_per_seq, max_context_len, partition_size, dtype)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def decode_shared_prefix(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                         v_cache: torch.Tensor, block_tables: torch.Tensor,
+                         context_lens: torch.Tensor, groups, *, scale: float,
+                         max_context_len: int, workspace: torch.Tensor,
+                         key: Optional[torch.Tensor] = None, value: Optional[torch.Tensor] = None,
+                         partition_size: int = 0, err_flag: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Decode that reads each group's shared blocks once; ``groups`` is the
+    (seqs, start, blocks) device triple of :meth:`SharedPrefixGroups.to`.  With
+    ``key``/``value`` the newest rows are also written, as in :func:`decode_append`."""
+    seqs, start, blocks = groups
+    S, Hq, D = q.shape
+    N, Hkv, bs, _ = k_cache.shape
+    _check(library().pa_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), _ptr(seqs), _ptr(start), _ptr(blocks),
+        int(blocks.numel()), int(seqs.numel()), S, Hq, Hkv, D, bs, block_tables.shape[1], N,
+        int(max_context_len), float(scale), int(partition_size), _dtype_code(q), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(err_flag), _stream(stream)),
+        "pa_decode_shared_prefix")
+    return out
