@@ -44,7 +44,8 @@ KERNEL_SOURCES = ("paged_kv_cache_456_b200/csrc/decode_kernel.cuh",
                   "paged_kv_cache_456_b200/csrc/decode_bf16.cu",
                   "paged_kv_cache_456_b200/csrc/decode_f32.cu",
                   "paged_kv_cache_456_b200/csrc/ptx.cuh",
-                  "paged_kv_cache_456_b200/csrc/pa_internal.h")
+                  "paged_kv_cache_456_b200/csrc/pa_internal.h",
+                  "paged_kv_cache_456_b200/csrc/shared_prefix.cu")
 
 
 def parse_args(argv=None):
@@ -58,6 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--append", choices=("fused", "separate"), default="fused",
                     help="slot write of the new tokens fused into decode (one call) or as its "
                          "own launch before it")
+    ap.add_argument("--dedup", action="store_true",
+                    help="prefix-deduplicated decode (pa_decode_shared_prefix): groups of "
+                         "sequences sharing leading blocks read them once")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=None)
     ap.add_argument("--num-blocks", type=int, default=None,
@@ -289,9 +293,20 @@ def run_ours(args, rank: int, world: int):
     ps = w.partition_size
     prefill = "query_start" in t     # several query tokens per sequence
     rows = t["q"].shape[0]            # query rows: one per sequence in decode
+    dedup = bool(getattr(args, "dedup", False)) and not prefill
+    plan = None
+    if dedup:
+        # the groups come from the host planner once (they change only when
+        # requests fork or finish); their arrays are step inputs like the tables
+        plan = ops.shared_prefix_plan(w.block_tables, w.context_lens)
+        t["group_seqs"], t["group_start"], t["group_blocks"] = plan.to(dev)
     if prefill:
         ws = ops.make_prefill_workspace(w.num_seqs, rows, w.num_q_heads, w.num_kv_heads,
                                         w.head_dim, w.max_context_len, ps, tdt, device=dev)
+    elif dedup:
+        ws = ops.make_shared_prefix_workspace(w.num_seqs, plan.num_listed, w.num_q_heads,
+                                              w.num_kv_heads, w.head_dim, w.max_blocks_per_seq,
+                                              w.max_context_len, ps, tdt, device=dev)
     else:
         ws = ops.make_workspace(rows, w.num_q_heads, w.num_kv_heads, w.head_dim,
                                 w.max_context_len, ps, tdt, device=dev)
@@ -310,6 +325,8 @@ def run_ours(args, rank: int, world: int):
     fused = "key" in t and args.append == "fused" and not prefill
     # decode is two kernels (the attention pass and the merge pass behind it)
     launches_per_step = 2 + ("key" in t and not fused) + ("block_mapping" in t)
+    if dedup and plan.num_groups:
+        launches_per_step += 1      # the shared-prefix pass
 
     def step(ev_mid=None):
         if "block_mapping" in t:
@@ -324,6 +341,8 @@ def run_ours(args, rank: int, world: int):
                         t["context_lens"], t["query_start"], scale=w.scale,
                         max_context_len=w.max_context_len, workspace=ws, partition_size=ps,
                         err_flag=err)
+        elif dedup:
+            shared_prefix_call(t, t, w, ws, ps, err, fused, stream)
         elif fused:
             ops.decode_append(t["out"], t["q"], t["key_seq"], t["value_seq"], t["k_cache"],
                               t["v_cache"], t["block_tables"], t["context_lens"], scale=w.scale,
@@ -361,7 +380,7 @@ def run_ours(args, rank: int, world: int):
     timed_err = int(err.item())
 
     # end to end through the public API: pinned host inputs in, output back
-    e2e = end_to_end(w, t, ws, ps, dev, stream, K, args.warmup, fused)
+    e2e = end_to_end(w, t, ws, ps, dev, stream, K, args.warmup, fused, dedup)
 
     # every rank reaches this one collective, errors or not; then all agree
     max_ms, e2e["ms"], bad = max_over_ranks([total_ms, e2e["ms"], float(timed_err | e2e["err"])],
@@ -373,9 +392,11 @@ def run_ours(args, rank: int, world: int):
     peak, peak_kind = measured_peaks()
     value = world * nbytes * K / (max_ms * 1e-3) / 1e9
     dec_avg = statistics.mean(dec_ms)
-    dec_bytes = w.decode_bytes() + (w.append_bytes() if fused else 0)
+    # (deduplicated: each shared block counts once -- what the call must move)
+    dec_bytes = ((w.unique_decode_bytes() if dedup else w.decode_bytes()) +
+                 (w.append_bytes() if fused else 0))
     achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
-    traffic = recorded_traffic(w.name)
+    traffic = recorded_traffic(w.name + ("+dedup" if dedup else ""))
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(max_ms / K, 5),
@@ -398,6 +419,14 @@ def run_ours(args, rank: int, world: int):
         "launch": cfg,
         "clocks": clocks.summary(),
     }
+    if dedup:
+        line["config"]["dedup"] = True
+        line["roofline"]["kernel"] = ("shared_prefix_kernel + paged_decode_kernel + merge "
+                                      "(the deduplicated decode call)")
+        line["dedup"] = {"groups": plan.num_groups, "listed": plan.num_listed,
+                         "shared_blocks": [int(b) for b in plan.blocks[:8]],
+                         "logical_kv_bytes": w.decode_bytes(),
+                         "unique_kv_bytes": w.unique_decode_bytes()}
     if prefill:
         # many query rows re-read their sequence's prefix (from L2): the attention
         # kernel is set against the tensor roofline, by its attention FLOPs
@@ -420,7 +449,19 @@ def run_ours(args, rank: int, world: int):
         print(json.dumps(line), flush=True)
 
 
-def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused):
+def shared_prefix_call(d, t, w, ws, ps, err, fused, stream):
+    """The deduplicated decode call: inputs from d (step inputs), cache from t."""
+    from paged_kv_cache_456_b200 import ops
+    ops.decode_shared_prefix(t["out"] if d is t else d["_out"], d["q"], t["k_cache"],
+                             t["v_cache"], d["block_tables"], d["context_lens"],
+                             (d["group_seqs"], d["group_start"], d["group_blocks"]),
+                             scale=w.scale, max_context_len=w.max_context_len, workspace=ws,
+                             key=d["key_seq"] if fused else None,
+                             value=d["value_seq"] if fused else None, partition_size=ps,
+                             err_flag=err, stream=stream)
+
+
+def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused, dedup=False):
     """The step through the public API with the step's inputs in pinned host
     memory: every step copies its inputs (q, the new K/V or slot ids, block
     tables, lengths, copy pairs) host to device in one transfer, runs the
@@ -433,7 +474,8 @@ def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused):
 
     step_inputs = ("q", "key_seq", "value_seq") if fused else ("q", "key", "value", "slot_mapping")
     names = [n for n in step_inputs + ("block_tables", "context_lens", "block_mapping",
-                                       "query_start") if n in t]
+                                       "query_start", "group_seqs", "group_start",
+                                       "group_blocks") if n in t]
     # one pinned staging buffer holding every input, 256-byte aligned pieces
     offs, size = {}, 0
     for n in names:
@@ -478,6 +520,8 @@ def end_to_end(w, t, ws, ps, dev, stream, K, warmup, fused):
                         d["context_lens"], d["query_start"], scale=w.scale,
                         max_context_len=w.max_context_len, workspace=ws, partition_size=ps,
                         err_flag=err, stream=stream)
+        elif dedup:
+            shared_prefix_call(dict(d, _out=out[b]), t, w, ws, ps, err, fused, stream)
         elif fused:
             ops.decode_append(out[b], d["q"], d["key_seq"], d["value_seq"], t["k_cache"],
                               t["v_cache"], d["block_tables"], d["context_lens"], scale=w.scale,

@@ -178,6 +178,21 @@ class Workload:
         qo = 2 * self.q.shape[0] * self.num_q_heads * self.head_dim * eb
         return kv + qo
 
+    def unique_decode_bytes(self) -> int:
+        """decode_bytes with every physical block counted once however many
+        sequences hold it (its live rows: the most any holder uses) -- what a
+        decode that reads each shared block once must move."""
+        eb = self.elem_bytes
+        rows = {}
+        for s in range(self.num_seqs):
+            n = int(self.context_lens[s])
+            for j in range(-(-n // self.block_size)):
+                b = int(self.tables_compact[s, j])
+                rows[b] = max(rows.get(b, 0), min(self.block_size, n - j * self.block_size))
+        kv = sum(rows.values()) * 2 * self.num_kv_heads * self.head_dim * eb
+        qo = 2 * self.q.shape[0] * self.num_q_heads * self.head_dim * eb
+        return kv + qo
+
     def attention_flops(self) -> int:
         """2 FLOP per multiply-add of q.K and of p.V, over every attended token."""
         if self.query_start is None:
@@ -265,6 +280,10 @@ def make_workload(rng: np.random.Generator, *, name: str, dtype: str,
             raise ValueError("prefix_tokens must be a multiple of the block size")
         if (lens < prefix_tokens).any():
             raise ValueError("every sequence must hold the whole prefix")
+        if new_token and (lens <= prefix_tokens).any():
+            # the new token is written into the sequence's own blocks, never
+            # into the shared prefix
+            raise ValueError("with new_token every sequence needs a token after the prefix")
         prefix = alloc.allocate(prefix_tokens)
         for s in range(S):
             t = alloc.fork(prefix)
