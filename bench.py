@@ -44,8 +44,9 @@ KERNEL_SOURCES = ("paged_kv_cache_456_b200/csrc/decode_kernel.cuh",
                   "paged_kv_cache_456_b200/csrc/decode_bf16.cu",
                   "paged_kv_cache_456_b200/csrc/decode_f32.cu",
                   "paged_kv_cache_456_b200/csrc/ptx.cuh",
-                  "paged_kv_cache_456_b200/csrc/pa_internal.h",
-                  "paged_kv_cache_456_b200/csrc/shared_prefix.cu")
+                  "paged_kv_cache_456_b200/csrc/pa_internal.h")
+# the deduplicated call adds the shared-prefix pass
+DEDUP_SOURCES = ("paged_kv_cache_456_b200/csrc/shared_prefix.cu",)
 
 
 def parse_args(argv=None):
@@ -79,12 +80,13 @@ def measured_peaks(key: str = "hbm_gbs"):
         return fallback, "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the decode kernel's code with comments and blank space removed,
-    so that a comment edit does not orphan recorded counters."""
+def kernel_source_hash(dedup: bool = False) -> str:
+    """Hash of the decode kernel's code (with the shared-prefix pass: of both)
+    with comments and blank space removed, so that a comment edit does not
+    orphan recorded counters."""
     import re
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES + (DEDUP_SOURCES if dedup else ()):
         with open(os.path.join(ROOT, rel)) as f:
             code = f.read()
         code = re.sub(r"/\*.*?\*/", " ", code, flags=re.S)
@@ -102,7 +104,7 @@ def recorded_traffic(workload: str):
     except (OSError, ValueError):
         return None
     entry = d.get(workload)
-    if not entry or entry.get("kernel_source_hash") != kernel_source_hash():
+    if not entry or entry.get("kernel_source_hash") != kernel_source_hash(workload.endswith("+dedup")):
         return None
     return entry.get("dram_bytes_per_launch")
 
