@@ -14,8 +14,9 @@
 // sets is the log-sum-exp combination of the parts, so the result is the
 // same attention up to rounding.
 //
-// Work: a unit is (group, chunk of 64 columns, kv head, range of up to
-// kRangeTiles shared blocks).  Each unit writes a partial state per column;
+// Work: a unit is (group, chunk of 64 columns, kv head, range of shared
+// blocks); the host picks the range length so that the units fill the
+// resident CTAs.  Each unit writes a partial state per column;
 // the last unit of a (group, chunk, kv head) to finish folds the ranges and
 // stores the state per (sequence, head).  Members are checked against the
 // block tables before their state is published: a member whose table does
@@ -38,10 +39,27 @@
 namespace pa {
 namespace {
 
-constexpr int kPWarps = 4;
-constexpr int kPCols = 16 * kPWarps;  // (member, head) columns of a unit: 16 per warp
-constexpr int kPStages = 3;           // K/V tiles in flight per CTA
-constexpr int kRangeTiles = 32;       // shared blocks per unit (512 tokens)
+// Shape of a CTA: warps, and 8-column blocks per warp (build-time knobs).
+// 8 warps of 8 columns measured fastest on prefix_cow (121.6 us for the
+// deduplicated call), ahead of 4 x 16 (131.2 us) and 4 x 8 (127.8 us): more
+// warps per SM hide the latency of each warp's dependent MMA / softmax chain.
+#ifndef PA_SP_WARPS
+#define PA_SP_WARPS 8
+#endif
+#ifndef PA_SP_NTW
+#define PA_SP_NTW 1
+#endif
+#ifndef PA_SP_MINB
+#define PA_SP_MINB 2
+#endif
+#ifndef PA_SP_MINRANGE
+#define PA_SP_MINRANGE 16
+#endif
+constexpr int kPWarps = PA_SP_WARPS;
+constexpr int NTW = PA_SP_NTW;                // 8-column blocks of a warp
+constexpr int kPCols = 8 * NTW * kPWarps;     // (member, head) columns of a unit
+constexpr int kPStages = 6;           // ring of K/V tiles: 5 in flight while one is used
+constexpr int kMinRangeTiles = PA_SP_MINRANGE;  // shortest range of shared blocks per unit
 constexpr int kMaxChunkMembers = kPCols + 1;
 
 struct PrefixArgs {
@@ -54,7 +72,7 @@ struct PrefixArgs {
   const int32_t* group_start;
   const int32_t* group_blocks;
   int num_groups, num_listed, num_seqs, num_q_heads, num_kv_heads;
-  int max_blocks_per_seq, num_blocks, len_cap, max_ranges;
+  int max_blocks_per_seq, num_blocks, len_cap, max_ranges, range_tiles;
   float scale_log2;
   int* counters;     // [num_listed * Hq] units finished per (chunk, kv head); zero between calls
   int* claim;        // [num_seqs] = pre_blocks; zeroed before the pass
@@ -104,7 +122,7 @@ __device__ __forceinline__ bool group_ok(const PrefixArgs& a, int g, int* gs, in
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kPWarps * 32)
+__global__ void __launch_bounds__(kPWarps * 32, PA_SP_MINB)
 shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
   constexpr int ROW = D * 2;              // bytes of one K or V row (bf16)
   constexpr int TILE = kBlockSize * ROW;  // one block of one kv head
@@ -116,9 +134,12 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
   __shared__ int s_wsum[kPWarps];
   __shared__ int s_last;
   __shared__ unsigned char s_ok[kMaxChunkMembers];
+  __shared__ int s_seq[kMaxChunkMembers];
+  __shared__ float s_M[kPCols], s_L[kPCols];
   // tiles 128-byte aligned for the swizzle; the unit prefix sums behind them
   unsigned char* ring = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   int* s_ubase = reinterpret_cast<int*>(ring + kPStages * 2 * TILE);  // [num_groups + 1]
+  int* s_phys = s_ubase + a.num_groups + 1;                            // [range_tiles]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mg = lane >> 2, mtq = lane & 3;  // mma fragment row group / thread in group
@@ -135,7 +156,7 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
       int gs, m, P, leader;
       int units = 0;
       if (group_ok(a, g, &gs, &m, &P, &leader)) {
-        units = ((m * G + kPCols - 1) / kPCols) * Hkv * ((P + kRangeTiles - 1) / kRangeTiles);
+        units = ((m * G + kPCols - 1) / kPCols) * Hkv * ((P + a.range_tiles - 1) / a.range_tiles);
       } else if (blockIdx.x == 0 && a.err_flag) {
         atomicOr(a.err_flag, kErrGroup);
       }
@@ -177,22 +198,22 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
     int gs = 0, m = 0, P = 0, leader = 0;
     group_ok(a, g, &gs, &m, &P, &leader);  // (true: only such groups have units)
     const int NC = (m * G + kPCols - 1) / kPCols;
-    const int R = (P + kRangeTiles - 1) / kRangeTiles;
+    const int R = (P + a.range_tiles - 1) / a.range_tiles;
     int local = u - s_ubase[g];
     const int c = local % NC;  // (consecutive units share the same K/V tiles)
     local /= NC;
     const int kvh = local % Hkv;
     const int r = local / Hkv;
-    const int t0 = r * kRangeTiles, t1 = min(P, t0 + kRangeTiles);
+    const int t0 = r * a.range_tiles, t1 = min(P, t0 + a.range_tiles);
     const int32_t* trow = a.block_tables + static_cast<size_t>(leader) * a.max_blocks_per_seq;
 
-    // ---- q of this warp's 16 columns as the B operand of S^T = K q^T: lane
+    // ---- q of this warp's 8 * NTW columns as the B operand of S^T = K q^T: lane
     // (g, t) holds column g of each 8-column half, head_dim pairs 2t, 2t+1
     // and 2t+8, 2t+9 of every 16-wide slice.  Columns past the group: zero.
-    uint32_t qb[2][MT][2];
+    uint32_t qb[NTW][MT][2];
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      const int col = c * kPCols + warp * 16 + n * 8 + mg;
+    for (int n = 0; n < NTW; ++n) {
+      const int col = c * kPCols + warp * 8 * NTW + n * 8 + mg;
       const int member = col / G;
       int seq = member < m ? a.group_seqs[gs + member] : -1;
       const bool ok = seq >= 0 && seq < a.num_seqs;
@@ -206,21 +227,27 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
     }
     // o^T[head_dim x columns] as C fragments (head_dim g, g + 8 of each slice;
     // columns 2t, 2t+1); running max and this lane's share of the sums
-    float oa[2][MT][4];
-    float mh[2][2], lh[2][2];
+    float oa[NTW][MT][4];
+    float mh[NTW][2], lh[NTW][2];
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
+    for (int n = 0; n < NTW; ++n) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) oa[n][mt][0] = oa[n][mt][1] = oa[n][mt][2] = oa[n][mt][3] = 0.f;
       mh[n][0] = mh[n][1] = -INFINITY;
       lh[n][0] = lh[n][1] = 0.f;
     }
 
+    // the range's block ids, once (-1: out of range)
+    for (int i = tid; i < t1 - t0; i += NTHR) {
+      const int b = __ldg(trow + t0 + i);
+      s_phys[i] = b >= 0 && b < a.num_blocks ? b : -1;
+    }
+    __syncthreads();
     // all 128 threads stage tile t (K then V, swizzled); a bad id reads nothing
     auto load = [&](int t) {
       const uint32_t dst = smem_addr(ring) + ((t - t0) % kPStages) * 2 * TILE;
-      int phys = __ldg(trow + t);
-      const bool ok = phys >= 0 && phys < a.num_blocks;
+      int phys = s_phys[t - t0];
+      const bool ok = phys >= 0;
       if (!ok) phys = 0;
       const size_t off = (static_cast<size_t>(phys) * Hkv + kvh) * TILE;
 #pragma unroll
@@ -231,30 +258,42 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
         cp_async16(dst + which * TILE + swz(row, ch), src, ok);
       }
     };
-    load(t0);
-    cp_async_commit();
-    if (t0 + 1 < t1) load(t0 + 1);
-    cp_async_commit();
-    for (int t = t0; t < t1; ++t) {
-      if (t + 2 < t1) load(t + 2);
+#pragma unroll
+    for (int i = 0; i < kPStages - 1; ++i) {
+      if (t0 + i < t1) load(t0 + i);
       cp_async_commit();
-      cp_async_wait<2>();  // this thread's copies of tile t are done
-      __syncthreads();     // ... and everyone's
+    }
+    for (int t = t0; t < t1; ++t) {
+      cp_async_wait<kPStages - 2>();  // this thread's copies of tile t are done
+      __syncthreads();                // ... and everyone's; every warp is past tile t - 1
+      // refill the stage of tile t - 1 with tile t + kPStages - 1
+      if (t + kPStages - 1 < t1) load(t + kPStages - 1);
+      cp_async_commit();
       const uint32_t kb = smem_addr(ring) + ((t - t0) % kPStages) * 2 * TILE, vb = kb + TILE;
-      // S^T[16 tokens x 16 columns] = K q^T
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // S^T[16 tokens x 16 columns] = K q^T (even and odd head_dim slices in
+      // separate accumulators: four dependent chains of MT / 2)
+      float sc[NTW][4], sd[NTW][4];
+#pragma unroll
+      for (int n = 0; n < NTW; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[n][e] = sd[n][e] = 0.f;
 #pragma unroll
       for (int ks = 0; ks < MT; ++ks) {
         uint32_t af[4];  // tokens 0-7 / 8-15 x head_dim ks*16 + 0-7, then + 8-15
         ldmatrix_x4(kb + swz((lm & 1) * 8 + lr, ks * 2 + (lm >> 1)), af);
-        mma_bf16_16816(sc[0], af, qb[0][ks][0], qb[0][ks][1]);
-        mma_bf16_16816(sc[1], af, qb[1][ks][0], qb[1][ks][1]);
+#pragma unroll
+        for (int n = 0; n < NTW; ++n)
+          mma_bf16_16816(ks & 1 ? sd[n] : sc[n], af, qb[n][ks][0], qb[n][ks][1]);
       }
+#pragma unroll
+      for (int n = 0; n < NTW; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[n][e] += sd[n][e];
       // online softmax per column on the fragments: sc[n] holds tokens g and
       // g + 8 of columns 2t, 2t+1
-      uint32_t b0[2], b1[2];
+      uint32_t b0[NTW], b1[NTW];
 #pragma unroll
-      for (int n = 0; n < 2; ++n) {
+      for (int n = 0; n < NTW; ++n) {
         float x[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) x[e] = sc[n][e] * a.scale_log2;
@@ -293,15 +332,14 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
       for (int mt = 0; mt < MT; ++mt) {
         uint32_t af[4];  // (transposed on load) tokens 0-7 x head_dim mt*16 + 0-7 / + 8-15, then tokens 8-15
         ldmatrix_x4_trans(vb + swz((lm >> 1) * 8 + lr, mt * 2 + (lm & 1)), af);
-        mma_bf16_16816(oa[0][mt], af, b0[0], b1[0]);
-        mma_bf16_16816(oa[1][mt], af, b0[1], b1[1]);
+#pragma unroll
+        for (int n = 0; n < NTW; ++n) mma_bf16_16816(oa[n][mt], af, b0[n], b1[n]);
       }
-      __syncthreads();  // the stage is refilled two tiles later
     }
 
     // ---- the range's partial state per column ------------------------------
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
+    for (int n = 0; n < NTW; ++n) {
       float lt[2] = {lh[n][0], lh[n][1]};
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -310,7 +348,7 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
       }
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const int col = c * kPCols + warp * 16 + n * 8 + 2 * mtq + cc;
+        const int col = c * kPCols + warp * 8 * NTW + n * 8 + 2 * mtq + cc;
         const int member = col / G;
         if (member >= m) continue;
         const size_t pi =
@@ -337,74 +375,128 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
     __threadfence();
 
     // ---- last range of (group, chunk, kv head): check the members, fold ----
+    // (spread over all threads: each step's loads are independent, so they
+    // overlap instead of paying the L2 latency one after the other)
     const int mlo = (c * kPCols) / G;
-    const int mhi = (min(m * G, (c + 1) * kPCols) - 1) / G;  // inclusive
-    for (int i = warp; i <= mhi - mlo; i += kPWarps) {
+    const int nm = (min(m * G, (c + 1) * kPCols) - 1) / G - mlo + 1;  // members in the chunk
+    for (int i = tid; i < nm; i += NTHR) {
       const int seq = a.group_seqs[gs + mlo + i];
       bool ok = seq >= 0 && seq < a.num_seqs;
       if (ok) {
         const int n = a.context_lens[seq];
         ok = n > 0 && n <= a.len_cap && kBlockSize * P <= n - 1;
       }
-      bool same = true;
-      if (ok) {
-        const int32_t* srow = a.block_tables + static_cast<size_t>(seq) * a.max_blocks_per_seq;
-        for (int j = lane; j < P; j += 32) {
-          const int b = __ldg(trow + j);
-          same &= b >= 0 && b < a.num_blocks && __ldg(srow + j) == b;
-        }
-      }
-      ok = __all_sync(0xffffffffu, ok && same);
-      if (lane == 0) {
-        s_ok[i] = ok;
-        if (!ok && kvh == 0 && a.err_flag) atomicOr(a.err_flag, kErrGroup);
-      }
+      s_seq[i] = ok ? seq : -1;
+      s_ok[i] = ok;
     }
     __syncthreads();
-    for (int cl = warp; cl < kPCols; cl += kPWarps) {
+    // every (member, shared block): the member's table holds the leader's block
+#pragma unroll 4
+    for (int idx = tid; idx < nm * P; idx += NTHR) {
+      const int i = idx / P, j = idx - i * P;
+      const int seq = s_seq[i];
+      if (seq < 0) continue;
+      const int b = __ldg(trow + j);
+      if (!(b >= 0 && b < a.num_blocks &&
+            __ldg(a.block_tables + static_cast<size_t>(seq) * a.max_blocks_per_seq + j) == b))
+        s_ok[i] = 0;  // (every writer stores the same value)
+    }
+    __syncthreads();
+    if (kvh == 0 && a.err_flag)
+      for (int i = tid; i < nm; i += NTHR)
+        if (!s_ok[i]) atomicOr(a.err_flag, kErrGroup);
+    // column weights of the ranges, w = 2^(m_r - M), into the idle ring
+    float* s_w = reinterpret_cast<float*>(ring);  // [kPCols][R]
+    for (int cl = tid; cl < kPCols; cl += NTHR) {
       const int col = c * kPCols + cl;
       const int member = col / G;
       if (member >= m || !s_ok[member - mlo]) continue;
-      const int seq = a.group_seqs[gs + member];
-      const int head = kvh * G + col % G;
-      const size_t pb = (static_cast<size_t>(gs + member) * Hq + head) * a.max_ranges;
+      const size_t pb = (static_cast<size_t>(gs + member) * Hq + kvh * G + col % G) * a.max_ranges;
       float M = -INFINITY;
+#pragma unroll 4
       for (int rr = 0; rr < R; ++rr) M = fmaxf(M, __ldcg(a.part_ml + pb + rr).x);
       float L = 0.f;
-      float acc[D / 32];
-#pragma unroll
-      for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+#pragma unroll 4
       for (int rr = 0; rr < R; ++rr) {
         const float2 ml = __ldcg(a.part_ml + pb + rr);
         const float w = exp2f(ml.x - M);
+        s_w[cl * R + rr] = w;
         L += w * ml.y;
-        const float* po = a.part_o + (pb + rr) * D + lane;
-#pragma unroll
-        for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(w, __ldcg(po + 32 * e), acc[e]);
       }
-      float* dst = a.pre_o + (static_cast<size_t>(seq) * Hq + head) * D + lane;
+      s_M[cl] = M;
+      s_L[cl] = L;
+    }
+    __syncthreads();
+    // outputs: thread t owns (column, 4 head_dim) items t, t + 128, ...; in
+    // batches of KB items, one pass over the ranges with the batch's loads
+    // in flight together
+    constexpr int Q4 = D / 4;
+    constexpr int NI = kPCols * Q4 / NTHR;
+    static_assert(kPCols * Q4 % NTHR == 0, "fold items must split evenly over the threads");
+    constexpr int KB = NI < 8 ? NI : 8;
+    for (int k0 = 0; k0 < NI; k0 += KB) {
+      const float4* src[KB];
+      float4 acc[KB];
 #pragma unroll
-      for (int e = 0; e < D / 32; ++e) dst[32 * e] = acc[e];
-      if (lane == 0) a.pre_ml[static_cast<size_t>(seq) * Hq + head] = make_float2(M, L);
+      for (int k = 0; k < KB; ++k) {
+        const int idx = tid + (k0 + k) * NTHR, cl = idx / Q4, q4 = idx % Q4;
+        const int col = c * kPCols + cl;
+        const int member = col / G;
+        const bool live = member < m && s_ok[member - mlo];
+        const size_t pb =
+            (static_cast<size_t>(gs + (live ? member : 0)) * Hq + kvh * G + col % G) * a.max_ranges;
+        src[k] = live ? reinterpret_cast<const float4*>(a.part_o + pb * D) + q4 : nullptr;
+        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int rr = 0; rr < R; ++rr) {
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+          if (!src[k]) continue;
+          const int cl = (tid + (k0 + k) * NTHR) / Q4;
+          const float4 o = __ldcg(src[k] + static_cast<size_t>(rr) * Q4);
+          const float w = s_w[cl * R + rr];
+          acc[k].x = fmaf(w, o.x, acc[k].x);
+          acc[k].y = fmaf(w, o.y, acc[k].y);
+          acc[k].z = fmaf(w, o.z, acc[k].z);
+          acc[k].w = fmaf(w, o.w, acc[k].w);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        if (!src[k]) continue;
+        const int idx = tid + (k0 + k) * NTHR, cl = idx / Q4, q4 = idx % Q4;
+        const int col = c * kPCols + cl;
+        const int member = col / G;
+        const size_t row = static_cast<size_t>(s_seq[member - mlo]) * Hq + kvh * G + col % G;
+        reinterpret_cast<float4*>(a.pre_o + row * D)[q4] = acc[k];
+        if (q4 == 0) a.pre_ml[row] = make_float2(s_M[cl], s_L[cl]);
+      }
     }
     // claim each checked member once (the chunk of its first column, kv head
     // 0); a sequence claimed twice is given up
     if (kvh == 0) {
-      for (int i = tid; i <= mhi - mlo; i += NTHR) {
+      for (int i = tid; i < nm; i += NTHR) {
         const int member = mlo + i;
         if (member * G < c * kPCols || !s_ok[i]) continue;
-        const int seq = a.group_seqs[gs + member];
+        const int seq = s_seq[i];
         if (atomicCAS(a.claim + seq, 0, P) != 0) {
           atomicExch(a.claim + seq, -1);
           if (a.err_flag) atomicOr(a.err_flag, kErrGroup);
         }
       }
     }
-    __syncthreads();  // (s_ok is rewritten by the next unit)
+    __syncthreads();  // (s_ok, s_seq and the ring are rewritten by the next unit)
   }
 }
 
 size_t round_up(size_t x, size_t al) { return (x + al - 1) / al * al; }
+
+// Shortest range a launch may use: kMinRangeTiles, and long enough that the
+// fold's weights (kPCols x ranges floats) fit the ring they reuse.
+int min_range_tiles(int max_blocks_per_seq, int head_dim) {
+  const int cap = kPStages * 2 * kBlockSize * head_dim * 2 / (4 * kPCols);  // ranges that fit
+  return std::max(kMinRangeTiles, (max_blocks_per_seq + cap - 1) / cap);
+}
 
 struct Layout {
   size_t counters, claim, part_ml, part_o, pre_ml, pre_o, bytes;
@@ -414,7 +506,8 @@ struct Layout {
 Layout layout(int num_seqs, int num_listed, int num_q_heads, int head_dim,
               int max_blocks_per_seq) {
   Layout l{};
-  l.max_ranges = (max_blocks_per_seq + kRangeTiles - 1) / kRangeTiles;
+  const int rt = min_range_tiles(max_blocks_per_seq, head_dim);
+  l.max_ranges = (max_blocks_per_seq + rt - 1) / rt;
   const size_t cols = static_cast<size_t>(num_listed) * num_q_heads;
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads;
   l.counters = 0;
@@ -494,6 +587,7 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
   a.num_blocks = l.num_blocks;
   a.len_cap = l.len_cap;
   a.max_ranges = lo.max_ranges;
+  a.range_tiles = 0;  // (set below, once the resident CTAs are known)
   a.scale_log2 = l.scale_log2;
   a.counters = reinterpret_cast<int*>(ws + lo.counters);
   a.claim = l.pre_blocks;
@@ -504,7 +598,9 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
   a.err_flag = l.err_flag;
 
   const size_t tile = static_cast<size_t>(kBlockSize) * l.head_dim * 2;
-  const size_t smem = 128 + kPStages * 2 * tile + (static_cast<size_t>(l.num_groups) + 1) * sizeof(int);
+  // (the range's block ids follow the unit starts; sized for the longest range below)
+  const size_t smem = 128 + kPStages * 2 * tile +
+                      (static_cast<size_t>(l.num_groups) + 1 + l.max_blocks_per_seq) * sizeof(int);
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   int occ = 0;
@@ -529,11 +625,20 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
     }
   }
   if (occ < 1) return cudaErrorInvalidConfiguration;
+  // ranges per (chunk, kv head) so that the units about fill the resident
+  // CTAs (from the fewest chunks the columns can form), but no shorter than
+  // min_range_tiles
+  const long long resident = static_cast<long long>(num_sms) * occ;
+  const long long min_chunks =
+      std::max(1LL, (static_cast<long long>(l.num_listed) * group + kPCols - 1) / kPCols);
+  const long long per = std::max(1LL, resident / (min_chunks * l.num_kv_heads));
+  a.range_tiles = static_cast<int>(std::max<long long>(
+      min_range_tiles(l.max_blocks_per_seq, l.head_dim), (l.max_blocks_per_seq + per - 1) / per));
   // units: at most (chunks of all groups) x kv heads x ranges
   const long long chunks = (static_cast<long long>(l.num_listed) * group + kPCols - 1) / kPCols +
                            l.num_groups;
-  const long long bound = chunks * l.num_kv_heads * lo.max_ranges;
-  const long long resident = static_cast<long long>(num_sms) * occ;
+  const long long bound = chunks * l.num_kv_heads *
+                          ((l.max_blocks_per_seq + a.range_tiles - 1) / a.range_tiles);
   const int grid = static_cast<int>(std::max(1LL, std::min(bound, resident)));
   void* params[] = {&a};
   return cudaLaunchKernel(fn, dim3(grid), dim3(kPWarps * 32), params, smem, stream);
