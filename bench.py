@@ -246,6 +246,9 @@ def run_reference(args, rank: int, world: int):
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+    if getattr(args, "dedup", False):
+        # (the same attention: the oracle reads every sequence's blocks itself)
+        line["config"]["dedup"] = True
     print(json.dumps(line), flush=True)
 
 
