@@ -208,7 +208,7 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
     const int32_t* trow = a.block_tables + static_cast<size_t>(leader) * a.max_blocks_per_seq;
 
     // ---- q of this warp's 8 * NTW columns as the B operand of S^T = K q^T: lane
-    // (g, t) holds column g of each 8-column half, head_dim pairs 2t, 2t+1
+    // (g, t) holds column g of each 8-column block, head_dim pairs 2t, 2t+1
     // and 2t+8, 2t+9 of every 16-wide slice.  Columns past the group: zero.
     uint32_t qb[NTW][MT][2];
 #pragma unroll
@@ -243,7 +243,7 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
       s_phys[i] = b >= 0 && b < a.num_blocks ? b : -1;
     }
     __syncthreads();
-    // all 128 threads stage tile t (K then V, swizzled); a bad id reads nothing
+    // all threads of the CTA stage tile t (K then V, swizzled); a bad id reads nothing
     auto load = [&](int t) {
       const uint32_t dst = smem_addr(ring) + ((t - t0) % kPStages) * 2 * TILE;
       int phys = s_phys[t - t0];
@@ -270,8 +270,8 @@ shared_prefix_kernel(const __grid_constant__ PrefixArgs a) {
       if (t + kPStages - 1 < t1) load(t + kPStages - 1);
       cp_async_commit();
       const uint32_t kb = smem_addr(ring) + ((t - t0) % kPStages) * 2 * TILE, vb = kb + TILE;
-      // S^T[16 tokens x 16 columns] = K q^T (even and odd head_dim slices in
-      // separate accumulators: four dependent chains of MT / 2)
+      // S^T[16 tokens x 8 * NTW columns] = K q^T (even and odd head_dim slices
+      // in separate accumulators: dependent chains of MT / 2)
       float sc[NTW][4], sd[NTW][4];
 #pragma unroll
       for (int n = 0; n < NTW; ++n)
