@@ -36,3 +36,14 @@ def test_new_rows_per_sequence_layout():
     live = np.nonzero(w.context_lens > 0)[0]
     assert np.array_equal(k[live].view(np.uint8), w.new_key.view(np.uint8))
     assert np.array_equal(v[live].view(np.uint8), w.new_value.view(np.uint8))
+
+
+def test_dedup_flag_and_its_counters(capsys):
+    # the reference arm names a deduplicated run in its config (same attention)
+    bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "1",
+                "--dedup"])
+    d = json.loads([ln for ln in capsys.readouterr().out.splitlines() if ln.strip()][0])
+    assert d["config"]["dedup"] is True
+    # recorded DRAM counters are keyed per path; a deduplicated run's hash
+    # also covers the shared-prefix pass
+    assert bench.kernel_source_hash(True) != bench.kernel_source_hash()

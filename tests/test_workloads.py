@@ -97,3 +97,18 @@ def test_prefill_workload_structure():
             assert np.isnan(bf16_bits_to_f32(w.k_pool[int(w.tables_compact[s, b]), :, off])).all()
     assert w.attention_flops() == 4 * w.num_q_heads * w.head_dim * sum(
         128 * (int(n) - 128) + 128 * 129 // 2 for n in w.context_lens)
+
+
+def test_unique_bytes_count_each_shared_block_once():
+    # no sharing: every block has one holder
+    for name in ("tiny", "7b"):
+        w = build_workload(name)
+        assert w.unique_decode_bytes() == w.decode_bytes()
+    # prefix_cow: 128 sequences hold the 128 prompt blocks; 64 of them hold
+    # a private copy of the last one instead.  Every other holder of a
+    # shared block adds 16 rows to the logical count only.
+    w = build_workload("prefix_cow")
+    row = 2 * w.num_kv_heads * w.head_dim * w.elem_bytes      # K and V of one token
+    S, shared, cow = 128, 128, 64
+    extra_rows = 16 * ((shared - 1) * (S - 1) + (S - cow - 1))
+    assert w.decode_bytes() - w.unique_decode_bytes() == extra_rows * row
