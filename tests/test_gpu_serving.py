@@ -3,7 +3,8 @@
 Every step applies the simulator's plan on the GPU -- copy-on-write copies
 (pa_copy_blocks), the prompt writes of newly admitted requests
 (pa_reshape_and_cache), then the fused slot write + decode of the batch
-(pa_decode_append) -- and the same plan on a CPU mirror of the pool with the
+(pa_decode_append, or pa_decode_shared_prefix with the groups the host
+planner finds among the requests sharing the system prompt) -- and the same plan on a CPU mirror of the pool with the
 oracle.  Each step's attention output is compared with the oracle's; at the
 end the two pools must be identical byte for byte.  Blocks are reused after
 requests finish or are preempted, so stale rows of earlier owners sit next
@@ -57,8 +58,10 @@ def to_dev(a, dtype):
     return (t.view(torch.bfloat16) if dtype == "bf16" else t).cuda()
 
 
-@pytest.mark.parametrize("dtype,G,D", [("f32", 2, 64), ("bf16", 8, 128), ("bf16", 1, 128)])
-def test_simulated_serving_steps(dtype, G, D):
+@pytest.mark.parametrize("dtype,G,D,dedup", [("f32", 2, 64, False), ("bf16", 8, 128, False),
+                                             ("bf16", 1, 128, False), ("bf16", 8, 128, True),
+                                             ("bf16", 4, 128, True)])
+def test_simulated_serving_steps(dtype, G, D, dedup):
     hkv, max_tokens, num_blocks = 2, 1024, 220
     rng = np.random.default_rng(11)
     arr = poisson_arrivals(rng, 40, 1.0, prompt_mean=150, output_mean=40, max_tokens=max_tokens,
@@ -83,7 +86,7 @@ def test_simulated_serving_steps(dtype, G, D):
                               torch.tensor(slots, dtype=torch.int64, device="cuda"), err_flag=err)
 
     write(-1, range(sim.prefix_len), sim.prefix_slots())
-    steps = preempted_seen = 0
+    steps = preempted_seen = grouped_steps = 0
     while (plan := sim.step()) is not None:
         steps += 1
         if plan.copies:
@@ -107,16 +110,29 @@ def test_simulated_serving_steps(dtype, G, D):
         assert e == 0
         out = torch.empty((B, hkv * G, D), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32,
                           device="cuda")
-        ws = ops.make_workspace(B, hkv * G, hkv, D, max_tokens, 0, out.dtype)
-        ops.decode_append(out, to_dev(q, dtype), to_dev(key, dtype), to_dev(value, dtype), k_dev,
-                          v_dev, torch.from_numpy(plan.block_tables).cuda(),
-                          torch.from_numpy(plan.context_lens).cuda(), scale=scale,
-                          max_context_len=max_tokens, workspace=ws, err_flag=err)
+        tables = torch.from_numpy(plan.block_tables).cuda()
+        lens = torch.from_numpy(plan.context_lens).cuda()
+        if dedup:
+            # the batch's sharers (the system prompt), found by the host planner
+            groups = ops.shared_prefix_plan(plan.block_tables, plan.context_lens)
+            ws = ops.make_shared_prefix_workspace(B, groups.num_listed, hkv * G, hkv, D,
+                                                  plan.block_tables.shape[1], max_tokens)
+            ops.decode_shared_prefix(out, to_dev(q, dtype), k_dev, v_dev, tables, lens,
+                                     groups.to(), scale=scale, max_context_len=max_tokens,
+                                     workspace=ws, key=to_dev(key, dtype),
+                                     value=to_dev(value, dtype), err_flag=err)
+            grouped_steps += groups.num_groups > 0
+        else:
+            ws = ops.make_workspace(B, hkv * G, hkv, D, max_tokens, 0, out.dtype)
+            ops.decode_append(out, to_dev(q, dtype), to_dev(key, dtype), to_dev(value, dtype),
+                              k_dev, v_dev, tables, lens, scale=scale,
+                              max_context_len=max_tokens, workspace=ws, err_flag=err)
         torch.cuda.synchronize()
         assert err.item() == 0, f"step {plan.step}: error bits {err.item()}"
         assert_attention_close(out, ref, dtype, f"step {plan.step}")
         preempted_seen = max(preempted_seen, sim.stats.preemptions)
     assert sim.stats.finished == 40 and preempted_seen > 0
+    assert grouped_steps > 0 or not dedup
     iv = torch.int16 if dtype == "bf16" else torch.int32
     for dev, host in ((k_dev, k_host), (v_dev, v_host)):
         got = dev.view(iv).cpu().numpy()
