@@ -12,29 +12,38 @@
 //    block) order and cut into equal contiguous ranges, one or more per
 //    worker of a persistent grid (as many CTAs as fit on the 148 SMs): every
 //    worker gets the same number of tiles however skewed the lengths are.
-//    A worker is one warp, or HS = 2 warps that split the G query heads of
-//    a tile between them when G = 8.
+//    A worker is one warp, or on the CUDA-core path with G = 8, HS = 2 warps
+//    that split the query heads of a tile between them.
 //  * Each worker streams its tiles through a ring of DEPTH shared-memory
-//    slots filled by its leader warp with the 1-D bulk-copy engine
-//    (cp.async.bulk, a "full" mbarrier per slot completed by byte count, an
-//    "empty" mbarrier per slot when two warps share it).  Only the live rows
-//    of a partial last block are fetched.  Block-table entries for the next
-//    32-64 tiles are loaded one per lane well ahead of use, and each slot's
-//    descriptor travels with it through shared memory.
+//    slots filled by its leader warp: 1-D bulk copies (cp.async.bulk) of the
+//    live rows on the CUDA-core path, 2-D tensor loads of whole 16-row tiles
+//    with the 128-byte swizzle on the tensor-core path; a "full" mbarrier per
+//    slot completes by byte count, an "empty" one per slot when two warps
+//    share it.  Block-table entries for the next 32-64 tiles are loaded one
+//    per lane well ahead of use, and each slot's descriptor travels with it
+//    through shared memory.
 //  * Fused slot write (when key/value are given): the newest row of each
 //    (sequence, KV head) is fetched from key/value instead of the cache, and
 //    the leader writes it from shared memory to its cache slot.
-//  * Arithmetic is fp32 on the CUDA cores (a one-token query is a
-//    bandwidth-bound gather, not a dense contraction): lanes split head_dim
-//    16 bytes at a time, partial dot products are combined by a butterfly
+//  * Arithmetic: fp32 on the CUDA cores for G <= 4 and for fp32 caches (a
+//    one-token query is a bandwidth-bound gather): lanes split head_dim 16
+//    bytes at a time, partial dot products are combined by a butterfly
 //    reduce-scatter of warp shuffles, the softmax is online (base 2, rescaled
 //    only when the running max grows by more than 2^8), and P.V accumulates
-//    in registers.
+//    in registers.  bf16 with G = 8 runs on the tensor cores (mma.sync,
+//    fp32 accumulation): 16 tokens x 8 heads per tile is exactly one MMA
+//    shape, and the CUDA cores alone would be bound by issue there.
 //  * A (seq, kv head) cut by a range boundary leaves partial results (m, l,
-//    o) in the workspace.  With few pieces, the warp that finishes the last
-//    piece merges them by log-sum-exp (a counter per item, no waiting, so
-//    nothing can hang); items with many pieces go to a list that a second,
-//    programmatically dependent kernel merges with all its threads.
+//    o) in the workspace; its first piece lists the item, and a second,
+//    programmatically dependent kernel merges the pieces by log-sum-exp.
+//    (The CUDA-core path can instead merge few-piece items in the warp that
+//    finishes the last piece, behind PA_FUSE_MAX_VALUES; off by default.)
+//  * Several query tokens per sequence (prefill): items are query rows, or
+//    on the tensor-core path pairs of rows (NR = 2), each over its own
+//    causal prefix, found on chip from query_start.
+//  * Shared-prefix continuation (pre_blocks): a sequence's first blocks were
+//    attended by the shared-prefix pass; the kernel walks the rest and
+//    starts the item from that pass's state.
 //  * Device-side index checks skip bad items and set err_flag bits; every
 //    wait is bounded.
 #pragma once
