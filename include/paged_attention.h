@@ -328,6 +328,20 @@ pa_status pa_shared_prefix_plan(const int32_t *block_tables, const int32_t *cont
                                 int32_t *group_start, int32_t *group_blocks, int *num_groups,
                                 int *num_listed);
 
+/* The same output for sharing that forms a tree (forks of forks): the groups
+ * are chosen on the trie of the sequences' block paths (each path: the
+ * table up to the block before the one holding the last token).  Bottom-up,
+ * the k sequences left ungrouped below a trie node of depth d are grouped
+ * there, sharing d blocks, when (k - 1) * d >= k * d_parent; otherwise they
+ * go up to the parent node.  It never saves fewer block reads than
+ * pa_shared_prefix_plan and saves more when a sub-group shares a longer run
+ * than its whole family.  Host pointers, as pa_shared_prefix_plan. */
+pa_status pa_shared_prefix_plan_tree(const int32_t *block_tables, const int32_t *context_lens,
+                                     int num_seqs, int max_blocks_per_seq, int block_size,
+                                     int min_shared_blocks, int32_t *group_seqs,
+                                     int32_t *group_start, int32_t *group_blocks,
+                                     int *num_groups, int *num_listed);
+
 pa_status pa_shared_prefix_workspace_size(int num_seqs, int num_listed, int num_q_heads,
                                           int num_kv_heads, int head_dim,
                                           int max_blocks_per_seq, int max_context_len,

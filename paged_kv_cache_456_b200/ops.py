@@ -34,6 +34,7 @@ EXPORTED = ("pa_status_str", "pa_decode_workspace_size", "pa_decode_workspace_in
             "pa_decode_launch_config", "pa_decode", "pa_decode_noalloc", "pa_decode_append",
             "pa_prefill", "pa_prefill_workspace_size", "pa_prefill_launch_config",
             "pa_reshape_and_cache", "pa_copy_blocks", "pa_shared_prefix_plan",
+            "pa_shared_prefix_plan_tree",
             "pa_shared_prefix_workspace_size", "pa_decode_shared_prefix")
 
 # size of the library's fixed scratch array used by pa_decode_noalloc
@@ -87,6 +88,8 @@ def library(path: Optional[str] = None) -> ctypes.CDLL:
     ip = ctypes.POINTER(i)
     lib.pa_shared_prefix_plan.argtypes = [vp, vp] + [i] * 4 + [vp, vp, vp, ip, ip]
     lib.pa_shared_prefix_plan.restype = i
+    lib.pa_shared_prefix_plan_tree.argtypes = [vp, vp] + [i] * 4 + [vp, vp, vp, ip, ip]
+    lib.pa_shared_prefix_plan_tree.restype = i
     lib.pa_shared_prefix_workspace_size.argtypes = [i] * 9 + [ctypes.POINTER(sz)]
     lib.pa_shared_prefix_workspace_size.restype = i
     lib.pa_decode_shared_prefix.argtypes = [vp] * 11 + [i] * 10 + [f, i, i, vp, sz, vp, vp]
@@ -306,8 +309,10 @@ class SharedPrefixGroups:
 
 
 def shared_prefix_plan(block_tables: np.ndarray, context_lens: np.ndarray,
-                       min_shared_blocks: int = 1) -> SharedPrefixGroups:
-    """Find the groups on the host (the library's planner; no device needed)."""
+                       min_shared_blocks: int = 1, tree: bool = False) -> SharedPrefixGroups:
+    """Find the groups on the host (the library's planner; no device needed):
+    one group per first block, or with ``tree`` groups chosen on the trie of
+    block paths (``pa_shared_prefix_plan_tree``)."""
     bt = np.ascontiguousarray(block_tables, dtype=np.int32)
     cl = np.ascontiguousarray(context_lens, dtype=np.int32)
     S = int(cl.shape[0])
@@ -318,10 +323,11 @@ def shared_prefix_plan(block_tables: np.ndarray, context_lens: np.ndarray,
     blocks = np.zeros(max(S, 1), dtype=np.int32)
     ng, nl = ctypes.c_int(0), ctypes.c_int(0)
     vp = ctypes.c_void_p
-    _check(library().pa_shared_prefix_plan(
+    fn = "pa_shared_prefix_plan_tree" if tree else "pa_shared_prefix_plan"
+    _check(getattr(library(), fn)(
         vp(bt.ctypes.data), vp(cl.ctypes.data), S, int(bt.shape[1]), 16, int(min_shared_blocks),
         vp(seqs.ctypes.data), vp(start.ctypes.data), vp(blocks.ctypes.data), ctypes.byref(ng),
-        ctypes.byref(nl)), "pa_shared_prefix_plan")
+        ctypes.byref(nl)), fn)
     return SharedPrefixGroups(seqs[:nl.value].copy(), start[:ng.value + 1].copy(),
                               blocks[:ng.value].copy())
 

@@ -164,3 +164,108 @@ def test_workspace_size_rejects_fp32(lib):
     out = ctypes.c_size_t(0)
     assert lib.pa_shared_prefix_workspace_size(4, 4, 8, 2, 128, 8, 128, 0, ops.PA_F32,
                                                ctypes.byref(out)) == ops.PA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# the tree planner (pa_shared_prefix_plan_tree)
+# ---------------------------------------------------------------------------
+def tree_reference(tables, lens, min_blocks=1):
+    """The header's rule on an explicit trie (dicts of children by block id),
+    resolved recursively: a different construction from the library's
+    sort + common-prefix stack."""
+    tmax = tables.shape[1]
+    root = {"depth": 0, "kids": {}, "here": []}
+    for s, n in enumerate(lens):
+        if n <= 0 or n > 16 * tmax or (n - 1) // 16 < min_blocks:
+            continue
+        node = root
+        for j in range((n - 1) // 16):
+            node = node["kids"].setdefault(int(tables[s, j]),
+                                           {"depth": j + 1, "kids": {}, "here": []})
+        node["here"].append(s)
+    groups = []
+
+    def walk(node, parent_depth):
+        free = list(node["here"])
+        for kid in node["kids"].values():
+            free += walk(kid, node["depth"])
+        # (a chain of single children is one node of the compressed trie:
+        # only a node that branches or ends paths decides)
+        k, d = len(free), node["depth"]
+        decides = len(node["kids"]) != 1 or node["here"]
+        if decides and k >= 2 and d >= min_blocks and (k - 1) * d >= k * parent_of[id(node)]:
+            groups.append((sorted(free), d))
+            return []
+        return free
+
+    # the parent depth that matters is that of the nearest deciding ancestor
+    parent_of = {}
+
+    def mark(node, deciding_depth):
+        decides = len(node["kids"]) != 1 or node["here"]
+        parent_of[id(node)] = deciding_depth
+        for kid in node["kids"].values():
+            mark(kid, node["depth"] if decides else deciding_depth)
+
+    mark(root, 0)
+    walk(root, 0)
+    groups.sort(key=lambda g: g[0][0])
+    return groups
+
+
+def fork_tree(seed, S=60, tmax=40):
+    """Sequences that fork earlier ones at random depths (forks of forks)."""
+    rng = np.random.default_rng(seed)
+    fresh = iter(range(10**6))
+    tables = np.zeros((S, tmax), dtype=np.int32)
+    lens = rng.integers(1, 16 * tmax + 1, size=S).astype(np.int32)
+    for s in range(S):
+        tables[s] = [next(fresh) for _ in range(tmax)]
+        if s and rng.random() < 0.85:
+            src = int(rng.integers(0, s))
+            k = int(rng.integers(1, tmax))
+            tables[s, :k] = tables[src, :k]
+    return tables, lens
+
+
+def savings(groups):
+    return sum((len(m) - 1) * P for m, P in groups)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_tree_plan_matches_its_reference(lib, seed):
+    tables, lens = fork_tree(seed)
+    plan = ops.shared_prefix_plan(tables, lens, tree=True)
+    assert as_groups(plan) == tree_reference(tables, lens)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_tree_plan_is_valid_and_saves_at_least_as_much(lib, seed):
+    tables, lens = fork_tree(100 + seed)
+    tree = as_groups(ops.shared_prefix_plan(tables, lens, tree=True))
+    flat = as_groups(ops.shared_prefix_plan(tables, lens))
+    seen = set()
+    for members, P in tree:
+        assert len(members) >= 2 and P >= 1 and members == sorted(members)
+        assert not (seen & set(members))
+        seen |= set(members)
+        for s in members:
+            assert (tables[s, :P] == tables[members[0], :P]).all() and 16 * P <= lens[s] - 1
+    assert savings(tree) >= savings(flat)
+
+
+def test_tree_plan_examples(lib):
+    t = np.arange(10 * 24, dtype=np.int32).reshape(10, 24)
+    lens = np.full(10, 16 * 24, dtype=np.int32)
+    t[1:, :10] = t[0, :10]          # ten sequences share 10 blocks
+    t[1:2, :11] = t[0, :11]         # two of them share 11: not worth a group of their own
+    assert as_groups(ops.shared_prefix_plan(t, lens, tree=True)) == [(list(range(10)), 10)]
+    t[1:4, :20] = t[0, :20]         # four share 20: (4-1)*20 >= 4*10, a group of their own
+    assert as_groups(ops.shared_prefix_plan(t, lens, tree=True)) == \
+        [([0, 1, 2, 3], 20), ([4, 5, 6, 7, 8, 9], 10)]
+    w = build_workload("prefix_cow")
+    assert as_groups(ops.shared_prefix_plan(w.block_tables, w.context_lens, tree=True)) == \
+        [(list(range(128)), 127)]
+    # different first blocks never share
+    u = np.arange(4 * 8, dtype=np.int32).reshape(4, 8)
+    assert ops.shared_prefix_plan(u, np.full(4, 100, np.int32), tree=True).num_groups == 0
