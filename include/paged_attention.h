@@ -161,7 +161,9 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
  *    returns PA_ERR_WORKSPACE and launches nothing.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture begins.
+ *    before any stream capture begins.  The address is kept for the life of
+ *    the process: after a cudaDeviceReset of that device (which destroys the
+ *    context the address belongs to), later calls on it are invalid.
  *  - All calls share the one array.  Each call first clears, on `stream`,
  *    the part that must start at zero; calls that can run at the same time
  *    on the GPU (different streams without ordering) race on the array.

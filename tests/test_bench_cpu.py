@@ -47,3 +47,13 @@ def test_dedup_flag_and_its_counters(capsys):
     # recorded DRAM counters are keyed per path; a deduplicated run's hash
     # also covers the shared-prefix pass
     assert bench.kernel_source_hash(True) != bench.kernel_source_hash()
+
+
+def test_default_run_times_the_four_large_workloads_headline_first():
+    args = bench.parse_args([])
+    names = bench.workload_names(args)
+    assert names == ("long", "7b", "gqa70b", "prefix_cow")
+    # the headline is the largest step by algorithmic bytes
+    sizes = {n: bench.step_bytes(build_workload(n), fused=True) for n in ("long", "7b")}
+    assert sizes["long"] > 2 * sizes["7b"]
+    assert bench.workload_names(bench.parse_args(["--workload", "tiny"])) == ("tiny",)

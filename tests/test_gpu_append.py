@@ -130,7 +130,8 @@ def test_host_checks():
 @pytest.mark.parametrize("name", ["tiny", "7b"])
 def test_full_size_fused_step(name):
     """The workloads whose step writes a new token, in the benchmark's launch
-    configuration: one fused call against the two-call step, bit for bit."""
+    configuration: one fused call against the two-call step, bit for bit,
+    and every output element against the oracle."""
     w = build_workload(name)
     a = upload(w)
     assert two_calls(w, a, w.partition_size) == 0
@@ -142,3 +143,7 @@ def test_full_size_fused_step(name):
     assert err == 0 and counters_zero(w, ws)
     assert same_bits(out_a, b["out"])
     assert same_bits(k_a, b["k_cache"]) and same_bits(v_a, b["v_cache"])
+    ref, _, _, oerr = oracle.workload_step(w)
+    assert oerr == 0
+    assert_attention_close(b["out"], ref, w.dtype, f"{name} (pa_decode_append, all rows)",
+                           record=True, strict_abs=w.dtype == "bf16")

@@ -31,16 +31,28 @@ def _cuda():
     ops.library()
 
 
-def assert_attention_close(gpu, ref, dtype, what=""):
+def assert_attention_close(gpu, ref, dtype, what="", record=False, strict_abs=False):
+    """The stated tolerance, element by element.  ``strict_abs`` also holds
+    bf16 results to max |gpu - ref| <= 1e-2 (the bound read as purely
+    absolute); ``record`` adds the margins to the end-of-run summary."""
     g = gpu.detach().float().cpu().numpy().astype(np.float64)
+    assert g.shape == ref.shape, f"{what}: shape {g.shape} vs {ref.shape}"
     assert np.isfinite(g).all(), f"{what}: non-finite output"
     err = np.abs(g - ref)
+    max_abs = float(err.max()) if err.size else 0.0
     if dtype == "f32":
-        assert err.max() <= F32_ATOL, f"{what}: max abs err {err.max():.3e}"
+        worst = max_abs / F32_ATOL
     else:
-        bound = BF16_ATOL + BF16_RTOL * np.abs(ref)
-        worst = (err / bound).max()
-        assert worst <= 1.0, f"{what}: max abs err {err.max():.3e}, worst err/bound {worst:.3f}"
+        worst = float((err / (BF16_ATOL + BF16_RTOL * np.abs(ref))).max()) if err.size else 0.0
+    if record:
+        from tests.conftest import PARITY_RECORDS
+        PARITY_RECORDS.append((what, int(err.size), max_abs, worst))
+    if dtype == "f32":
+        assert max_abs <= F32_ATOL, f"{what}: max abs err {max_abs:.3e}"
+    else:
+        assert worst <= 1.0, f"{what}: max abs err {max_abs:.3e}, worst err/bound {worst:.3f}"
+        if strict_abs:
+            assert max_abs <= BF16_ATOL, f"{what}: max abs err {max_abs:.3e} > {BF16_ATOL}"
 
 
 def run_gpu(w, partition_size=None, t=None, err=None):
@@ -76,7 +88,7 @@ def test_tiny_workload_full_step():
     ref, k_ref, v_ref, oerr = oracle.workload_step(w)
     t, err, ws = run_gpu(w)
     assert err == 0 and oerr == 0
-    assert_attention_close(t["out"], ref, w.dtype, "tiny")
+    assert_attention_close(t["out"], ref, w.dtype, "tiny (pa_decode)", record=True)
     # the slot write is bit-exact and leaves every other slot (NaN sentinels too) alone
     kc = t["k_cache"].cpu().numpy()[w.used_blocks]
     vc = t["v_cache"].cpu().numpy()[w.used_blocks]
@@ -297,12 +309,12 @@ def test_bad_slot_and_bad_pair_are_skipped_and_flagged():
 # ---------------------------------------------------------------------------
 # the full-size workloads, in the launch configuration the benchmark times
 # ---------------------------------------------------------------------------
-def sampled_reference(w, sel, k_pool, v_pool):
-    out, err = oracle.paged_decode(w.q[sel], k_pool, v_pool, w.tables_compact[sel],
-                                   w.context_lens[sel], scale=w.scale, dtype=w.dtype,
-                                   max_context_len=w.max_context_len)
+def full_reference(w):
+    """The oracle's whole step (copies, slot write, attention) on every
+    sequence of the workload: fp64 output and the caches after the step."""
+    out, k_ref, v_ref, err = oracle.workload_step(w)
     assert err == 0
-    return out
+    return out, k_ref, v_ref
 
 
 def pick_sequences(w, count, seed=0):
@@ -315,22 +327,18 @@ def pick_sequences(w, count, seed=0):
 
 @pytest.mark.parametrize("name", ["7b", "gqa70b", "prefix_cow", "long"])
 def test_full_size_workloads(name):
+    """The workload's whole step in the benchmark's launch configuration;
+    every output element against the oracle, every used block bit-exact."""
     w = build_workload(name)
-    k_ref, v_ref = w.k_pool.copy(), w.v_pool.copy()
-    if w.block_mapping_compact is not None:
-        assert oracle.copy_blocks(k_ref, v_ref, w.block_mapping_compact) == 0
-    if w.new_key is not None:
-        assert oracle.reshape_and_cache(k_ref, v_ref, w.new_key, w.new_value,
-                                        w.slot_mapping_compact) == 0
+    ref, k_ref, v_ref = full_reference(w)
     t, err, ws = run_gpu(w)
     assert err == 0
     # slot write and copies: every used block bit-exact
     idx = torch.from_numpy(w.used_blocks).cuda()
-    for dev, ref in ((t["k_cache"], k_ref), (t["v_cache"], v_ref)):
+    for dev, host in ((t["k_cache"], k_ref), (t["v_cache"], v_ref)):
         got = dev[idx].view(torch.int16).cpu().numpy()
-        assert np.array_equal(got, ref.view(np.int16)), "cache bytes differ"
-    sel = pick_sequences(w, 3 if name == "long" else 8)
-    ref = sampled_reference(w, sel, k_ref, v_ref)
-    assert_attention_close(t["out"][torch.from_numpy(sel).cuda()], ref, w.dtype, name)
-    assert torch.isfinite(t["out"].float()).all()
+        assert np.array_equal(got, host.view(np.int16)), "cache bytes differ"
+    del idx
+    assert_attention_close(t["out"], ref, w.dtype, f"{name} (pa_decode, all rows)", record=True,
+                           strict_abs=True)
     assert counters_zero(w, ws)

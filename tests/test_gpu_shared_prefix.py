@@ -19,7 +19,7 @@ import oracle
 from paged_kv_cache_456_b200 import ops
 from paged_kv_cache_456_b200.workloads import build_workload, make_workload, upload
 
-from tests.test_gpu_parity import assert_attention_close, pick_sequences
+from tests.test_gpu_parity import assert_attention_close
 
 pytestmark = pytest.mark.gpu
 
@@ -206,17 +206,82 @@ def test_no_groups_is_plain_decode():
 
 
 def test_full_prefix_cow_workload():
+    """The benchmark's deduplicated step: every output element against the
+    oracle, every used block bit-exact after the copy-on-write copies."""
     w = build_workload("prefix_cow")     # (copy-on-write copies, then attention)
     t, err, _ = run_shared(w)
     assert err == 0
-    k_ref, v_ref = w.k_pool.copy(), w.v_pool.copy()
-    assert oracle.copy_blocks(k_ref, v_ref, w.block_mapping_compact) == 0
+    ref, k_ref, v_ref, e = reference(w)
+    assert e == 0
     idx = torch.from_numpy(w.used_blocks).cuda()
     for dev, host in ((t["k_cache"], k_ref), (t["v_cache"], v_ref)):
         assert np.array_equal(dev[idx].view(torch.int16).cpu().numpy(), host.view(np.int16))
-    sel = pick_sequences(w, 12)
-    ref, e = oracle.paged_decode(w.q[sel], k_ref, v_ref, w.tables_compact[sel], w.context_lens[sel],
-                                 scale=w.scale, dtype=w.dtype, max_context_len=w.max_context_len)
+    assert_attention_close(t["out"], ref, "bf16", "prefix_cow (deduplicated, all rows)",
+                           record=True, strict_abs=True)
+
+
+def fork_tree_workload(seed=17, G=4, D=128):
+    """Sharing that forms a tree: a 20-block root prompt held by 24 sequences;
+    two forks of it hold 12 more blocks each (8 sequences each), and one of
+    those forks is forked again for 4 sequences (8 blocks more)."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(16 * 44 + 1, 16 * 44 + 300, size=28)
+    w = make_workload(rng, name="tree", dtype="bf16", num_q_heads=2 * G, num_kv_heads=2,
+                      head_dim=D, context_lens=lens, num_blocks=int(sum(-(-lens // 16))) + 8)
+    share(w, range(1, 24), 0, 20)        # root prompt: sequences 0..23
+    share(w, range(1, 8), 0, 32)         # fork A: 0..7 share 32 blocks
+    share(w, range(9, 16), 8, 32)        # fork B: 8..15 share 32 blocks
+    share(w, range(13, 16), 12, 40)      # fork of B: 12..15 share 40 blocks
+    return w                             # 24..27 share nothing
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_tree_plan_on_the_device(fused):
+    """A plan from pa_shared_prefix_plan_tree (groups at different depths,
+    members whose blocks past the group's depth are shared with sibling
+    groups) through the pass and the decode continuation, against the oracle
+    and against plain decode."""
+    w = fork_tree_workload()
+    if fused:
+        rng = np.random.default_rng(99)
+        k_new = rng.standard_normal((w.num_seqs, w.num_kv_heads, w.head_dim), dtype=np.float32)
+        v_new = rng.standard_normal((w.num_seqs, w.num_kv_heads, w.head_dim), dtype=np.float32)
+    plan = ops.shared_prefix_plan(w.block_tables, w.context_lens, tree=True)
+    depths = sorted(int(b) for b in plan.blocks[:plan.num_groups])
+    assert len(set(depths)) >= 2, depths          # groups at different depths
+    t = upload(w)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = ops.make_shared_prefix_workspace(w.num_seqs, plan.num_listed, w.num_q_heads,
+                                          w.num_kv_heads, w.head_dim, w.max_blocks_per_seq,
+                                          w.max_context_len, w.partition_size)
+    k_ref, v_ref = w.k_pool.copy(), w.v_pool.copy()
+    key = value = None
+    if fused:
+        # the new token of each sequence (its last position, in a private block)
+        from paged_kv_cache_456_b200.workloads import f32_to_bf16_bits
+        kb, vb = f32_to_bf16_bits(k_new), f32_to_bf16_bits(v_new)
+        key = torch.from_numpy(kb).view(torch.bfloat16).cuda()
+        value = torch.from_numpy(vb).view(torch.bfloat16).cuda()
+        n = w.context_lens.astype(np.int64)
+        slots = w.tables_compact[np.arange(w.num_seqs), (n - 1) // 16].astype(np.int64) * 16 + \
+            (n - 1) % 16
+        assert oracle.reshape_and_cache(k_ref, v_ref, kb, vb, slots) == 0
+    ops.decode_shared_prefix(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                             t["context_lens"], plan.to(), scale=w.scale,
+                             max_context_len=w.max_context_len, workspace=ws, key=key,
+                             value=value, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref, e = oracle.paged_decode(w.q, k_ref, v_ref, w.tables_compact, w.context_lens,
+                                 scale=w.scale, dtype=w.dtype)
     assert e == 0
-    assert_attention_close(t["out"][torch.from_numpy(sel).cuda()], ref, "bf16", "prefix_cow")
-    assert torch.isfinite(t["out"].float()).all()
+    assert_attention_close(t["out"], ref, "bf16", f"tree plan fused={fused}")
+    # plain decode of the same step agrees within the same bound
+    dec = torch.empty_like(t["out"])
+    ws2 = ops.make_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                             w.max_context_len, 0, torch.bfloat16)
+    ops.decode(dec, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+               scale=w.scale, max_context_len=w.max_context_len, workspace=ws2, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert_attention_close(dec, ref, "bf16", "plain decode after the tree-plan step")

@@ -6,7 +6,10 @@ device synchronisation an allocation may cause.  pa_decode_noalloc takes its
 scratch from a fixed array inside the library instead of a caller workspace.
 These tests call it through the C ABI twice in a row (different inputs each
 time, so the second call starts from whatever the first left in the shared
-array) and compare it with pa_decode using its own workspace.
+array), on the CUDA-core path (bf16 and fp32 caches) and on the tensor-core
+path (bf16, 8 query heads per KV head).  Each call must give the same bits
+as pa_decode with a workspace of its own (same plan, same kernels) and stay
+within the oracle's tolerance.
 
 This file is named so pytest collects it last.
 """
@@ -14,10 +17,14 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from paged_kv_cache_456_b200 import ops
 from paged_kv_cache_456_b200.workloads import random_workload, upload
 
 pytestmark = pytest.mark.gpu
+
+F32_ATOL = 1e-5
+BF16_TOL = 1e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -29,28 +36,37 @@ def _cuda():
     ops.library()
 
 
-def _close(a, b):
-    a = a.float().cpu().numpy().astype(np.float64)
-    b = b.float().cpu().numpy().astype(np.float64)
-    assert np.isfinite(a).all()
-    assert (np.abs(a - b) <= 1e-2 + 1e-2 * np.abs(b)).all(), np.abs(a - b).max()
+def _within_oracle(gpu, ref, dtype):
+    g = gpu.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(g).all()
+    err = np.abs(g - ref)
+    if dtype == "f32":
+        assert err.max() <= F32_ATOL, err.max()
+    else:
+        assert (err <= BF16_TOL + BF16_TOL * np.abs(ref)).all(), err.max()
 
 
+SHAPES = [("bf16", 128, 4), ("bf16", 128, 8), ("f32", 64, 4)]
+
+
+@pytest.mark.parametrize("dtype,D,G", SHAPES, ids=lambda x: str(x))
 @pytest.mark.parametrize("partition_size", [0, 64])
-def test_noalloc_matches_pa_decode_on_two_calls_in_a_row(partition_size):
+def test_noalloc_matches_pa_decode_on_two_calls_in_a_row(dtype, D, G, partition_size):
     lens = [1, 16, 17, 300, 1000, 45, 0, 2049]
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    iv = torch.int16 if dtype == "bf16" else torch.int32
     for seed in (1, 2):                     # two calls in a row on the shared scratch
-        w = random_workload(seed, dtype="bf16", num_q_heads=16, num_kv_heads=4, head_dim=128,
+        w = random_workload(seed, dtype=dtype, num_q_heads=2 * G, num_kv_heads=2, head_dim=D,
                             lens=lens, spare_blocks=20)
         need = ops.workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                                  w.max_context_len, partition_size, torch.bfloat16)
+                                  w.max_context_len, partition_size, tdt)
         assert need <= ops.NOALLOC_SCRATCH_BYTES
         t = upload(w)
         ws = ops.make_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                                w.max_context_len, partition_size, torch.bfloat16)
-        ref = torch.empty_like(t["out"])
+                                w.max_context_len, partition_size, tdt)
+        own = torch.empty_like(t["out"])
         err = torch.zeros(2, dtype=torch.int32, device="cuda")
-        ops.decode(ref, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+        ops.decode(own, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
                    scale=w.scale, max_context_len=w.max_context_len, workspace=ws,
                    partition_size=partition_size, err_flag=err[0:1])
         t["out"].fill_(3.0)
@@ -59,7 +75,12 @@ def test_noalloc_matches_pa_decode_on_two_calls_in_a_row(partition_size):
                            partition_size=partition_size, err_flag=err[1:2])
         torch.cuda.synchronize()
         assert err.tolist() == [0, 0]
-        _close(t["out"], ref)
+        assert torch.equal(t["out"].view(iv), own.view(iv))
+        ref, oerr = oracle.paged_decode(w.q, w.k_pool, w.v_pool, w.tables_compact,
+                                        w.context_lens, scale=w.scale, dtype=w.dtype)
+        assert oerr == 0
+        _within_oracle(t["out"], ref, dtype)
+        assert (t["out"][6] == 0).all()     # the empty sequence
 
 
 def test_noalloc_rejects_a_request_larger_than_its_scratch():
