@@ -93,34 +93,8 @@ struct DecodePlan {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// A cache as the 2-D bf16 tensor [rows][head_dim] read by the tensor-core
-// path in boxes of 16 rows x 64 elements (128 bytes) with the 128-byte
-// swizzle.  The encoder is a host-side driver routine, looked up once.
 pa_status encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim) {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!encode) {
-      void* fn = nullptr;
-      cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
-                                           &q) != cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || !fn) {
-        cudaGetLastError();
-        return PA_ERR_CUDA;
-      }
-      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    }
-  }
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pa::kBlockSize)};
-  const cuuint32_t elem_strides[2] = {1, 1};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
-                            dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+  return pa::encode_cache_map(map, base, rows, head_dim) ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status occupancy(const pa::DecodeKernelInfo& k, size_t smem, int* occ) {
@@ -169,10 +143,9 @@ pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, in
 
 // table_rows >= 0: several query tokens per sequence; num_seqs counts query
 // rows and the kernel also keeps their table rows and query_start on chip.
-// shared_prefix: the kernel keeps each sequence's block offset on chip.
 pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                     int max_context_len, int partition_size, pa_dtype dtype, DecodePlan* p,
-                    int table_rows = -1, bool shared_prefix = false) {
+                    int table_rows = -1) {
   pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                     max_context_len, partition_size, dtype);
   if (st != PA_OK) return st;
@@ -200,7 +173,6 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     if (p->kernel.rows_per_item > 1)
       seq_ints += static_cast<size_t>(num_seqs) + table_rows + 1;  // group rows, group starts
   }
-  if (shared_prefix) seq_ints += static_cast<size_t>(num_seqs);  // blocks attended already
   const size_t seq_bytes = round_up(seq_ints * sizeof(int), 16);
   p->smem = static_cast<size_t>(p->kernel.cta_bytes) + seq_bytes;
   if (p->smem > static_cast<size_t>(dev.smem_optin)) return PA_ERR_UNSUPPORTED;
@@ -237,6 +209,36 @@ pa_status make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
 }
 
 }  // namespace
+
+// A cache as the 2-D bf16 tensor [rows][head_dim] read by the tensor-core
+// paths in boxes of 16 rows x 64 elements (128 bytes) with the 128-byte
+// swizzle.  The encoder is a host-side driver routine, looked up once.
+bool pa::encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return false;
+      }
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(pa::kBlockSize)};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                            dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 size_t pa::decode_zero_prefix_bytes(int num_seqs, int num_kv_heads) {
   return 8 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
@@ -281,10 +283,30 @@ static int prefill_items(int num_seqs, int num_query_tokens, int num_q_heads, in
   return static_cast<int>(items < num_query_tokens ? items : num_query_tokens);
 }
 
+// Several query tokens per sequence go to the tcgen05 kernel (bf16 caches)
+// unless the library is built with PA_PREFILL_TC=0; fp32 caches always take
+// the decode kernel with query rows as items.
+#ifndef PA_PREFILL_TC
+#define PA_PREFILL_TC 1
+#endif
+static bool prefill_on_tensor_cores(int num_q_heads, int num_kv_heads, int head_dim,
+                                    pa_dtype dtype) {
+  return PA_PREFILL_TC && dtype == PA_BF16 && num_kv_heads > 0 && num_q_heads > 0 &&
+         num_q_heads % num_kv_heads == 0 &&
+         pa::tc_prefill_supported(head_dim, num_q_heads / num_kv_heads);
+}
+
 pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_q_heads,
                                     int num_kv_heads, int head_dim, int max_context_len,
                                     int partition_size, pa_dtype dtype, size_t* bytes) {
   if (!bytes || num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (prefill_on_tensor_cores(num_q_heads, num_kv_heads, head_dim, dtype)) {
+    const pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
+                                            max_context_len, partition_size, dtype);
+    if (st != PA_OK) return st;
+    *bytes = round_up(pa::tc_prefill_workspace_bytes(num_seqs), 256);
+    return PA_OK;
+  }
   DecodePlan p;
   const int items = prefill_items(num_seqs, num_query_tokens, num_q_heads, num_kv_heads,
                                   head_dim, dtype);
@@ -323,6 +345,18 @@ pa_status pa_prefill_launch_config(int num_seqs, int num_query_tokens, int num_q
                                    int partition_size, pa_dtype dtype, int* grid,
                                    int* warps_per_cta, int* pipeline_depth, int* smem_bytes) {
   if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (prefill_on_tensor_cores(num_q_heads, num_kv_heads, head_dim, dtype)) {
+    pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
+                                      max_context_len, partition_size, dtype);
+    if (st != PA_OK) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != PA_OK) return st;
+    if (grid) *grid = dev.sms;
+    if (warps_per_cta) *warps_per_cta = pa::kTcWarps;
+    if (pipeline_depth) *pipeline_depth = 2;
+    if (smem_bytes) *smem_bytes = pa::tc_launch_smem(head_dim);
+    return PA_OK;
+  }
   DecodePlan p;
   const int items = prefill_items(num_seqs, num_query_tokens, num_q_heads, num_kv_heads,
                                   head_dim, dtype);
@@ -365,8 +399,7 @@ pa_status decode_impl(void* out, const void* q, const void* key, const void* val
     return PA_ERR_UNSUPPORTED;
   DecodePlan p;
   if ((st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                      partition_size, dtype, &p, query_start ? table_rows : -1,
-                      pre != nullptr)) != PA_OK)
+                      partition_size, dtype, &p, query_start ? table_rows : -1)) != PA_OK)
     return st;
   if (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace))
     return PA_ERR_WORKSPACE;
@@ -479,6 +512,56 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
   if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
   if (num_query_tokens == 0) return PA_OK;
   if (num_seqs == 0 || !query_start) return PA_ERR_INVALID_ARG;
+  if (prefill_on_tensor_cores(num_q_heads, num_kv_heads, head_dim, dtype)) {
+    pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
+                                      max_context_len, partition_size, dtype);
+    if (st != PA_OK) return st;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0 || block_size <= 0 || !std::isfinite(scale))
+      return PA_ERR_INVALID_ARG;
+    if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+      return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+      return PA_ERR_INVALID_ARG;
+    const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
+    if (rows + pa::kBlockSize >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < pa::tc_prefill_workspace_bytes(num_seqs) ||
+        !aligned16(workspace))
+      return PA_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != PA_OK) return st;
+    if (static_cast<size_t>(pa::tc_launch_smem(head_dim)) > static_cast<size_t>(dev.smem_optin))
+      return PA_ERR_UNSUPPORTED;
+    CUtensorMap tk, tv;
+    if ((st = encode_cache_map(&tk, k_cache, rows, head_dim)) != PA_OK ||
+        (st = encode_cache_map(&tv, v_cache, rows, head_dim)) != PA_OK)
+      return st;
+    pa::TcPrefillLaunch l{};
+    l.q = q;
+    l.out = out;
+    l.block_tables = block_tables;
+    l.context_lens = context_lens;
+    l.query_start = query_start;
+    l.num_seqs = num_seqs;
+    l.num_query_rows = num_query_tokens;
+    l.num_q_heads = num_q_heads;
+    l.num_kv_heads = num_kv_heads;
+    l.head_dim = head_dim;
+    l.max_blocks_per_seq = max_blocks_per_seq;
+    l.num_blocks = num_blocks;
+    const long long cap = static_cast<long long>(max_blocks_per_seq) * pa::kBlockSize;
+    l.len_cap = static_cast<int>(max_context_len < cap ? max_context_len : cap);
+    l.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    l.workspace = workspace;
+    l.err_flag = err_flag;
+    l.tm_k = &tk;
+    l.tm_v = &tv;
+    if (pa::launch_tc_prefill(l, dev.sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+      cudaGetLastError();
+      return PA_ERR_CUDA;
+    }
+    return PA_OK;
+  }
   const int items = prefill_items(num_seqs, num_query_tokens, num_q_heads, num_kv_heads,
                                   head_dim, dtype);
   return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens,
@@ -496,7 +579,7 @@ pa_status pa_shared_prefix_workspace_size(int num_seqs, int num_listed, int num_
   if (dtype != PA_BF16) return dtype == PA_F32 ? PA_ERR_UNSUPPORTED : PA_ERR_INVALID_ARG;
   DecodePlan p;
   const pa_status st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                                 partition_size, dtype, &p, -1, true);
+                                 partition_size, dtype, &p);
   if (st != PA_OK) return st;
   const size_t extra = pa::shared_prefix_workspace_bytes(num_seqs, num_listed, num_q_heads,
                                                          head_dim, max_blocks_per_seq);
@@ -541,7 +624,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, con
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
   DecodePlan p;
   if ((st = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                      partition_size, dtype, &p, -1, true)) != PA_OK)
+                      partition_size, dtype, &p)) != PA_OK)
     return st;
   const size_t dec_bytes = round_up(p.ws_bytes, 256);
   pa::SharedPrefixLaunch l{};
@@ -566,6 +649,14 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, con
   l.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   l.workspace = static_cast<char*>(workspace) + dec_bytes;
   l.err_flag = err_flag;
+  CUtensorMap tk, tv;
+  const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
+  if (rows + pa::kBlockSize < (1LL << 31) && num_groups > 0 &&
+      encode_cache_map(&tk, k_cache, rows, head_dim) == PA_OK &&
+      encode_cache_map(&tv, v_cache, rows, head_dim) == PA_OK) {
+    l.tm_k = &tk;
+    l.tm_v = &tv;
+  }
   if (pa::launch_shared_prefix(l, p.sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return PA_ERR_CUDA;

@@ -146,6 +146,8 @@ struct SharedPrefixLaunch {
   float scale_log2;
   void* workspace;              // shared_prefix_workspace_bytes(...) bytes, zero on first use
   int32_t* err_flag;
+  const CUtensorMap* tm_k;      // the caches' tensor maps (tensor-core pass)
+  const CUtensorMap* tm_v;
   // outputs for the decode kernel (inside the workspace)
   int32_t* pre_blocks;
   float* pre_o;
@@ -157,5 +159,72 @@ size_t shared_prefix_workspace_bytes(int num_seqs, int num_listed, int num_q_hea
 // Fills pre_blocks / pre_o / pre_ml of `l` from its workspace and launches the
 // pass; returns cudaSuccess or the launch error.
 cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_t stream);
+
+// A cache as the 2-D bf16 tensor [num_blocks * num_kv_heads * 16][head_dim],
+// read in boxes of 16 rows x 64 elements with the 128-byte swizzle (abi.cu).
+bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim);
+
+// ---- tensor-core attention of many query columns (tc_attention.cu) ----------
+// Several query tokens per sequence: one column per (query row, query head),
+// 128 columns per MMA tile, on the tcgen05 tensor cores (bf16).
+struct TcPrefillLaunch {
+  const void* q;
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start;
+  int num_seqs;        // block-table rows
+  int num_query_rows;  // rows of q and out
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int len_cap;
+  float scale_log2;
+  void* workspace;     // tc_prefill_workspace_bytes(num_seqs) bytes (no zeroing needed)
+  int32_t* err_flag;
+  const CUtensorMap* tm_k;
+  const CUtensorMap* tm_v;
+};
+bool tc_prefill_supported(int head_dim, int group);
+size_t tc_prefill_workspace_bytes(int num_seqs);
+int tc_launch_smem(int head_dim);
+constexpr int kTcWarps = 6;
+cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_t stream);
+
+// The shared-prefix pass on the tcgen05 tensor cores: (member, query head)
+// columns of a group, 128 per tile, over ranges of the group's shared blocks.
+struct TcSharedLaunch {
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* group_seqs;
+  const int32_t* group_start;
+  const int32_t* group_blocks;
+  int num_groups;
+  int num_listed;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int len_cap;
+  int max_ranges;      // ranges the partial arrays hold per column
+  float scale_log2;
+  int* unit_start;     // [num_groups + 1]
+  int* counters;       // [num_listed * Hq], zero between calls
+  int* claim;          // [num_seqs], zeroed before the pass
+  float2* part_ml;
+  float* part_o;
+  float2* pre_ml;
+  float* pre_o;
+  int32_t* err_flag;
+  const CUtensorMap* tm_k;
+  const CUtensorMap* tm_v;
+};
+bool tc_shared_prefix_supported(int head_dim, int group);
+cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaStream_t stream);
 
 }  // namespace pa

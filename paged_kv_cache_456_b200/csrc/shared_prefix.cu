@@ -61,6 +61,12 @@ constexpr int kPCols = 8 * NTW * kPWarps;     // (member, head) columns of a uni
 constexpr int kPStages = 6;           // ring of K/V tiles: 5 in flight while one is used
 constexpr int kMinRangeTiles = PA_SP_MINRANGE;  // shortest range of shared blocks per unit
 constexpr int kMaxChunkMembers = kPCols + 1;
+// The pass runs on the tcgen05 tensor cores (tc_attention.cu) unless built
+// with PA_SHARED_TC=0, which keeps the warp-level MMA pass below.
+#ifndef PA_SHARED_TC
+#define PA_SHARED_TC 1
+#endif
+constexpr bool kSharedOnTensorCores = PA_SHARED_TC != 0;
 
 struct PrefixArgs {
   const __nv_bfloat16* q;
@@ -499,7 +505,7 @@ int min_range_tiles(int max_blocks_per_seq, int head_dim) {
 }
 
 struct Layout {
-  size_t counters, claim, part_ml, part_o, pre_ml, pre_o, bytes;
+  size_t counters, claim, part_ml, part_o, pre_ml, pre_o, unit_start, bytes;
   int max_ranges;
 };
 
@@ -516,7 +522,9 @@ Layout layout(int num_seqs, int num_listed, int num_q_heads, int head_dim,
   l.part_o = round_up(l.part_ml + cols * l.max_ranges * sizeof(float2), 256);
   l.pre_ml = round_up(l.part_o + cols * l.max_ranges * head_dim * sizeof(float), 256);
   l.pre_o = round_up(l.pre_ml + rows * sizeof(float2), 256);
-  l.bytes = round_up(l.pre_o + rows * head_dim * sizeof(float), 256);
+  // (the tensor-core pass: work units before each group; groups <= sequences)
+  l.unit_start = round_up(l.pre_o + rows * head_dim * sizeof(float), 256);
+  l.bytes = round_up(l.unit_start + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
   return l;
 }
 
@@ -568,6 +576,37 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
   cudaError_t e = cudaMemsetAsync(l.pre_blocks, 0, static_cast<size_t>(l.num_seqs) * sizeof(int),
                                   stream);
   if (e != cudaSuccess || l.num_groups == 0) return e;
+  if (kSharedOnTensorCores && l.tm_k && tc_shared_prefix_supported(l.head_dim, group)) {
+    TcSharedLaunch t{};
+    t.q = l.q;
+    t.block_tables = l.block_tables;
+    t.context_lens = l.context_lens;
+    t.group_seqs = l.group_seqs;
+    t.group_start = l.group_start;
+    t.group_blocks = l.group_blocks;
+    t.num_groups = l.num_groups;
+    t.num_listed = l.num_listed;
+    t.num_seqs = l.num_seqs;
+    t.num_q_heads = l.num_q_heads;
+    t.num_kv_heads = l.num_kv_heads;
+    t.head_dim = l.head_dim;
+    t.max_blocks_per_seq = l.max_blocks_per_seq;
+    t.num_blocks = l.num_blocks;
+    t.len_cap = l.len_cap;
+    t.max_ranges = lo.max_ranges;
+    t.scale_log2 = l.scale_log2;
+    t.unit_start = reinterpret_cast<int*>(ws + lo.unit_start);
+    t.counters = reinterpret_cast<int*>(ws + lo.counters);
+    t.claim = l.pre_blocks;
+    t.part_ml = reinterpret_cast<float2*>(ws + lo.part_ml);
+    t.part_o = reinterpret_cast<float*>(ws + lo.part_o);
+    t.pre_ml = l.pre_ml;
+    t.pre_o = l.pre_o;
+    t.err_flag = l.err_flag;
+    t.tm_k = l.tm_k;
+    t.tm_v = l.tm_v;
+    return launch_tc_shared_prefix(t, num_sms, stream);
+  }
 
   PrefixArgs a;
   a.q = static_cast<const __nv_bfloat16*>(l.q);
