@@ -304,7 +304,9 @@ pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_
     const pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
                                             max_context_len, partition_size, dtype);
     if (st != PA_OK) return st;
-    *bytes = round_up(pa::tc_prefill_workspace_bytes(num_seqs), 256);
+    *bytes = round_up(pa::tc_prefill_workspace_bytes(num_seqs, num_query_tokens, num_q_heads,
+                                                     num_kv_heads),
+                      256);
     return PA_OK;
   }
   DecodePlan p;
@@ -525,7 +527,9 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
       return PA_ERR_INVALID_ARG;
     const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * pa::kBlockSize;
     if (rows + pa::kBlockSize >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
-    if (!workspace || workspace_bytes < pa::tc_prefill_workspace_bytes(num_seqs) ||
+    if (!workspace ||
+        workspace_bytes < pa::tc_prefill_workspace_bytes(num_seqs, num_query_tokens,
+                                                          num_q_heads, num_kv_heads) ||
         !aligned16(workspace))
       return PA_ERR_WORKSPACE;
     DeviceInfo dev;

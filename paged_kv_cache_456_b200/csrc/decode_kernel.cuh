@@ -72,6 +72,17 @@ constexpr int kMaxOwnRanges = 4;  // range starts a warp keeps in shared memory
 #endif
 constexpr bool kProxyFence = PA_PROXY_FENCE != 0;
 
+// K/V tiles are read once per call: loaded under the L2 evict-first policy
+// (1), the partial results the merge pass reads back stay in L2 instead of
+// being pushed out by the stream; 0 loads them under the default policy.
+// Measured on B200 (fraction of the copy peak, decode + merge): 7b 0.784 ->
+// 0.802, gqa70b 0.736 -> 0.759, long 0.869 -> 0.882; a shared prefix re-read
+// by many sequences loses a little (prefix_cow 0.928 -> 0.916).
+#ifndef PA_KV_EVICT_FIRST
+#define PA_KV_EVICT_FIRST 1
+#endif
+constexpr bool kKvEvictFirst = PA_KV_EVICT_FIRST != 0;
+
 // -- element conversion ---------------------------------------------------------
 template <typename T>
 struct Elem;
@@ -301,7 +312,7 @@ constexpr int kPrefix = 1 << 29; // first tile of an item that continues a share
 
 __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const int* s_start,
                                                const int* s_len, const int* s_row,
-                                               const int* s_boff, const Ranges& rg,
+                                               const Ranges& rg,
                                                const OwnRanges& own, const DecodeArgs& a) {
   StageDesc d{0, 0, 0, 0};
   if (g >= hi) return d;
@@ -322,8 +333,10 @@ __device__ __forceinline__ StageDesc make_desc(long long g, long long hi, const 
   if (g == item_a || own.is_start(g, rg)) flags |= kFirst;
   if (g + 1 == item_a + nb || own.is_start(g + 1, rg)) flags |= kLast;
   const int trow = s_row ? s_row[s] : s;  // (query rows share their sequence's table)
-  // (shared-prefix decode: the sequence's first boff blocks were attended already)
-  const int boff = s_boff ? s_boff[s] : 0;
+  // (shared-prefix decode: the sequence's first boff blocks were attended
+  // already; read beside the table entry rather than kept on chip, which
+  // would cost the CTA shared memory per sequence)
+  const int boff = a.pre_blocks ? max(__ldg(a.pre_blocks + s), 0) : 0;
   if (boff > 0 && g == item_a) flags |= kPrefix;
   int phys = __ldg(a.block_tables + static_cast<size_t>(trow) * a.max_blocks_per_seq + boff + blk);
   if (phys < 0 || phys >= a.num_blocks) {
@@ -418,8 +431,6 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   // NR > 1: first query row | (rows << 24) of each group; first group of each sequence
   int* s_r0 = s_qs + a.num_table_rows + 1;                                   // [S]
   int* s_gs = s_r0 + S;                                                      // [rows + 1]
-  // shared-prefix decode: leading blocks of each sequence attended already
-  int* s_boff = (!prefill && a.pre_blocks) ? s_len + S : nullptr;            // [S]
 
   if (leader && lane == 0) {
 #pragma unroll
@@ -521,7 +532,6 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
       if (n < 0) n = 0;
       s_len[s] = n;
       if (prefill) s_row[s] = row;
-      if (s_boff) s_boff[s] = n > 0 ? max(a.pre_blocks[s], 0) : 0;
       if (NR > 1) s_r0[s] = r0nr;
       local += (n + kBlockSize - 1) / kBlockSize;
     }
@@ -620,7 +630,7 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
   int known = n0;                      // positions with a tile assigned
   bool no_more = rg.R == rg.Rs;        // no chunks left to claim
   auto static_desc = [&](int p) -> StageDesc {
-    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, s_row, s_boff, rg, own, a) : StageDesc{0, 0, 0, 0};
+    return p < n0 ? make_desc(lo + p, hi, s_start, s_len, s_row, rg, own, a) : StageDesc{0, 0, 0, 0};
   };
   StageDesc A{0, 0, 0, 0}, B{0, 0, 0, 0};
   int base = 0;
@@ -640,14 +650,15 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
     const long long g0 = rg.Ws + static_cast<long long>(c) * rg.CS;
     const int len = static_cast<int>(rg.CS < W - g0 ? rg.CS : W - g0);
     const int pa = base + lane, pb = base + 32 + lane;
-    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, s_row, s_boff, rg, own, a);
-    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, s_row, s_boff, rg, own, a);
+    if (pa >= known && pa < known + len) A = make_desc(g0 + (pa - known), W, s_start, s_len, s_row, rg, own, a);
+    if (pb >= known && pb < known + len) B = make_desc(g0 + (pb - known), W, s_start, s_len, s_row, rg, own, a);
     known += len;
   };
   auto top_up = [&](int frontier) {
     while (!no_more && known - frontier < kClaimAhead) claim();
   };
 
+  const uint64_t kv_policy = kKvEvictFirst ? l2_policy_evict_first() : 0;
   // Leader: fill ring slot j % DEPTH with tile j (K and V rows, plus the q rows
   // of all GT heads on a piece start) -- or with the end marker -- once every
   // warp has released the slot.  The slot's descriptor goes with it.
@@ -680,8 +691,13 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
           const int y = (e.phys * Hkv + kvh) * kBlockSize;
 #pragma unroll
           for (int hx = 0; hx < D / 64; ++hx) {
-            tma_load_2d(dst + hx * 2048, &a.tm_k, hx * 64, y, bar);
-            tma_load_2d(dst + C::TILE + hx * 2048, &a.tm_v, hx * 64, y, bar);
+            if (kKvEvictFirst) {
+              tma_load_2d_hint(dst + hx * 2048, &a.tm_k, hx * 64, y, bar, kv_policy);
+              tma_load_2d_hint(dst + C::TILE + hx * 2048, &a.tm_v, hx * 64, y, bar, kv_policy);
+            } else {
+              tma_load_2d(dst + hx * 2048, &a.tm_k, hx * 64, y, bar);
+              tma_load_2d(dst + C::TILE + hx * 2048, &a.tm_v, hx * 64, y, bar);
+            }
           }
           if (app) {
             const size_t src = (static_cast<size_t>(e.seq) * Hkv + kvh) * C::ROW;
@@ -707,8 +723,14 @@ paged_decode_kernel(const __grid_constant__ DecodeArgs a) {
         // with a fused append the last live row comes from key/value, not the cache
         const uint32_t cached = (e.meta & kAppend) ? kv_bytes - C::ROW : kv_bytes;
         if (cached) {
-          bulk_copy_g2s(dst, static_cast<const char*>(a.k_cache) + off, cached, bar);
-          bulk_copy_g2s(dst + C::TILE, static_cast<const char*>(a.v_cache) + off, cached, bar);
+          if (kKvEvictFirst) {
+            bulk_copy_g2s_hint(dst, static_cast<const char*>(a.k_cache) + off, cached, bar, kv_policy);
+            bulk_copy_g2s_hint(dst + C::TILE, static_cast<const char*>(a.v_cache) + off, cached, bar,
+                               kv_policy);
+          } else {
+            bulk_copy_g2s(dst, static_cast<const char*>(a.k_cache) + off, cached, bar);
+            bulk_copy_g2s(dst + C::TILE, static_cast<const char*>(a.v_cache) + off, cached, bar);
+          }
         }
         if (e.meta & kAppend) {
           const size_t src = (static_cast<size_t>(e.seq) * Hkv + kvh) * C::ROW;

@@ -182,13 +182,14 @@ struct TcPrefillLaunch {
   int num_blocks;
   int len_cap;
   float scale_log2;
-  void* workspace;     // tc_prefill_workspace_bytes(num_seqs) bytes (no zeroing needed)
+  void* workspace;     // tc_prefill_workspace_bytes(...) bytes (no zeroing needed)
   int32_t* err_flag;
   const CUtensorMap* tm_k;
   const CUtensorMap* tm_v;
 };
 bool tc_prefill_supported(int head_dim, int group);
-size_t tc_prefill_workspace_bytes(int num_seqs);
+size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_heads,
+                                  int num_kv_heads);
 int tc_launch_smem(int head_dim);
 constexpr int kTcWarps = 6;
 cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_t stream);
@@ -214,6 +215,8 @@ struct TcSharedLaunch {
   int max_ranges;      // ranges the partial arrays hold per column
   float scale_log2;
   int* unit_start;     // [num_groups + 1]
+  int4* units;         // [max_units][2] work-unit records
+  int max_units;
   int* counters;       // [num_listed * Hq], zero between calls
   int* claim;          // [num_seqs], zeroed before the pass
   float2* part_ml;

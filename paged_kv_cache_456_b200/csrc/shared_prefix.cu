@@ -505,8 +505,9 @@ int min_range_tiles(int max_blocks_per_seq, int head_dim) {
 }
 
 struct Layout {
-  size_t counters, claim, part_ml, part_o, pre_ml, pre_o, unit_start, bytes;
+  size_t counters, claim, part_ml, part_o, pre_ml, pre_o, unit_start, units, bytes;
   int max_ranges;
+  long long max_units;
 };
 
 Layout layout(int num_seqs, int num_listed, int num_q_heads, int head_dim,
@@ -524,7 +525,13 @@ Layout layout(int num_seqs, int num_listed, int num_q_heads, int head_dim,
   l.pre_o = round_up(l.pre_ml + rows * sizeof(float2), 256);
   // (the tensor-core pass: work units before each group; groups <= sequences)
   l.unit_start = round_up(l.pre_o + rows * head_dim * sizeof(float), 256);
-  l.bytes = round_up(l.unit_start + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
+  // its unit records: per group ceil(members * G / 128) <= members * G / 128 + 1
+  // column tiles for each KV head and range, so at most
+  // (ceil(listed * Hq / 128) + listed * Hq) x max_ranges in all
+  l.units = round_up(l.unit_start + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
+  l.max_units = ((static_cast<long long>(num_listed) * num_q_heads + 127) / 128 +
+                 static_cast<long long>(num_listed) * num_q_heads) * l.max_ranges;
+  l.bytes = round_up(l.units + static_cast<size_t>(l.max_units) * 32, 256);
   return l;
 }
 
@@ -596,6 +603,8 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
     t.max_ranges = lo.max_ranges;
     t.scale_log2 = l.scale_log2;
     t.unit_start = reinterpret_cast<int*>(ws + lo.unit_start);
+    t.units = reinterpret_cast<int4*>(ws + lo.units);
+    t.max_units = static_cast<int>(std::min<long long>(lo.max_units, 1 << 30));
     t.counters = reinterpret_cast<int*>(ws + lo.counters);
     t.claim = l.pre_blocks;
     t.part_ml = reinterpret_cast<float2*>(ws + lo.part_ml);

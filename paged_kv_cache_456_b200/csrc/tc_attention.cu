@@ -95,6 +95,8 @@ struct TcArgs {
   int oob_row;                      // a row of the cache tensors' 2-D view past their end
   float scale_log2;
   int* unit_start;                  // [rows + 1] work units before each sequence / group
+  int4* units;                      // [max_units][2] one record per work unit (plan kernel)
+  int max_units;
   int* counters;                    // shared: [num_listed * Hq] ranges finished, zero between calls
   int* claim;                       // shared: [num_seqs] blocks attended per sequence
   float2* part_ml;                  // shared: [num_listed * Hq][max_ranges]
@@ -208,12 +210,44 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     if (w < warp) run += s_wsum[w];
     total += s_wsum[w];
   }
+  // each row's units as records {row, kv head, column tile, last key + 1}
+  // {prefill: first query row, rows, context length, 0 | shared: first
+  // member, members, shared blocks, range | ranges << 16}, so that the
+  // attention kernel finds a unit with one load instead of a search
   for (int r = r0; r < r1; ++r) {
     const int units = a.unit_start[r];
     a.unit_start[r] = run;
+    if constexpr (MODE == kModePrefill) {
+      int q0 = 0, Q = 0, n = 0, bit = 0;
+      if (units > 0 && prefill_seq(a, r, &q0, &Q, &n, &bit)) {
+        const int nct = (Q + RPT - 1) / RPT;
+        for (int k = 0; k < units && run + k < a.max_units; ++k) {
+          const int ct = k % nct, kvh = k / nct;
+          const int jl = min(Q, (ct + 1) * RPT) - 1;  // the tile's last query row
+          a.units[2 * (run + k)] = make_int4(r, kvh, ct, n - Q + jl + 1);
+          a.units[2 * (run + k) + 1] = make_int4(q0, Q, n, 0);
+        }
+      }
+    } else {
+      int gs, m, P, leader;
+      if (units > 0 && shared_group(a, r, &gs, &m, &P, &leader)) {
+        const int nct = (m * G + kCols - 1) / kCols;
+        const int Rr = (P + a.range_blocks - 1) / a.range_blocks;
+        for (int k = 0; k < units && run + k < a.max_units; ++k) {
+          const int ct = k % nct, kvh = (k / nct) % Hkv, rr = k / (nct * Hkv);
+          const int k1 = min(P, (rr + 1) * a.range_blocks) * kBlockSize;
+          a.units[2 * (run + k)] = make_int4(leader, kvh, ct, k1);
+          a.units[2 * (run + k) + 1] = make_int4(gs, m, P, rr | (Rr << 16));
+        }
+      }
+    }
     run += units;
   }
-  if (tid == 0) a.unit_start[R] = total;
+  if (tid == 0) {
+    // (the workspace is sized for the most units a call can have)
+    if (total > a.max_units) seterr(a, kErrTimeout);
+    a.unit_start[R] = min(total, a.max_units);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -232,42 +266,32 @@ struct Unit {
   int gs, m, P, r, R;
 };
 
-template <int G, int MODE>
-__device__ __forceinline__ bool decode_unit(const TcArgs& a, int u, Unit* x) {
-  constexpr int RPT = kCols / G;
-  // largest row with unit_start[row] <= u (rows without units share their start)
-  int lo = 0, up = a.rows - 1;
-  while (lo < up) {
-    const int mid = (lo + up + 1) >> 1;
-    if (__ldg(a.unit_start + mid) <= u) lo = mid; else up = mid - 1;
-  }
-  int local = u - __ldg(a.unit_start + lo);
-  const int Hkv = a.num_kv_heads;
+// Work unit u from the plan kernel's records.  The plan kernel writes them
+// while this grid may already be running (programmatic dependent launch), so
+// they are read through L2 (ld.global.cg), never through the non-coherent
+// read-only path: on B200 that path returned a previous call's records when a
+// workspace was reused, and whole units went missing.
+template <int MODE>
+__device__ __forceinline__ void load_unit(const TcArgs& a, int u, Unit* x) {
+  const int4 r0 = __ldcg(a.units + 2 * u), r1 = __ldcg(a.units + 2 * u + 1);
+  x->row = r0.x;
+  x->kvh = r0.y;
+  x->ct = r0.z;
+  x->k1 = r0.w;
   if constexpr (MODE == kModePrefill) {
-    int bit;
-    if (!prefill_seq(a, lo, &x->q0, &x->Q, &x->n, &bit)) return false;
-    const int nct = (x->Q + RPT - 1) / RPT;
-    x->row = lo;
-    x->ct = local % nct;
-    x->kvh = local / nct;
-    const int jl = min(x->Q, (x->ct + 1) * RPT) - 1;  // the tile's last query row
+    x->q0 = r1.x;
+    x->Q = r1.y;
+    x->n = r1.z;
     x->k0 = 0;
-    x->k1 = x->n - x->Q + jl + 1;
   } else {
-    int leader;
-    if (!shared_group(a, lo, &x->gs, &x->m, &x->P, &leader)) return false;
-    const int nct = (x->m * G + kCols - 1) / kCols;
-    x->R = (x->P + a.range_blocks - 1) / a.range_blocks;
-    x->row = leader;
-    x->ct = local % nct;
-    local /= nct;
-    x->kvh = local % Hkv;
-    x->r = local / Hkv;
+    x->gs = r1.x;
+    x->m = r1.y;
+    x->P = r1.z;
+    x->r = r1.w & 0xffff;
+    x->R = r1.w >> 16;
     x->k0 = x->r * a.range_blocks * kBlockSize;
-    x->k1 = min(x->P, (x->r + 1) * a.range_blocks) * kBlockSize;
   }
   x->nt = (x->k1 - x->k0 + kKeys - 1) / kKeys;
-  return x->nt > 0;
 }
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool fill) {
@@ -340,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
 
   // the unit layout comes from the plan kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int total = __ldg(a.unit_start + a.rows);
+  const int total = __ldcg(a.unit_start + a.rows);  // (written by the plan kernel: see load_unit)
 
   auto timeout = [&]() {
     if (atomicExch(&s_abort, 1) == 0) seterr(a, kErrTimeout);
@@ -369,19 +393,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       ++vidx;
       return true;
     };
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      Unit x;
-      if (!decode_unit<G, MODE>(a, u, &x)) continue;
+    Unit x, nx;
+    if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, x = nx) {
+      if (u + static_cast<int>(gridDim.x) < total) load_unit<MODE>(a, u + gridDim.x, &nx);
       const int32_t* trow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
-      for (int j = 0; j < x.nt; ++j) {
-        if (aborted()) { ok = false; break; }
-        // this tile's block rows: lane b < 8 fetches block b's table entry
-        int y = a.oob_row;
+      // block rows of the unit's first tile; then always one tile ahead
+      auto rows_of = [&](int j) -> int {
         const int lb = x.k0 / kBlockSize + j * kTileBlocks + lane;
-        if (lane < kTileBlocks && lb * kBlockSize < x.k1) {
+        int y = a.oob_row;
+        if (lane < kTileBlocks && j < x.nt && lb * kBlockSize < x.k1) {
           const int phys = __ldg(trow + lb);
           if (phys >= 0 && phys < a.num_blocks) y = (phys * Hkv + x.kvh) * kBlockSize;
         }
+        return y;
+      };
+      int ynext = rows_of(0);
+      for (int j = 0; j < x.nt; ++j) {
+        if (aborted()) { ok = false; break; }
+        const int y = ynext;
+        ynext = rows_of(j + 1);
         const int st = kidx % kStages;
         if (kidx >= kStages &&
             !__all_sync(0xffffffffu, mbar_wait_bounded(KEMPTY + 8 * st, ((kidx / kStages) - 1) & 1))) {
@@ -437,9 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         ++sidx;
         return true;
       };
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        Unit x;
-        if (!decode_unit<G, MODE>(a, u, &x)) continue;
+      Unit x, nx;
+      if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, x = nx) {
+        if (u + static_cast<int>(gridDim.x) < total) load_unit<MODE>(a, u + gridDim.x, &nx);
         if (aborted_one() || !mbar_wait_bounded(QFULL, qidx & 1)) { ok = false; break; }
         ++qidx;
         tc::fence_after_sync();
@@ -473,10 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   } else {
     // ---------------- softmax: thread t owns column t ---------------------------
     const int col = tid;
+    const int h = col % G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    int sidx = 0, oidx = 0, qidx = 0, tile = 0, syncs = 0, reds = 0;
+    int sidx = 0, oidx = 0, tile = 0, syncs = 0, reds = 0;
     bool ok = true;
-    // all 128 softmax threads meet (false if the wait ran out)
     // a bounded wait whose outcome the whole warp shares, so that no lane
     // leaves ahead of the others (the TMEM moves are warp-wide)
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
@@ -496,26 +528,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       ++reds;
       return true;
     };
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      Unit x;
-      if (!decode_unit<G, MODE>(a, u, &x)) continue;
-      // ---- this column: query row, head, visible keys
-      const int h = col % G;
-      int qrow = -1, kend = 0;
+    // this column's query row in unit y (-1: none), and the keys it sees
+    auto column_of = [&](const Unit& y, int* kend) -> int {
+      int qrow = -1;
       if constexpr (MODE == kModePrefill) {
-        const int jr = x.ct * RPT + col / G;
-        if (jr < x.Q) {
-          qrow = x.q0 + jr;
-          kend = min(x.k1, x.n - x.Q + jr + 1);
+        const int jr = y.ct * RPT + col / G;
+        *kend = 0;
+        if (jr < y.Q) {
+          qrow = y.q0 + jr;
+          *kend = min(y.k1, y.n - y.Q + jr + 1);
         }
       } else {
-        const int member = x.ct * RPT + col / G;
-        if (member < x.m) {
-          const int seq = a.group_seqs[x.gs + member];
+        const int member = y.ct * RPT + col / G;
+        if (member < y.m) {
+          const int seq = a.group_seqs[y.gs + member];
           if (seq >= 0 && seq < a.num_seqs) qrow = seq;
         }
-        kend = x.k1;
+        *kend = y.k1;
       }
+      return qrow;
+    };
+    // this column's q row into the swizzled Q tile (zeros for no row)
+    auto load_q = [&](const Unit& y, int qrow) {
+      const __nv_bfloat16* src =
+          a.q + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + y.kvh * G + h) * D;
+      const uint32_t qb = smem_addr(sQ) + col * 128;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c)
+        cp_async16_zfill(qb + (c / 8) * (kCols * 128) + (((c % 8) ^ (col % 8)) << 4), src + c * 8,
+                         qrow >= 0);
+    };
+    Unit x, nx;
+    if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
+    bool q_issued = false;  // this unit's Q already requested (during the last unit)
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, x = nx) {
+      const bool has_next = u + static_cast<int>(gridDim.x) < total;
+      if (has_next) load_unit<MODE>(a, u + gridDim.x, &nx);
+      int kend;
+      const int qrow = column_of(x, &kend);
       // ---- the unit's blocks must be in range (prefill: a bad one empties the sequence)
       bool bad = false;
       if constexpr (MODE == kModePrefill) {
@@ -528,52 +578,51 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         if (!group_or(bad, &bad)) { ok = false; break; }
         if (bad && col == 0) seterr(a, kErrBlockId);
       }
-      // ---- q row of this column into the swizzled Q tile
-      {
-        const __nv_bfloat16* src =
-            a.q + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + x.kvh * G + h) * D;
-        const uint32_t qb = smem_addr(sQ) + col * 128;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          cp_async16_zfill(qb + (c / 8) * (kCols * 128) + (((c % 8) ^ (col % 8)) << 4), src + c * 8,
-                           qrow >= 0);
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(QFULL);
-        ++qidx;
-      }
+      // ---- Q: requested now, or already during the previous unit's last tile
+      if (!q_issued) load_q(x, qrow);
+      q_issued = false;
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(QFULL);
+
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < x.nt; ++j, ++tile) {
         if (aborted() || !wait_all(SFULL + 8 * (sidx & 1), (sidx >> 1) & 1)) { ok = false; break; }
         tc::fence_after_sync();
-        float xs[kKeys];
-        {
-          uint32_t r[32];
-#pragma unroll
-          for (int c = 0; c < kKeys / 32; ++c) {
-            tc::tmem_ld32(lane_base + (sidx & 1) * kKeys + c * 32, r);
-            tc::tmem_wait_ld(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) xs[c * 32 + i] = __uint_as_float(r[i]);
-          }
-        }
+        uint32_t sv[kKeys];
+        tc::tmem_ld128(lane_base + (sidx & 1) * kKeys, sv);
+        tc::tmem_wait_ld(sv);
         ++sidx;
-        // scale to log2 units and mask the keys this column does not see
+        if (j == x.nt - 1 && has_next) {
+          // every S of this unit is complete: the Q tile is free for the next unit
+          int kn;
+          load_q(nx, column_of(nx, &kn));
+          q_issued = true;
+        }
+        // scale to log2 units, mask the keys this column does not see, and take
+        // the maximum over 8 independent chains
         const int kb = x.k0 + j * kKeys;
-        float mx = -INFINITY;
+        float m8[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
         if (kb + kKeys <= kend) {
 #pragma unroll
           for (int t = 0; t < kKeys; ++t) {
-            xs[t] *= a.scale_log2;
-            mx = fmaxf(mx, xs[t]);
+            const float v = __uint_as_float(sv[t]) * a.scale_log2;
+            sv[t] = __float_as_uint(v);
+            m8[t & 7] = fmaxf(m8[t & 7], v);
           }
         } else {
 #pragma unroll
           for (int t = 0; t < kKeys; ++t) {
-            xs[t] = kb + t < kend ? xs[t] * a.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, xs[t]);
+            const float v = kb + t < kend ? __uint_as_float(sv[t]) * a.scale_log2 : -INFINITY;
+            sv[t] = __float_as_uint(v);
+            m8[t & 7] = fmaxf(m8[t & 7], v);
           }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         if (j > 0) {
           // O of the previous tile is complete: its P slot is free and O is stable
           if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
@@ -587,32 +636,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           l_run *= al;
           m_run = mx;
         }
-        // O rows are rescaled by the whole warp together (the TMEM moves are
-        // warp-wide); rows that do not grow are multiplied by 1
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tc::tmem_ld32(lane_base + 2 * kKeys + c * 32, r);
-            tc::tmem_wait_ld(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * al);
-            tc::tmem_st32(lane_base + 2 * kKeys + c * 32, r);
-          }
-          tc::tmem_wait_st();
-        }
-        // weights, rounded to bf16 for the product; the sum takes them as rounded
+        // weights, rounded to bf16 for the product; the sum (8 chains) takes
+        // them as rounded
         const bool none = m_run == -INFINITY;
         const uint32_t pb = smem_addr(sP) + col * 128;
+        float l8[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) l8[c] = 0.f;
 #pragma unroll
         for (int c = 0; c < kKeys / 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = none ? 0.f : exp2f(xs[c * 8 + 2 * e] - m_run);
-            const float p1 = none ? 0.f : exp2f(xs[c * 8 + 2 * e + 1] - m_run);
+            const float p0 = none ? 0.f : exp2f(__uint_as_float(sv[c * 8 + 2 * e]) - m_run);
+            const float p1 = none ? 0.f : exp2f(__uint_as_float(sv[c * 8 + 2 * e + 1]) - m_run);
             const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-            l_run += __low2float(pp) + __high2float(pp);
+            l8[2 * e] += __low2float(pp);
+            l8[2 * e + 1] += __high2float(pp);
             w[e] = *reinterpret_cast<const uint32_t*>(&pp);
           }
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
@@ -620,6 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
                        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                        : "memory");
         }
+        l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         if constexpr (MODE == kModePrefill) {
           // rows past the sequence's end in its last block hold stale data: a
           // zero weight times a NaN would still poison O, so they are zeroed
@@ -640,6 +681,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
             }
           }
         }
+        // O rows are rescaled by the whole warp together (the TMEM moves are
+        // warp-wide; rows that do not grow are multiplied by 1), after the S row
+        // is spent and before P is released to the MMA that accumulates onto O
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tc::tmem_ld32(lane_base + 2 * kKeys + c * 32, r);
+            tc::tmem_wait_ld(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * al);
+            tc::tmem_st32(lane_base + 2 * kKeys + c * 32, r);
+          }
+          tc::tmem_wait_st();
+        }
         fence_proxy_async_smem();
         tc::fence_before_sync();
         mbar_arrive(PFULL);
@@ -655,21 +711,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         uint4* dst = reinterpret_cast<uint4*>(
             a.out + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + x.kvh * G + h) * D);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tc::tmem_ld32(lane_base + 2 * kKeys + c * 32, r);
-          tc::tmem_wait_ld(r);
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t ov[64];
+          tc::tmem_ld64(lane_base + 2 * kKeys + hf * 64, ov);
+          tc::tmem_wait_ld(ov);
           if (qrow >= 0) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int c = 0; c < 8; ++c) {
               uint32_t w[4];
 #pragma unroll
               for (int f = 0; f < 4; ++f) {
                 const __nv_bfloat162 pp = __floats2bfloat162_rn(
-                    __uint_as_float(r[e * 8 + 2 * f]) * inv, __uint_as_float(r[e * 8 + 2 * f + 1]) * inv);
+                    __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
                 w[f] = *reinterpret_cast<const uint32_t*>(&pp);
               }
-              dst[c * 4 + e] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[hf * 8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
@@ -681,16 +737,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
                                          a.max_ranges + x.r
                                : 0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tc::tmem_ld32(lane_base + 2 * kKeys + c * 32, r);
-          tc::tmem_wait_ld(r);
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t ov[64];
+          tc::tmem_ld64(lane_base + 2 * kKeys + hf * 64, ov);
+          tc::tmem_wait_ld(ov);
           if (live) {
-            float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + c * 32);
+            float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + hf * 64);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              po[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                  __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+            for (int e = 0; e < 16; ++e)
+              po[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
           }
         }
         if (live) a.part_ml[pi] = make_float2(m_run, l_run);
@@ -759,9 +815,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
             for (int e = 0; e < D / 4; ++e) dst[e] = acc[e];
             a.pre_ml[orow] = make_float2(M, L);
           }
-          // claim each checked member once (its first column's tile, KV head 0);
-          // a sequence claimed twice is given up
-          if (x.kvh == 0 && col < nm && s_ok[col] && (mlo + col) * G >= x.ct * kCols) {
+          // claim each checked member once (KV head 0; a member's columns all
+          // lie in one tile, since 128 is a multiple of G); a sequence claimed
+          // twice is given up
+          if (x.kvh == 0 && col < nm && s_ok[col]) {
             const int seq = s_seq[col];
             if (atomicCAS(a.claim + seq, 0, x.P) != 0) {
               atomicExch(a.claim + seq, -1);
@@ -773,6 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       }
     }
     if (!ok) timeout();
+    asm volatile("cp.async.wait_all;" ::: "memory");  // (a prefetch left in flight by an abort)
   }
 
   // ---- teardown: every role is out of its loop; the MMAs have drained -------
@@ -862,8 +920,23 @@ bool tc_prefill_supported(int head_dim, int group) {
   return pick<kModePrefill>(head_dim, group, &p, &m);
 }
 
-size_t tc_prefill_workspace_bytes(int num_seqs) {
-  return (static_cast<size_t>(num_seqs) + 1) * sizeof(int);
+// Most work units a prefill call can have: each sequence's column tiles,
+// ceil(Q_s * G / 128) <= Q_s * G / 128 + 1, for every KV head.
+static long long prefill_max_units(int num_seqs, int num_query_tokens, int num_q_heads,
+                                   int num_kv_heads) {
+  const long long G = num_q_heads / num_kv_heads;
+  return static_cast<long long>(num_kv_heads) *
+         ((static_cast<long long>(num_query_tokens) * G + kCols - 1) / kCols + num_seqs);
+}
+static size_t prefill_records_offset(int num_seqs) {
+  return ((static_cast<size_t>(num_seqs) + 1) * sizeof(int) + 255) / 256 * 256;
+}
+
+size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_heads,
+                                  int num_kv_heads) {
+  return prefill_records_offset(num_seqs) +
+         static_cast<size_t>(prefill_max_units(num_seqs, num_query_tokens, num_q_heads,
+                                               num_kv_heads)) * 2 * sizeof(int4);
 }
 
 int tc_launch_smem(int head_dim) { return static_cast<int>(tc_smem_bytes(head_dim)); }
@@ -888,6 +961,10 @@ cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_
   a.oob_row = l.num_blocks * l.num_kv_heads * kBlockSize;
   a.scale_log2 = l.scale_log2;
   a.unit_start = static_cast<int*>(l.workspace);
+  a.units = reinterpret_cast<int4*>(static_cast<char*>(l.workspace) +
+                                    prefill_records_offset(l.num_seqs));
+  a.max_units = static_cast<int>(std::min<long long>(
+      prefill_max_units(l.num_seqs, l.num_query_rows, l.num_q_heads, l.num_kv_heads), 1 << 30));
   a.err_flag = l.err_flag;
   a.tm_k = *l.tm_k;
   a.tm_v = *l.tm_v;
@@ -933,6 +1010,8 @@ cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaSt
   while ((l.max_blocks_per_seq + rb - 1) / rb > l.max_ranges) rb += kTileBlocks;
   a.range_blocks = static_cast<int>(rb);
   a.unit_start = l.unit_start;
+  a.units = l.units;
+  a.max_units = l.max_units;
   a.counters = l.counters;
   a.claim = l.claim;
   a.part_ml = l.part_ml;

@@ -52,7 +52,7 @@ def test_dedup_flag_and_its_counters(capsys):
 def test_default_run_times_the_four_large_workloads_headline_first():
     args = bench.parse_args([])
     names = bench.workload_names(args)
-    assert names == ("long", "7b", "gqa70b", "prefix_cow")
+    assert names == ("long", "7b", "gqa70b", "prefix_cow", "prefill")
     # the headline is the largest step by algorithmic bytes
     sizes = {n: bench.step_bytes(build_workload(n), fused=True) for n in ("long", "7b")}
     assert sizes["long"] > 2 * sizes["7b"]

@@ -99,6 +99,34 @@ def test_repeat_calls_are_bit_identical():
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
+def test_workspace_reused_by_different_calls():
+    """Calls with different work on one workspace: each call's unit layout is
+    written by its own plan kernel, and no call may see the previous call's
+    (a stale layout once dropped whole units here)."""
+    cases = [prefill_case(80 + i, dtype="bf16", num_q_heads=32, num_kv_heads=4, head_dim=128,
+                          lens=lens, queries=qs)
+             for i, (lens, qs) in enumerate([((1500, 900, 1200, 2000), (64, 64, 64, 64)),
+                                             ((700, 300, 129), (200, 100, 129)),
+                                             ((1500, 900, 1200, 2000), (64, 64, 64, 64))])]
+    big = max(ops.make_prefill_workspace(w.num_seqs, q.shape[0], w.num_q_heads, w.num_kv_heads,
+                                         w.head_dim, w.max_context_len, 0, torch.bfloat16).numel()
+              for w, q, _ in cases)
+    ws = torch.zeros(big, dtype=torch.uint8, device="cuda")
+    for w, q, qs in cases * 2:
+        t = upload(w)
+        qd = torch.from_numpy(np.ascontiguousarray(q)).view(torch.bfloat16).cuda()
+        out = torch.full(qd.shape, 7.0, dtype=torch.bfloat16, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ops.prefill(out, qd, t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                    torch.from_numpy(qs).cuda(), scale=w.scale, max_context_len=w.max_context_len,
+                    workspace=ws, err_flag=err)
+        torch.cuda.synchronize()
+        ref, _ = oracle.paged_prefill(q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens, qs,
+                                      scale=w.scale, dtype=w.dtype)
+        assert err.item() == 0
+        assert_attention_close(out, ref, "bf16", "reused workspace")
+
+
 def test_bad_block_zeroes_that_sequence_only():
     w, q, qs = prefill_case(78, dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=128,
                             lens=(200, 150, 90), queries=(20, 30, 10))
