@@ -191,7 +191,7 @@ bool tc_prefill_supported(int head_dim, int group);
 size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_heads,
                                   int num_kv_heads);
 int tc_launch_smem(int head_dim);
-constexpr int kTcWarps = 6;
+constexpr int kTcWarps = 10;
 cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_t stream);
 
 // The shared-prefix pass on the tcgen05 tensor cores: (member, query head)

@@ -67,10 +67,10 @@ constexpr int kCols = 128;                      // M: query columns of a tile
 constexpr int kKeys = 128;                      // N: keys of a K/V tile
 constexpr int kTileBlocks = kKeys / kBlockSize; // 8 blocks per K/V tile
 constexpr int kStages = 2;                      // slots of the K ring and of the V ring
-constexpr int kSoftmaxThreads = 128;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 256;            // two per column: keys 0-63 / 64-127
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;                  // S[2] at columns 0 / 128, O at 256
 constexpr int kPlanThreads = 1024;
 constexpr int kModePrefill = 0;
@@ -294,6 +294,15 @@ __device__ __forceinline__ void load_unit(const TcArgs& a, int u, Unit* x) {
   x->nt = (x->k1 - x->k0 + kKeys - 1) / kKeys;
 }
 
+// 2^x by the ex2.approx.ftz.f32 instruction.  Results below the smallest
+// normal float flush to zero; the weights it makes are rounded to bf16 and
+// are at most 2^8, so nothing of them is lost that the sum could see.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool fill) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
                "r"(fill ? 16 : 0)
@@ -328,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_red[3];
+  __shared__ float s_xch[2][2][kCols];  // per half: row maxima of a tile / row sums of a unit
   // shared mode: the fold's member checks
   __shared__ int s_seq[kCols];
   __shared__ unsigned char s_ok[kCols];
@@ -503,11 +513,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     }
     __syncwarp();
   } else {
-    // ---------------- softmax: thread t owns column t ---------------------------
-    const int col = tid;
+    // ---------------- softmax: two threads per column -----------------------------
+    // Thread t (0..255) serves column col = t % 128, which is TMEM lane col
+    // (warps w and w + 4 share a lane quarter), and half hf = t / 128 of it:
+    // keys 64 hf .. 64 hf + 63 of every tile, head_dim D/2 hf .. D/2 hf + D/2 - 1
+    // of O, and its own share of the row sum.  The two threads of a column
+    // swap their partial row maxima once per tile and their sums once per unit.
+    const int col = tid % kCols, hf = tid / kCols;
     const int h = col % G;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    int sidx = 0, oidx = 0, tile = 0, syncs = 0, reds = 0;
+    constexpr int HK = kKeys / 2;   // keys per thread and tile
+    constexpr int HD = D / 2;       // O columns per thread
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    int sidx = 0, oidx = 0, tile = 0, syncs = 0, reds = 0, xs = 0;
     bool ok = true;
     // a bounded wait whose outcome the whole warp shares, so that no lane
     // leaves ahead of the others (the TMEM moves are warp-wide)
@@ -518,14 +535,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       mbar_arrive(SYNC);
       return wait_all(SYNC, (syncs++) & 1);
     };
-    // OR of a flag over the 128 threads; slot reds % 3 is cleared two uses ahead
+    // OR of a flag over the softmax threads; slot reds % 3 is cleared two uses ahead
     auto group_or = [&](bool v, bool* res) -> bool {
       const int slot = reds % 3;
       if (v) atomicOr(&s_red[slot], 1);
       if (!group_sync()) return false;
       *res = *reinterpret_cast<volatile int*>(&s_red[slot]) != 0;
-      if (col == 0) s_red[(reds + 2) % 3] = 0;
+      if (tid == 0) s_red[(reds + 2) % 3] = 0;
       ++reds;
+      return true;
+    };
+    // the other half's value of this column (the exchange slot alternates, so
+    // that one sync per exchange suffices)
+    auto swap_half = [&](float v, float* other) -> bool {
+      const int sl = (xs++) & 1;
+      s_xch[sl][hf][col] = v;
+      if (!group_sync()) return false;
+      *other = s_xch[sl][hf ^ 1][col];
       return true;
     };
     // this column's query row in unit y (-1: none), and the keys it sees
@@ -548,15 +574,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       }
       return qrow;
     };
-    // this column's q row into the swizzled Q tile (zeros for no row)
+    // this thread's half of its column's q row into the swizzled Q tile
+    // (zeros for no row)
     auto load_q = [&](const Unit& y, int qrow) {
       const __nv_bfloat16* src =
           a.q + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + y.kvh * G + h) * D;
       const uint32_t qb = smem_addr(sQ) + col * 128;
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c)
+      for (int cc = 0; cc < D / 16; ++cc) {
+        const int c = hf * (D / 16) + cc;  // 16-byte chunk of the row
         cp_async16_zfill(qb + (c / 8) * (kCols * 128) + (((c % 8) ^ (col % 8)) << 4), src + c * 8,
                          qrow >= 0);
+      }
     };
     Unit x, nx;
     if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
@@ -571,12 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       if constexpr (MODE == kModePrefill) {
         const int nb = (x.n + kBlockSize - 1) / kBlockSize;
         const int32_t* trow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
-        for (int b = col; b < nb; b += kSoftmaxThreads) {
+        for (int b = tid; b < nb; b += kSoftmaxThreads) {
           const int phys = __ldg(trow + b);
           bad |= !(phys >= 0 && phys < a.num_blocks);
         }
         if (!group_or(bad, &bad)) { ok = false; break; }
-        if (bad && col == 0) seterr(a, kErrBlockId);
+        if (bad && tid == 0) seterr(a, kErrBlockId);
       }
       // ---- Q: requested now, or already during the previous unit's last tile
       if (!q_issued) load_q(x, qrow);
@@ -590,8 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       for (int j = 0; j < x.nt; ++j, ++tile) {
         if (aborted() || !wait_all(SFULL + 8 * (sidx & 1), (sidx >> 1) & 1)) { ok = false; break; }
         tc::fence_after_sync();
-        uint32_t sv[kKeys];
-        tc::tmem_ld128(lane_base + (sidx & 1) * kKeys, sv);
+        uint32_t sv[HK];
+        tc::tmem_ld64(lane_base + (sidx & 1) * kKeys + hf * HK, sv);
         tc::tmem_wait_ld(sv);
         ++sidx;
         if (j == x.nt - 1 && has_next) {
@@ -601,28 +630,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           q_issued = true;
         }
         // scale to log2 units, mask the keys this column does not see, and take
-        // the maximum over 8 independent chains
-        const int kb = x.k0 + j * kKeys;
+        // the maximum over 8 independent chains, then with the other half's
+        const int kb = x.k0 + j * kKeys + hf * HK;
         float m8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
-        if (kb + kKeys <= kend) {
+        if (kb + HK <= kend) {
 #pragma unroll
-          for (int t = 0; t < kKeys; ++t) {
+          for (int t = 0; t < HK; ++t) {
             const float v = __uint_as_float(sv[t]) * a.scale_log2;
             sv[t] = __float_as_uint(v);
             m8[t & 7] = fmaxf(m8[t & 7], v);
           }
         } else {
 #pragma unroll
-          for (int t = 0; t < kKeys; ++t) {
+          for (int t = 0; t < HK; ++t) {
             const float v = kb + t < kend ? __uint_as_float(sv[t]) * a.scale_log2 : -INFINITY;
             sv[t] = __float_as_uint(v);
             m8[t & 7] = fmaxf(m8[t & 7], v);
           }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        {
+          float mo;
+          if (!swap_half(mx, &mo)) { ok = false; break; }
+          mx = fmaxf(mx, mo);  // (both halves now hold the same tile maximum)
+        }
         if (j > 0) {
           // O of the previous tile is complete: its P slot is free and O is stable
           if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
@@ -632,31 +666,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         const bool grow = mx > m_run + kRescaleThreshold;
         float al = 1.f;
         if (grow) {
-          al = exp2f(m_run - mx);  // (0 while nothing was seen)
+          al = ex2_fast(m_run - mx);  // (0 while nothing was seen)
           l_run *= al;
           m_run = mx;
         }
         // weights, rounded to bf16 for the product; the sum (8 chains) takes
-        // them as rounded
+        // them as rounded; this half's 64 keys are P's K-block hf
         const bool none = m_run == -INFINITY;
-        const uint32_t pb = smem_addr(sP) + col * 128;
+        const uint32_t pb = smem_addr(sP) + hf * (kCols * 128) + col * 128;
         float l8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) l8[c] = 0.f;
 #pragma unroll
-        for (int c = 0; c < kKeys / 8; ++c) {
+        for (int c = 0; c < HK / 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = none ? 0.f : exp2f(__uint_as_float(sv[c * 8 + 2 * e]) - m_run);
-            const float p1 = none ? 0.f : exp2f(__uint_as_float(sv[c * 8 + 2 * e + 1]) - m_run);
+            const float p0 = none ? 0.f : ex2_fast(__uint_as_float(sv[c * 8 + 2 * e]) - m_run);
+            const float p1 = none ? 0.f : ex2_fast(__uint_as_float(sv[c * 8 + 2 * e + 1]) - m_run);
             const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
             l8[2 * e] += __low2float(pp);
             l8[2 * e + 1] += __high2float(pp);
             w[e] = *reinterpret_cast<const uint32_t*>(&pp);
           }
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                           pb + (c / 8) * (kCols * 128) + (((c % 8) ^ (col % 8)) << 4)),
+                           pb + (((c % 8) ^ (col % 8)) << 4)),
                        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                        : "memory");
         }
@@ -665,14 +699,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           // rows past the sequence's end in its last block hold stale data: a
           // zero weight times a NaN would still poison O, so they are zeroed
           const int tail = x.n % kBlockSize;
-          const int lastb = x.n / kBlockSize;  // logical block holding them
-          if (tail && lastb * kBlockSize >= kb && lastb * kBlockSize < kb + kKeys) {
+          const int lastb = x.n / kBlockSize;        // logical block holding them
+          const int kt = x.k0 + j * kKeys;           // the tile's first key
+          if (tail && lastb * kBlockSize >= kt && lastb * kBlockSize < kt + kKeys) {
             const int st = tile % kStages;
             if (!wait_all(VFULL + 8 * st, (tile / kStages) & 1)) { ok = false; break; }
-            const int b = (lastb * kBlockSize - kb) / kBlockSize;
+            const int b = (lastb * kBlockSize - kt) / kBlockSize;
             unsigned char* vt = sV + st * KT;
             const int nz = (kBlockSize - tail) * 8 * KB;  // 16-byte chunks to clear
-            for (int i = col; i < nz; i += kSoftmaxThreads) {
+            for (int i = tid; i < nz; i += kSoftmaxThreads) {
               const int hx = i / ((kBlockSize - tail) * 8);
               const int rem = i % ((kBlockSize - tail) * 8);
               const int row = b * kBlockSize + tail + rem / 8;
@@ -681,18 +716,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
             }
           }
         }
-        // O rows are rescaled by the whole warp together (the TMEM moves are
-        // warp-wide; rows that do not grow are multiplied by 1), after the S row
-        // is spent and before P is released to the MMA that accumulates onto O
+        // this half of the O row is rescaled by the whole warp together (the
+        // TMEM moves are warp-wide; rows that do not grow are multiplied by 1),
+        // after the S row is spent and before P is released to the MMA
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < HD / 32; ++c) {
             uint32_t r[32];
-            tc::tmem_ld32(lane_base + 2 * kKeys + c * 32, r);
+            tc::tmem_ld32(lane_base + 2 * kKeys + hf * HD + c * 32, r);
             tc::tmem_wait_ld(r);
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * al);
-            tc::tmem_st32(lane_base + 2 * kKeys + c * 32, r);
+            tc::tmem_st32(lane_base + 2 * kKeys + hf * HD + c * 32, r);
           }
           tc::tmem_wait_st();
         }
@@ -701,32 +736,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         mbar_arrive(PFULL);
       }
       if (!ok) break;
-      // ---- the unit's O row
+      // ---- the unit's O row: this thread's half, over the column's whole sum
       if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
       ++oidx;
       tc::fence_after_sync();
+      float lo;
+      if (!swap_half(l_run, &lo)) { ok = false; break; }
+      const float l_all = l_run + lo;
+      uint32_t ov[HD];
+      if constexpr (HD == 64) tc::tmem_ld64(lane_base + 2 * kKeys + hf * HD, ov);
+      else tc::tmem_ld32(lane_base + 2 * kKeys + hf * HD, ov);
+      tc::tmem_wait_ld(ov);
       if constexpr (MODE == kModePrefill) {
-        // (every lane runs the warp-wide TMEM loads; only live columns store)
-        const float inv = bad ? 0.f : 1.f / l_run;
-        uint4* dst = reinterpret_cast<uint4*>(
-            a.out + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + x.kvh * G + h) * D);
+        // (every lane ran the warp-wide TMEM load; only live columns store)
+        if (qrow >= 0) {
+          const float inv = bad ? 0.f : 1.f / l_all;
+          uint4* dst = reinterpret_cast<uint4*>(
+              a.out + (static_cast<size_t>(qrow) * Hq + x.kvh * G + h) * D + hf * HD);
 #pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-          uint32_t ov[64];
-          tc::tmem_ld64(lane_base + 2 * kKeys + hf * 64, ov);
-          tc::tmem_wait_ld(ov);
-          if (qrow >= 0) {
+          for (int c = 0; c < HD / 8; ++c) {
+            uint32_t w[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint32_t w[4];
-#pragma unroll
-              for (int f = 0; f < 4; ++f) {
-                const __nv_bfloat162 pp = __floats2bfloat162_rn(
-                    __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
-                w[f] = *reinterpret_cast<const uint32_t*>(&pp);
-              }
-              dst[hf * 8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int f = 0; f < 4; ++f) {
+              const __nv_bfloat162 pp = __floats2bfloat162_rn(
+                  __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
+              w[f] = *reinterpret_cast<const uint32_t*>(&pp);
             }
+            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       } else {
@@ -736,23 +772,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         const size_t pi = live ? (static_cast<size_t>(x.gs + member) * Hq + x.kvh * G + h) *
                                          a.max_ranges + x.r
                                : 0;
+        if (live) {
+          float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + hf * HD);
 #pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-          uint32_t ov[64];
-          tc::tmem_ld64(lane_base + 2 * kKeys + hf * 64, ov);
-          tc::tmem_wait_ld(ov);
-          if (live) {
-            float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + hf * 64);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              po[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
-                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
-          }
+          for (int e = 0; e < HD / 4; ++e)
+            po[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+          if (hf == 0) a.part_ml[pi] = make_float2(m_run, l_all);
         }
-        if (live) a.part_ml[pi] = make_float2(m_run, l_run);
         __threadfence();
         if (!group_sync()) { ok = false; break; }
-        if (col == 0) {
+        if (tid == 0) {
           int* cnt = a.counters + (static_cast<size_t>(x.gs) * G + x.ct * kCols) * Hkv + x.kvh;
           const int prev = atomicAdd(cnt, 1);
           s_last = prev == x.R - 1;
@@ -764,19 +794,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           const int mlo = x.ct * RPT;
           const int nm = min(x.m - mlo, RPT);  // members of this tile
           const int32_t* lrow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
-          if (col < nm) {
-            const int seq = a.group_seqs[x.gs + mlo + col];
+          if (tid < nm) {
+            const int seq = a.group_seqs[x.gs + mlo + tid];
             bool okm = seq >= 0 && seq < a.num_seqs;
             if (okm) {
               const int n = a.context_lens[seq];
               okm = n > 0 && n <= a.len_cap && kBlockSize * x.P <= n - 1;
             }
-            s_seq[col] = okm ? seq : -1;
-            s_ok[col] = okm;
+            s_seq[tid] = okm ? seq : -1;
+            s_ok[tid] = okm;
           }
           if (!group_sync()) { ok = false; break; }
           // every (member, shared block): the member's table holds the leader's block
-          for (int idx = col; idx < nm * x.P; idx += kSoftmaxThreads) {
+          for (int idx = tid; idx < nm * x.P; idx += kSoftmaxThreads) {
             const int i = idx / x.P, jb = idx - i * x.P;
             const int seq = s_seq[i];
             if (seq < 0) continue;
@@ -786,40 +816,48 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
               s_ok[i] = 0;  // (every writer stores the same value)
           }
           if (!group_sync()) { ok = false; break; }
-          if (x.kvh == 0 && col < nm && !s_ok[col]) seterr(a, kErrGroup);
+          if (x.kvh == 0 && tid < nm && !s_ok[tid]) seterr(a, kErrGroup);
           if (live && s_ok[col / G]) {
+            // this thread folds its half of the column's head_dim
             const size_t pb0 = (static_cast<size_t>(x.gs + member) * Hq + x.kvh * G + h) * a.max_ranges;
             float M = -INFINITY;
             for (int rr = 0; rr < x.R; ++rr) M = fmaxf(M, __ldcg(a.part_ml + pb0 + rr).x);
-            float L = 0.f;
-            float4 acc[D / 4];
-#pragma unroll
-            for (int e = 0; e < D / 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int rr = 0; rr < x.R; ++rr) {
-              const float2 ml = __ldcg(a.part_ml + pb0 + rr);
-              const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-              L += w * ml.y;
-              const float4* po = reinterpret_cast<const float4*>(a.part_o + (pb0 + rr) * D);
-#pragma unroll
-              for (int e = 0; e < D / 4; ++e) {
-                const float4 o4 = __ldcg(po + e);
-                acc[e].x = fmaf(w, o4.x, acc[e].x);
-                acc[e].y = fmaf(w, o4.y, acc[e].y);
-                acc[e].z = fmaf(w, o4.z, acc[e].z);
-                acc[e].w = fmaf(w, o4.w, acc[e].w);
-              }
-            }
             const size_t orow = static_cast<size_t>(s_seq[col / G]) * Hq + x.kvh * G + h;
-            float4* dst = reinterpret_cast<float4*>(a.pre_o + orow * D);
+            // (in passes of 32 dims, to keep the accumulators in registers)
+            constexpr int QD = HD < 32 ? HD : 32;
+            float L = 0.f;
+#pragma unroll 1
+            for (int q0 = 0; q0 < HD; q0 += QD) {
+              float4 acc[QD / 4];
 #pragma unroll
-            for (int e = 0; e < D / 4; ++e) dst[e] = acc[e];
-            a.pre_ml[orow] = make_float2(M, L);
+              for (int e = 0; e < QD / 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+              L = 0.f;
+              for (int rr = 0; rr < x.R; ++rr) {
+                const float2 ml = __ldcg(a.part_ml + pb0 + rr);
+                const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+                L += w * ml.y;
+                const float4* po =
+                    reinterpret_cast<const float4*>(a.part_o + (pb0 + rr) * D + hf * HD + q0);
+#pragma unroll
+                for (int e = 0; e < QD / 4; ++e) {
+                  const float4 o4 = __ldcg(po + e);
+                  acc[e].x = fmaf(w, o4.x, acc[e].x);
+                  acc[e].y = fmaf(w, o4.y, acc[e].y);
+                  acc[e].z = fmaf(w, o4.z, acc[e].z);
+                  acc[e].w = fmaf(w, o4.w, acc[e].w);
+                }
+              }
+              float4* dst = reinterpret_cast<float4*>(a.pre_o + orow * D + hf * HD + q0);
+#pragma unroll
+              for (int e = 0; e < QD / 4; ++e) dst[e] = acc[e];
+            }
+            if (hf == 0) a.pre_ml[orow] = make_float2(M, L);
           }
           // claim each checked member once (KV head 0; a member's columns all
           // lie in one tile, since 128 is a multiple of G); a sequence claimed
           // twice is given up
-          if (x.kvh == 0 && col < nm && s_ok[col]) {
-            const int seq = s_seq[col];
+          if (x.kvh == 0 && tid < nm && s_ok[tid]) {
+            const int seq = s_seq[tid];
             if (atomicCAS(a.claim + seq, 0, x.P) != 0) {
               atomicExch(a.claim + seq, -1);
               seterr(a, kErrGroup);
