@@ -309,7 +309,8 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
  * checks both on the device; a member that fails, or a sequence that two
  * groups list, is attended in full by the decode kernel and PA_ERRBIT_GROUP
  * is set.  A sequence in no group is attended as by pa_decode.
- * num_listed = group_start[num_groups]; num_groups <= 16384.
+ * num_listed = group_start[num_groups]; num_groups <= 16384
+ * (PA_ERR_UNSUPPORTED above) and num_groups <= num_listed (PA_ERR_INVALID_ARG).
  *
  * pa_shared_prefix_plan finds such groups on the HOST (its pointers are
  * host pointers, unlike every other entry point's): sequences whose first

@@ -289,10 +289,12 @@ static int prefill_items(int num_seqs, int num_query_tokens, int num_q_heads, in
 #ifndef PA_PREFILL_TC
 #define PA_PREFILL_TC 1
 #endif
-static bool prefill_on_tensor_cores(int num_q_heads, int num_kv_heads, int head_dim,
-                                    pa_dtype dtype) {
+// (the tensor-core kernel numbers its pairs of 128-column tiles in 16 bits)
+static bool prefill_on_tensor_cores(int num_query_tokens, int num_q_heads, int num_kv_heads,
+                                    int head_dim, pa_dtype dtype) {
   return PA_PREFILL_TC && dtype == PA_BF16 && num_kv_heads > 0 && num_q_heads > 0 &&
          num_q_heads % num_kv_heads == 0 &&
+         static_cast<long long>(num_query_tokens) * (num_q_heads / num_kv_heads) < (1LL << 24) &&
          pa::tc_prefill_supported(head_dim, num_q_heads / num_kv_heads);
 }
 
@@ -300,7 +302,7 @@ pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_
                                     int num_kv_heads, int head_dim, int max_context_len,
                                     int partition_size, pa_dtype dtype, size_t* bytes) {
   if (!bytes || num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
-  if (prefill_on_tensor_cores(num_q_heads, num_kv_heads, head_dim, dtype)) {
+  if (prefill_on_tensor_cores(num_query_tokens, num_q_heads, num_kv_heads, head_dim, dtype)) {
     const pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
                                             max_context_len, partition_size, dtype);
     if (st != PA_OK) return st;
@@ -347,7 +349,7 @@ pa_status pa_prefill_launch_config(int num_seqs, int num_query_tokens, int num_q
                                    int partition_size, pa_dtype dtype, int* grid,
                                    int* warps_per_cta, int* pipeline_depth, int* smem_bytes) {
   if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
-  if (prefill_on_tensor_cores(num_q_heads, num_kv_heads, head_dim, dtype)) {
+  if (prefill_on_tensor_cores(num_query_tokens, num_q_heads, num_kv_heads, head_dim, dtype)) {
     pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
                                       max_context_len, partition_size, dtype);
     if (st != PA_OK) return st;
@@ -355,7 +357,7 @@ pa_status pa_prefill_launch_config(int num_seqs, int num_query_tokens, int num_q
     if ((st = device_info(&dev)) != PA_OK) return st;
     if (grid) *grid = dev.sms;
     if (warps_per_cta) *warps_per_cta = pa::kTcWarps;
-    if (pipeline_depth) *pipeline_depth = 2;
+    if (pipeline_depth) *pipeline_depth = 3;
     if (smem_bytes) *smem_bytes = pa::tc_launch_smem(head_dim);
     return PA_OK;
   }
@@ -514,7 +516,7 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
   if (num_seqs < 0 || num_query_tokens < 0) return PA_ERR_INVALID_ARG;
   if (num_query_tokens == 0) return PA_OK;
   if (num_seqs == 0 || !query_start) return PA_ERR_INVALID_ARG;
-  if (prefill_on_tensor_cores(num_q_heads, num_kv_heads, head_dim, dtype)) {
+  if (prefill_on_tensor_cores(num_query_tokens, num_q_heads, num_kv_heads, head_dim, dtype)) {
     pa_status st = check_decode_shape(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
                                       max_context_len, partition_size, dtype);
     if (st != PA_OK) return st;
@@ -615,6 +617,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, con
   if (num_groups > 0 && (!group_seqs || !group_start || !group_blocks || num_listed == 0))
     return PA_ERR_INVALID_ARG;
   if (num_groups > 16384) return PA_ERR_UNSUPPORTED;  // (the pass keeps one int per group on chip)
+  if (num_groups > num_listed) return PA_ERR_INVALID_ARG;  // (a group lists one member at least)
   if (key && (!aligned16(key) || !aligned16(value))) return PA_ERR_INVALID_ARG;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return PA_ERR_INVALID_ARG;

@@ -217,7 +217,7 @@ struct TcSharedLaunch {
   int* unit_start;     // [num_groups + 1]
   int4* units;         // [max_units][2] work-unit records
   int max_units;
-  int* counters;       // [num_listed * Hq], zero between calls
+  int* group_ranges;   // [num_groups] ranges of each group's shared blocks (plan kernel)
   int* claim;          // [num_seqs], zeroed before the pass
   float2* part_ml;
   float* part_o;

@@ -14,11 +14,13 @@
 // sets is the log-sum-exp combination of the parts, so the result is the
 // same attention up to rounding.
 //
-// Work: a unit is (group, chunk of 64 columns, kv head, range of shared
-// blocks); the host picks the range length so that the units fill the
-// resident CTAs.  Each unit writes a partial state per column;
+// The pass runs on the tcgen05 tensor cores (tc_attention.cu: units of 128
+// columns, a separate fold kernel).  The warp-level MMA pass below is kept
+// as a build option.  Its work: a unit is (group, chunk of 64 columns, kv
+// head, range of shared blocks); the host picks the range length so that the
+// units fill the resident CTAs.  Each unit writes a partial state per column;
 // the last unit of a (group, chunk, kv head) to finish folds the ranges and
-// stores the state per (sequence, head).  Members are checked against the
+// stores the state per (sequence, head).  Either way members are checked against the
 // block tables before their state is published: a member whose table does
 // not hold the group's blocks, whose length leaves no token after them, or
 // that two groups list, is not claimed (PA_ERRBIT_GROUP) and the decode
@@ -505,7 +507,7 @@ int min_range_tiles(int max_blocks_per_seq, int head_dim) {
 }
 
 struct Layout {
-  size_t counters, claim, part_ml, part_o, pre_ml, pre_o, unit_start, units, bytes;
+  size_t counters, claim, part_ml, part_o, pre_ml, pre_o, unit_start, group_ranges, units, bytes;
   int max_ranges;
   long long max_units;
 };
@@ -523,15 +525,18 @@ Layout layout(int num_seqs, int num_listed, int num_q_heads, int head_dim,
   l.part_o = round_up(l.part_ml + cols * l.max_ranges * sizeof(float2), 256);
   l.pre_ml = round_up(l.part_o + cols * l.max_ranges * head_dim * sizeof(float), 256);
   l.pre_o = round_up(l.pre_ml + rows * sizeof(float2), 256);
-  // (the tensor-core pass: work units before each group; groups <= sequences)
+  // (the tensor-core pass: work units before each group and each group's
+  // ranges; a group lists at least one member, so groups <= listed)
   l.unit_start = round_up(l.pre_o + rows * head_dim * sizeof(float), 256);
+  l.group_ranges = round_up(l.unit_start + (static_cast<size_t>(num_listed) + 1) * sizeof(int), 256);
   // its unit records: per group ceil(members * G / 128) <= members * G / 128 + 1
   // column tiles for each KV head and range, so at most
   // (ceil(listed * Hq / 128) + listed * Hq) x max_ranges in all
-  l.units = round_up(l.unit_start + (static_cast<size_t>(num_seqs) + 1) * sizeof(int), 256);
+  l.units = round_up(l.group_ranges + static_cast<size_t>(num_listed) * sizeof(int), 256);
   l.max_units = ((static_cast<long long>(num_listed) * num_q_heads + 127) / 128 +
                  static_cast<long long>(num_listed) * num_q_heads) * l.max_ranges;
-  l.bytes = round_up(l.units + static_cast<size_t>(l.max_units) * 32, 256);
+  // (the records twice: sorted, and in group order)
+  l.bytes = round_up(l.units + static_cast<size_t>(l.max_units) * 64, 256);
   return l;
 }
 
@@ -604,8 +609,8 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
     t.scale_log2 = l.scale_log2;
     t.unit_start = reinterpret_cast<int*>(ws + lo.unit_start);
     t.units = reinterpret_cast<int4*>(ws + lo.units);
-    t.max_units = static_cast<int>(std::min<long long>(lo.max_units, 1 << 30));
-    t.counters = reinterpret_cast<int*>(ws + lo.counters);
+    t.max_units = static_cast<int>(std::min<long long>(lo.max_units, 1 << 28));
+    t.group_ranges = reinterpret_cast<int*>(ws + lo.group_ranges);
     t.claim = l.pre_blocks;
     t.part_ml = reinterpret_cast<float2*>(ws + lo.part_ml);
     t.part_o = reinterpret_cast<float*>(ws + lo.part_o);

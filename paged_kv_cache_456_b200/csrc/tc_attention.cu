@@ -10,42 +10,46 @@
 // section "Idea 1: PagedAttention").  Here a column is one (query row, query
 // head) pair of one KV head, and 128 of them form the M side of the MMAs:
 //
-//   S[128 columns x 128 keys]  = Q[128 x D] . K[128 keys x D]^T   (TMEM, fp32)
+//   S[128 columns x 64 keys]  = Q[128 x D] . K[64 keys x D]^T    (TMEM, fp32)
 //   P = exp2(S * scale * log2 e - m)  (one thread per column, bf16, to smem)
-//   O[128 columns x D]        += P[128 x 128 keys] . V[128 keys x D]  (TMEM)
+//   O[128 columns x D]       += P[128 x 64 keys] . V[64 keys x D]  (TMEM)
 //
 // with the online softmax of the decode kernels (running max m in log2 units,
 // rescaled only when it grows by more than 2^8; the sum l takes the weights
-// as rounded for the product).  The keys of a tile are 8 blocks of 16 tokens,
+// as rounded for the product).  The keys of a tile are 4 blocks of 16 tokens,
 // each fetched by 2-D tensor loads (16 rows x 64 elements, 128-byte swizzle)
 // through the block table; a block past the range is loaded from outside the
 // tensor, which fills it with zeros.
 //
-// CTA roles (192 threads, one CTA per SM, persistent over the work units):
-//   warps 0-3  softmax: thread t owns column t (TMEM lane t): loads its q row,
+// A CTA works on two column tiles (A and B) of the same work at once, which
+// share every K/V tile, so that one tile's softmax overlaps the other's
+// MMAs and waits.  CTA roles (320 threads, one CTA per SM, persistent over
+// the work units):
+//   warps 0-3  softmax of tile A, warps 4-7 of tile B: thread t of a
+//              warpgroup owns column t (TMEM lane t): loads its q row,
 //              reads its row of S, writes its row of P, rescales and finally
 //              reads its row of O -- no cross-thread reduction anywhere;
-//   warp 4     producer: K and V tiles into two 2-slot rings (K runs one tile
+//   warp 8     producer: K and V tiles into two 3-slot rings (K runs one tile
 //              ahead of V, so each wait is in the order the slots free up);
-//   warp 5     MMA issuer (one thread) and TMEM owner (512 columns: two S
-//              buffers so that S of tile j+1 is computed while the softmax
-//              works on tile j, and O).
+//   warp 9     MMA issuer (one thread) and TMEM owner (512 columns: two S
+//              buffers per tile, so that S of tile j+2 is computed while the
+//              softmax works on tile j, and O of each tile).
 // Every mbarrier wait is bounded; a wait that runs out sets PA_ERRBIT_TIMEOUT,
 // and every role then leaves its loop; the TMEM is freed on every exit path
 // once the MMAs issued so far have completed.
 //
 // Work units:
-//   prefill  (sequence, KV head, column tile): a tile is 128/G consecutive
-//            query rows x G heads; keys 0 .. the tile's last row's position;
-//            the normalised output is stored.
-//   shared   (group, range of shared blocks, KV head, column tile): a tile
-//            is 128/G members x G heads; the range's partial state is stored
-//            and the last range of a (group, tile, KV head) to finish folds
-//            them by log-sum-exp into the state the decode kernel continues
-//            from (after checking each member's table, as the other pass did).
-// A one-CTA plan kernel lays the units out (prefix sums over sequences or
-// groups) in the workspace first; the attention kernel is launched behind it
-// with programmatic dependent launch.
+//   prefill  (sequence, KV head, pair of column tiles): a tile is 128/G
+//            consecutive query rows x G heads; keys 0 .. the position of the
+//            pair's last row; the normalised output is stored.
+//   shared   (group, range of shared blocks, KV head, pair of column tiles):
+//            a tile is 128/G members x G heads; the range's partial state is
+//            stored, and a fold kernel launched behind the pass combines the
+//            ranges by log-sum-exp into the state the decode kernel
+//            continues from (after checking each member's table).
+// A one-CTA plan kernel writes the units' records into the workspace first;
+// the attention kernel (and the fold kernel behind it) are launched with
+// programmatic dependent launch.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -64,15 +68,20 @@ namespace pa {
 namespace {
 
 constexpr int kCols = 128;                      // M: query columns of a tile
-constexpr int kKeys = 128;                      // N: keys of a K/V tile
-constexpr int kTileBlocks = kKeys / kBlockSize; // 8 blocks per K/V tile
-constexpr int kStages = 2;                      // slots of the K ring and of the V ring
-constexpr int kSoftmaxThreads = 256;            // two per column: keys 0-63 / 64-127
+constexpr int kPair = 2;                        // column tiles a CTA works on together
+constexpr int kKeys = 64;                       // N: keys of a K/V tile
+constexpr int kTileBlocks = kKeys / kBlockSize; // 4 blocks per K/V tile
+constexpr int kStages = 3;                      // slots of the K ring and of the V ring
+constexpr int kWgThreads = 128;                 // softmax warpgroup: one thread per column
+constexpr int kSoftmaxThreads = kPair * kWgThreads;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
-constexpr int kTmemCols = 512;                  // S[2] at columns 0 / 128, O at 256
+constexpr int kTmemCols = 512;                  // S of tile t at 128 t (+64), O of tile t at 256 + 128 t
 constexpr int kPlanThreads = 1024;
+constexpr int kSortBuckets = 256;               // unit lengths the plan kernel tells apart
+constexpr int kPlanRowsOnChip = 4096;           // unit starts the plan kernel keeps on chip
+constexpr int kMaxFoldRanges = 16;              // shared: ranges of a group's shared blocks, at most
 constexpr int kModePrefill = 0;
 constexpr int kModeShared = 1;
 
@@ -90,14 +99,15 @@ struct TcArgs {
   int num_seqs;                     // shared: sequences
   int num_listed;                   // shared: group_seqs entries
   int num_q_heads, num_kv_heads, max_blocks_per_seq, num_blocks, len_cap;
-  int range_blocks;                 // shared: shared blocks per range (a multiple of 8)
+  int num_sms;                      // shared: the plan sizes ranges to fill this many CTAs
   int max_ranges;                   // shared: ranges the partial arrays hold per column
   int oob_row;                      // a row of the cache tensors' 2-D view past their end
   float scale_log2;
   int* unit_start;                  // [rows + 1] work units before each sequence / group
-  int4* units;                      // [max_units][2] one record per work unit (plan kernel)
+  int4* units;                      // [max_units][2] one record per work unit, longest first
+  int4* units_raw;                  // [max_units][2] the same records in row order (plan kernel)
   int max_units;
-  int* counters;                    // shared: [num_listed * Hq] ranges finished, zero between calls
+  int* group_ranges;                // shared: [groups] ranges of each group (0: none folded)
   int* claim;                       // shared: [num_seqs] blocks attended per sequence
   float2* part_ml;                  // shared: [num_listed * Hq][max_ranges]
   float* part_o;                    // shared: [num_listed * Hq][max_ranges][D]
@@ -166,13 +176,44 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
   const int R = a.rows, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
   const int per = (R + kPlanThreads - 1) / kPlanThreads;
   const int r0 = min(R, tid * per), r1 = min(R, r0 + per);
+  // shared: ranges per group, so that all units together about fill the
+  // SMs: the pairs of column tiles x KV heads of every group are counted
+  // first, and each group's shared blocks are then cut into as many ranges
+  // (of whole K/V tiles, at least two) as one wave needs
+  __shared__ int s_target;
+  if constexpr (MODE == kModeShared) {
+    int base = 0;
+    for (int r = r0; r < r1; ++r) {
+      int gs, m, P, leader;
+      if (shared_group(a, r, &gs, &m, &P, &leader))
+        base += Hkv * (((m * G + kCols - 1) / kCols + kPair - 1) / kPair);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) base += __shfl_xor_sync(0xffffffffu, base, o);
+    if (lane == 0) s_wsum[warp] = base;
+    __syncthreads();
+    if (tid == 0) {
+      int tot = 0;
+      for (int w = 0; w < kPlanThreads / 32; ++w) tot += s_wsum[w];
+      s_target = tot > 0 ? max(1, (a.num_sms + tot - 1) / tot) : 1;
+    }
+    __syncthreads();
+  }
+  // a group's ranges: count and length in blocks (a multiple of a K/V tile)
+  auto ranges_of = [&](int P, int* rb) -> int {
+    int Rg = min(min(min(a.max_ranges, kMaxFoldRanges), max(1, P / (2 * kTileBlocks))), s_target);
+    int b = (P + Rg - 1) / Rg;
+    b = (b + kTileBlocks - 1) / kTileBlocks * kTileBlocks;
+    *rb = b;
+    return (P + b - 1) / b;
+  };
   int local = 0;
   for (int r = r0; r < r1; ++r) {
     int units = 0;
     if constexpr (MODE == kModePrefill) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
       if (prefill_seq(a, r, &q0, &Q, &n, &bit)) {
-        units = Hkv * ((Q + RPT - 1) / RPT);
+        units = Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair);
       } else if (bit) {
         seterr(a, bit);
         if (bit != kErrQuery || (a.query_start[r] >= 0 && a.query_start[r] <= a.query_start[r + 1] &&
@@ -185,13 +226,16 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
         }
       }
     } else {
-      int gs, m, P, leader;
+      int gs, m, P, leader, Rg = 0;
       if (shared_group(a, r, &gs, &m, &P, &leader)) {
-        const int nct = (m * G + kCols - 1) / kCols;
-        units = nct * Hkv * ((P + a.range_blocks - 1) / a.range_blocks);
+        const int npair = ((m * G + kCols - 1) / kCols + kPair - 1) / kPair;
+        int rb;
+        Rg = ranges_of(P, &rb);
+        units = npair * Hkv * Rg;
       } else {
         seterr(a, kErrGroup);
       }
+      a.group_ranges[r] = Rg;
     }
     a.unit_start[r] = units;  // (turned into starts below)
     local += units;
@@ -210,43 +254,117 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     if (w < warp) run += s_wsum[w];
     total += s_wsum[w];
   }
-  // each row's units as records {row, kv head, column tile, last key + 1}
-  // {prefill: first query row, rows, context length, 0 | shared: first
-  // member, members, shared blocks, range | ranges << 16}, so that the
-  // attention kernel finds a unit with one load instead of a search
   for (int r = r0; r < r1; ++r) {
     const int units = a.unit_start[r];
     a.unit_start[r] = run;
+    // (a group whose units do not all fit the workspace is not folded)
+    if (MODE == kModeShared && run + units > a.max_units) a.group_ranges[r] = 0;
+    run += units;
+  }
+  if (tid == 0) a.unit_start[R] = total;
+  __syncthreads();
+  // each unit as a record {row, kv head | pair of column tiles << 16, first
+  // key, last key + 1} {prefill: first query row, rows, context length, 0 |
+  // shared: first member, members, shared blocks, range | ranges << 16},
+  // written by all threads (each finds its unit's row by a search over the
+  // unit starts, kept on chip when they fit), so that the attention kernel
+  // finds a unit with one load instead of a search
+  __shared__ int s_us[kPlanRowsOnChip + 1];
+  const bool on_chip = R <= kPlanRowsOnChip;
+  if (on_chip)
+    for (int r = tid; r <= R; r += kPlanThreads) s_us[r] = __ldcg(a.unit_start + r);
+  __syncthreads();
+  auto start_of = [&](int r) -> int { return on_chip ? s_us[r] : __ldcg(a.unit_start + r); };
+  for (int u = tid; u < min(total, a.max_units); u += kPlanThreads) {
+    int lo = 0, up = R - 1;  // largest row with start_of(row) <= u
+    while (lo < up) {
+      const int mid = (lo + up + 1) >> 1;
+      if (start_of(mid) <= u) lo = mid; else up = mid - 1;
+    }
+    const int r = lo, k = u - start_of(lo);
     if constexpr (MODE == kModePrefill) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
-      if (units > 0 && prefill_seq(a, r, &q0, &Q, &n, &bit)) {
-        const int nct = (Q + RPT - 1) / RPT;
-        for (int k = 0; k < units && run + k < a.max_units; ++k) {
-          const int ct = k % nct, kvh = k / nct;
-          const int jl = min(Q, (ct + 1) * RPT) - 1;  // the tile's last query row
-          a.units[2 * (run + k)] = make_int4(r, kvh, ct, n - Q + jl + 1);
-          a.units[2 * (run + k) + 1] = make_int4(q0, Q, n, 0);
-        }
-      }
+      prefill_seq(a, r, &q0, &Q, &n, &bit);  // (true: only such rows have units)
+      const int npair = ((Q + RPT - 1) / RPT + kPair - 1) / kPair;
+      const int pr = k % npair, kvh = k / npair;
+      const int jl = min(Q, (pr + 1) * kPair * RPT) - 1;  // the pair's last query row
+      a.units_raw[2 * u] = make_int4(r, kvh | (pr << 16), 0, n - Q + jl + 1);
+      a.units_raw[2 * u + 1] = make_int4(q0, Q, n, 0);
     } else {
       int gs, m, P, leader;
-      if (units > 0 && shared_group(a, r, &gs, &m, &P, &leader)) {
-        const int nct = (m * G + kCols - 1) / kCols;
-        const int Rr = (P + a.range_blocks - 1) / a.range_blocks;
-        for (int k = 0; k < units && run + k < a.max_units; ++k) {
-          const int ct = k % nct, kvh = (k / nct) % Hkv, rr = k / (nct * Hkv);
-          const int k1 = min(P, (rr + 1) * a.range_blocks) * kBlockSize;
-          a.units[2 * (run + k)] = make_int4(leader, kvh, ct, k1);
-          a.units[2 * (run + k) + 1] = make_int4(gs, m, P, rr | (Rr << 16));
-        }
-      }
+      shared_group(a, r, &gs, &m, &P, &leader);  // (true: only such groups have units)
+      const int npair = ((m * G + kCols - 1) / kCols + kPair - 1) / kPair;
+      int rb;
+      const int Rr = ranges_of(P, &rb);
+      const int pr = k % npair, kvh = (k / npair) % Hkv, rr = k / (npair * Hkv);
+      const int k1 = min(P, (rr + 1) * rb) * kBlockSize;
+      a.units_raw[2 * u] = make_int4(leader, kvh | (pr << 16), rr * rb * kBlockSize, k1);
+      a.units_raw[2 * u + 1] = make_int4(gs, m, P, rr | (Rr << 16));
     }
-    run += units;
   }
   if (tid == 0) {
     // (the workspace is sized for the most units a call can have)
     if (total > a.max_units) seterr(a, kErrTimeout);
-    a.unit_start[R] = min(total, a.max_units);
+    if (total > a.max_units) a.unit_start[R] = a.max_units;
+  }
+  // Units differ in length (a causal tile's keys end at its last row; ranges
+  // and sequences differ), and the attention kernel deals them to its CTAs in
+  // rounds, so they are ordered longest first (a counting sort by K/V tiles)
+  // and the CTAs take them in snake order: that spreads the long ones.
+  __shared__ int s_hist[kSortBuckets];
+  __shared__ int s_pos[kSortBuckets];
+  const int T = min(total, a.max_units);
+  for (int b = tid; b < kSortBuckets; b += kPlanThreads) s_hist[b] = 0;
+  __syncthreads();  // (also: every thread's raw records are written)
+  auto bucket = [&](int u) -> int {
+    const int4 r0 = __ldcg(a.units_raw + 2 * u);
+    const int nt = (r0.w - r0.z + kKeys - 1) / kKeys;
+    return nt < kSortBuckets - 1 ? nt : kSortBuckets - 1;
+  };
+  // (lanes with the same bucket add together: one shared-memory atomic per
+  // distinct bucket and warp, not one per unit -- equal lengths are common)
+  const int Tw = (T + 31) / 32 * 32;
+  for (int u = tid; u < Tw; u += kPlanThreads) {
+    const int b = u < T ? bucket(u) : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, b);
+    if (b >= 0 && lane == __ffs(same) - 1) atomicAdd(&s_hist[b], __popc(same));
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // bucket starts, longest first: an exclusive scan from the top bucket down
+    constexpr int PER = kSortBuckets / 32;
+    int v[PER], sum = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      v[i] = s_hist[kSortBuckets - 1 - (lane * PER + i)];
+      sum += v[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int tt = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += tt;
+    }
+    int run2 = incl - sum;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      s_pos[kSortBuckets - 1 - (lane * PER + i)] = run2;
+      run2 += v[i];
+    }
+  }
+  __syncthreads();
+  for (int u = tid; u < Tw; u += kPlanThreads) {
+    const int b = u < T ? bucket(u) : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, b);
+    const int leader = __ffs(same) - 1;
+    int base = 0;
+    if (b >= 0 && lane == leader) base = atomicAdd(&s_pos[b], __popc(same));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (b >= 0) {
+      const int pos = base + __popc(same & ((1u << lane) - 1));
+      a.units[2 * pos] = __ldcg(a.units_raw + 2 * u);
+      a.units[2 * pos + 1] = __ldcg(a.units_raw + 2 * u + 1);
+    }
   }
 }
 
@@ -256,7 +374,7 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
 struct Unit {
   int row;    // block-table row
   int kvh;
-  int ct;     // column tile
+  int pr;     // pair of column tiles: tiles 2 pr and 2 pr + 1
   int k0;     // first key of the unit
   int k1;     // one past its last key
   int nt;     // K/V tiles
@@ -275,21 +393,20 @@ template <int MODE>
 __device__ __forceinline__ void load_unit(const TcArgs& a, int u, Unit* x) {
   const int4 r0 = __ldcg(a.units + 2 * u), r1 = __ldcg(a.units + 2 * u + 1);
   x->row = r0.x;
-  x->kvh = r0.y;
-  x->ct = r0.z;
+  x->kvh = r0.y & 0xffff;
+  x->pr = r0.y >> 16;
+  x->k0 = r0.z;
   x->k1 = r0.w;
   if constexpr (MODE == kModePrefill) {
     x->q0 = r1.x;
     x->Q = r1.y;
     x->n = r1.z;
-    x->k0 = 0;
   } else {
     x->gs = r1.x;
     x->m = r1.y;
     x->P = r1.z;
     x->r = r1.w & 0xffff;
     x->R = r1.w >> 16;
-    x->k0 = x->r * a.range_blocks * kBlockSize;
   }
   x->nt = (x->k1 - x->k0 + kKeys - 1) / kKeys;
 }
@@ -312,55 +429,55 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, 
 template <int D, int G, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_constant__ TcArgs a) {
   constexpr int KB = D / 64;                 // 64-element (128-byte) blocks of head_dim
-  constexpr int QT = kCols * D * 2;          // bytes of the Q tile
+  constexpr int QT = kCols * D * 2;          // bytes of a Q tile
   constexpr int KT = kKeys * D * 2;          // bytes of a K (or V) tile
-  constexpr int PT = kCols * kKeys * 2;      // bytes of the P tile
+  constexpr int PT = kCols * kKeys * 2;      // bytes of a P tile (one 128-byte row per column)
   constexpr int HALF = kKeys * 128;          // bytes of a 64-element half of a K/V tile
   constexpr int RPT = kCols / G;
   constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(kCols, kKeys, false);
   constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(kCols, D, true);
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(kKeys == 64, "a P row is one 128-byte swizzle row");
 
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   unsigned char* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  unsigned char* sQ = sm;
-  unsigned char* sK = sQ + QT;               // [kStages][KT]
+  unsigned char* sQ = sm;                    // [kPair][QT]
+  unsigned char* sK = sQ + kPair * QT;       // [kStages][KT]
   unsigned char* sV = sK + kStages * KT;     // [kStages][KT]
-  unsigned char* sP = sV + kStages * KT;     // [PT]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + PT);
-  // barriers: kfull[2] kempty[2] vfull[2] vempty[2] sfull[2] pfull odone qfull drain sync
+  unsigned char* sP = sV + kStages * KT;     // [kPair][PT]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPair * PT);
+  // barriers: kfull[3] kempty[3] vfull[3] vempty[3] | per tile t: sfull[t][2],
+  // pfull[t], odone[t], sync[t] | qfull drain
   const uint32_t b0 = smem_addr(bars);
-  const uint32_t KFULL = b0, KEMPTY = b0 + 16, VFULL = b0 + 32, VEMPTY = b0 + 48, SFULL = b0 + 64;
-  const uint32_t PFULL = b0 + 80, ODONE = b0 + 88, QFULL = b0 + 96, DRAIN = b0 + 104;
-  const uint32_t SYNC = b0 + 112;  // the softmax threads among themselves (bounded, unlike bar.sync)
+  const uint32_t KFULL = b0, KEMPTY = b0 + 24, VFULL = b0 + 48, VEMPTY = b0 + 72;
+  const uint32_t TB = b0 + 96;  // tile t's barriers at TB + 40 t: sfull[2], pfull, odone, sync
+  const uint32_t QFULL = b0 + 96 + 40 * kPair, DRAIN = QFULL + 8;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_red[3];
-  __shared__ float s_xch[2][2][kCols];  // per half: row maxima of a tile / row sums of a unit
-  // shared mode: the fold's member checks
-  __shared__ int s_seq[kCols];
-  __shared__ unsigned char s_ok[kCols];
-  __shared__ int s_last;
+  __shared__ int s_red[kPair][3];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hq = a.num_q_heads, Hkv = a.num_kv_heads;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(KFULL + 8 * i, 1);
       mbar_init(KEMPTY + 8 * i, 1);
       mbar_init(VFULL + 8 * i, 1);
       mbar_init(VEMPTY + 8 * i, 1);
-      mbar_init(SFULL + 8 * i, 1);
     }
-    mbar_init(PFULL, kSoftmaxThreads);
-    mbar_init(ODONE, 1);
+    for (int t = 0; t < kPair; ++t) {
+      mbar_init(TB + 40 * t, 1);        // sfull[0]
+      mbar_init(TB + 40 * t + 8, 1);    // sfull[1]
+      mbar_init(TB + 40 * t + 16, kWgThreads);  // pfull
+      mbar_init(TB + 40 * t + 24, 1);   // odone
+      mbar_init(TB + 40 * t + 32, kWgThreads);  // sync (the tile's warpgroup among itself)
+      s_red[t][0] = s_red[t][1] = s_red[t][2] = 0;
+    }
     mbar_init(QFULL, kSoftmaxThreads);
     mbar_init(DRAIN, 1);
-    mbar_init(SYNC, kSoftmaxThreads);
     s_abort = 0;
-    s_red[0] = s_red[1] = s_red[2] = 0;
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -374,10 +491,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
 
   // the unit layout comes from the plan kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // shared: the fold kernel behind this one may start its member checks
+  if constexpr (MODE == kModeShared) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int total = __ldcg(a.unit_start + a.rows);  // (written by the plan kernel: see load_unit)
 
   auto timeout = [&]() {
     if (atomicExch(&s_abort, 1) == 0) seterr(a, kErrTimeout);
+  };
+  // this CTA's k-th unit: rounds of gridDim.x units (longest first), taken
+  // in snake order so that the long ones spread over the CTAs
+  auto unit_of = [&](int k) -> int {
+    const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    return k * g + ((k & 1) ? g - 1 - b : b);
   };
   auto aborted_one = [&]() { return *reinterpret_cast<volatile int*>(&s_abort) != 0; };
   // (the producer and softmax warps test it with all lanes and act on one answer)
@@ -386,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   if (warp == kProducerWarp) {
     // ---------------- producer: K runs one tile ahead of V ----------------------
     int kidx = 0, vidx = 0;
-    int yprev = a.oob_row;  // (lane b < 8: tile row of block b of the previous tile)
+    int yprev = a.oob_row;  // (lane b < 4: tile row of block b of the previous tile)
     bool have_prev = false, ok = true;
     auto issue_v = [&](int ysrc) -> bool {
       const int st = vidx % kStages;
@@ -404,9 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       return true;
     };
     Unit x, nx;
-    if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, x = nx) {
-      if (u + static_cast<int>(gridDim.x) < total) load_unit<MODE>(a, u + gridDim.x, &nx);
+    if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
+    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
+      if (unit_of(k + 1) < total) load_unit<MODE>(a, unit_of(k + 1), &nx);
       const int32_t* trow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
       // block rows of the unit's first tile; then always one tile ahead
       auto rows_of = [&](int j) -> int {
@@ -455,55 +580,77 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       mbar_wait_bounded(VFULL + 8 * (i % kStages), (i / kStages) & 1);
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer -------------------------------------------------
+    // Per K/V tile j: S_A(j), S_B(j) were issued two tiles ahead; as each
+    // warpgroup releases P_t(j): O_t += P_t(j) V(j), then S_t(j + 2) into the
+    // S buffer P_t(j) has freed.
     if (lane == 0) {
-      int kidx = 0, vidx = 0, sidx = 0, pidx = 0, qidx = 0;
+      int kidx = 0, vidx = 0, qidx = 0;
+      int sidx[kPair] = {0, 0}, pidx[kPair] = {0, 0};
       bool ok = true;
       const uint32_t qbase = smem_addr(sQ), pbase = smem_addr(sP);
-      auto issue_s = [&]() -> bool {
-        const int st = kidx % kStages;
-        if (!mbar_wait_bounded(KFULL + 8 * st, (kidx / kStages) & 1)) return false;
-        tc::fence_after_sync();
-        const uint32_t kbase = smem_addr(sK + st * KT);
-        const uint32_t dS = tmem + (sidx & 1) * kKeys;
+      // S_t of the K tile in ring slot kidx (its K has landed)
+      auto issue_s = [&](int t) {
+        const uint32_t kbase = smem_addr(sK + (kidx % kStages) * KT);
+        const uint32_t dS = tmem + t * 2 * kKeys + (sidx[t] & 1) * kKeys;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k / 4) * (kCols * 128) + (k % 4) * 32;
           const uint32_t koff = (k / 4) * HALF + (k % 4) * 32;
-          tc::mma_bf16_ss(dS, tc::sdesc_sw128(qbase + off, 16, 1024),
+          tc::mma_bf16_ss(dS, tc::sdesc_sw128(qbase + t * QT + off, 16, 1024),
                           tc::sdesc_sw128(kbase + koff, 16, 1024), IDESC_S, k > 0);
         }
-        tc::commit(KEMPTY + 8 * st);
-        tc::commit(SFULL + 8 * (sidx & 1));
-        ++kidx;
-        ++sidx;
+        tc::commit(TB + 40 * t + 8 * (sidx[t] & 1));
+        ++sidx[t];
+      };
+      auto k_landed = [&]() -> bool {
+        if (!mbar_wait_bounded(KFULL + 8 * (kidx % kStages), (kidx / kStages) & 1)) return false;
+        tc::fence_after_sync();
         return true;
       };
+      auto k_done = [&]() {  // both tiles' S of this K tile issued: its slot frees on completion
+        tc::commit(KEMPTY + 8 * (kidx % kStages));
+        ++kidx;
+      };
       Unit x, nx;
-      if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, x = nx) {
-        if (u + static_cast<int>(gridDim.x) < total) load_unit<MODE>(a, u + gridDim.x, &nx);
+      if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
+      for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
+        if (unit_of(k + 1) < total) load_unit<MODE>(a, unit_of(k + 1), &nx);
         if (aborted_one() || !mbar_wait_bounded(QFULL, qidx & 1)) { ok = false; break; }
         ++qidx;
         tc::fence_after_sync();
-        for (int j = 0; j < 2 && j < x.nt && ok; ++j) ok = issue_s();
+        for (int j = 0; j < 2 && j < x.nt && ok; ++j) {
+          if (!(ok = k_landed())) break;
+          issue_s(0);
+          issue_s(1);
+          k_done();
+        }
         for (int j = 0; j < x.nt && ok; ++j) {
-          if (aborted_one() || !mbar_wait_bounded(PFULL, pidx & 1)) { ok = false; break; }
-          ++pidx;
           const int st = vidx % kStages;
-          if (!mbar_wait_bounded(VFULL + 8 * st, (vidx / kStages) & 1)) { ok = false; break; }
-          tc::fence_after_sync();
           const uint32_t vbase = smem_addr(sV + st * KT);
+          const bool ahead = j + 2 < x.nt;
 #pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k) {
-            const uint32_t poff = (k / 4) * (kCols * 128) + (k % 4) * 32;
-            tc::mma_bf16_ss(tmem + 2 * kKeys, tc::sdesc_sw128(pbase + poff, 16, 1024),
-                            tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
-                            (j > 0 || k > 0) ? 1u : 0u);
+          for (int t = 0; t < kPair; ++t) {
+            if (aborted_one() || !mbar_wait_bounded(TB + 40 * t + 16, pidx[t] & 1)) { ok = false; break; }
+            ++pidx[t];
+            if (t == 0 && !mbar_wait_bounded(VFULL + 8 * st, (vidx / kStages) & 1)) { ok = false; break; }
+            tc::fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < kKeys / 16; ++k)
+              tc::mma_bf16_ss(tmem + 2 * kPair * kKeys + t * D,
+                              tc::sdesc_sw128(pbase + t * PT + k * 32, 16, 1024),
+                              tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
+                              (j > 0 || k > 0) ? 1u : 0u);
+            tc::commit(TB + 40 * t + 24);  // odone[t]
+            if (t == kPair - 1) {
+              tc::commit(VEMPTY + 8 * st);
+              ++vidx;
+            }
+            if (ahead) {
+              if (t == 0 && !(ok = k_landed())) break;
+              issue_s(t);
+              if (t == kPair - 1) k_done();
+            }
           }
-          tc::commit(VEMPTY + 8 * st);
-          tc::commit(ODONE);
-          ++vidx;
-          if (j + 2 < x.nt) ok = issue_s();
         }
       }
       if (!ok) timeout();
@@ -513,59 +660,49 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     }
     __syncwarp();
   } else {
-    // ---------------- softmax: two threads per column -----------------------------
-    // Thread t (0..255) serves column col = t % 128, which is TMEM lane col
-    // (warps w and w + 4 share a lane quarter), and half hf = t / 128 of it:
-    // keys 64 hf .. 64 hf + 63 of every tile, head_dim D/2 hf .. D/2 hf + D/2 - 1
-    // of O, and its own share of the row sum.  The two threads of a column
-    // swap their partial row maxima once per tile and their sums once per unit.
-    const int col = tid % kCols, hf = tid / kCols;
+    // ---------------- softmax: warpgroup t = warp / 4 serves column tile 2 pr + t;
+    // thread col owns column col (TMEM lane col of that tile's S and O)
+    const int t = warp / 4, col = tid % kWgThreads;
     const int h = col % G;
-    constexpr int HK = kKeys / 2;   // keys per thread and tile
-    constexpr int HD = D / 2;       // O columns per thread
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-    int sidx = 0, oidx = 0, tile = 0, syncs = 0, reds = 0, xs = 0;
+    const uint32_t SFULL = TB + 40 * t, PFULL = SFULL + 16, ODONE = SFULL + 24, SYNC = SFULL + 32;
+    const uint32_t s_col = t * 2 * kKeys, o_col = 2 * kPair * kKeys + t * D;  // TMEM columns
+    unsigned char* const myQ = sQ + t * QT;
+    unsigned char* const myP = sP + t * PT;
+    int sidx = 0, oidx = 0, tile = 0, syncs = 0, reds = 0;
     bool ok = true;
     // a bounded wait whose outcome the whole warp shares, so that no lane
     // leaves ahead of the others (the TMEM moves are warp-wide)
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
     };
-    auto group_sync = [&]() -> bool {
+    auto group_sync = [&]() -> bool {  // the 128 threads of this warpgroup
       mbar_arrive(SYNC);
       return wait_all(SYNC, (syncs++) & 1);
     };
-    // OR of a flag over the softmax threads; slot reds % 3 is cleared two uses ahead
+    // OR of a flag over the warpgroup; slot reds % 3 is cleared two uses ahead
     auto group_or = [&](bool v, bool* res) -> bool {
       const int slot = reds % 3;
-      if (v) atomicOr(&s_red[slot], 1);
+      if (v) atomicOr(&s_red[t][slot], 1);
       if (!group_sync()) return false;
-      *res = *reinterpret_cast<volatile int*>(&s_red[slot]) != 0;
-      if (tid == 0) s_red[(reds + 2) % 3] = 0;
+      *res = *reinterpret_cast<volatile int*>(&s_red[t][slot]) != 0;
+      if (col == 0) s_red[t][(reds + 2) % 3] = 0;
       ++reds;
-      return true;
-    };
-    // the other half's value of this column (the exchange slot alternates, so
-    // that one sync per exchange suffices)
-    auto swap_half = [&](float v, float* other) -> bool {
-      const int sl = (xs++) & 1;
-      s_xch[sl][hf][col] = v;
-      if (!group_sync()) return false;
-      *other = s_xch[sl][hf ^ 1][col];
       return true;
     };
     // this column's query row in unit y (-1: none), and the keys it sees
     auto column_of = [&](const Unit& y, int* kend) -> int {
       int qrow = -1;
+      const int ct = y.pr * kPair + t;
       if constexpr (MODE == kModePrefill) {
-        const int jr = y.ct * RPT + col / G;
+        const int jr = ct * RPT + col / G;
         *kend = 0;
         if (jr < y.Q) {
           qrow = y.q0 + jr;
           *kend = min(y.k1, y.n - y.Q + jr + 1);
         }
       } else {
-        const int member = y.ct * RPT + col / G;
+        const int member = ct * RPT + col / G;
         if (member < y.m) {
           const int seq = a.group_seqs[y.gs + member];
           if (seq >= 0 && seq < a.num_seqs) qrow = seq;
@@ -574,25 +711,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       }
       return qrow;
     };
-    // this thread's half of its column's q row into the swizzled Q tile
-    // (zeros for no row)
+    // this column's q row into its tile's swizzled Q (zeros for no row)
     auto load_q = [&](const Unit& y, int qrow) {
       const __nv_bfloat16* src =
           a.q + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + y.kvh * G + h) * D;
-      const uint32_t qb = smem_addr(sQ) + col * 128;
+      const uint32_t qb = smem_addr(myQ) + col * 128;
 #pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) {
-        const int c = hf * (D / 16) + cc;  // 16-byte chunk of the row
+      for (int c = 0; c < D / 8; ++c)
         cp_async16_zfill(qb + (c / 8) * (kCols * 128) + (((c % 8) ^ (col % 8)) << 4), src + c * 8,
                          qrow >= 0);
-      }
     };
     Unit x, nx;
-    if (blockIdx.x < total) load_unit<MODE>(a, blockIdx.x, &x);
+    if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
     bool q_issued = false;  // this unit's Q already requested (during the last unit)
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, x = nx) {
-      const bool has_next = u + static_cast<int>(gridDim.x) < total;
-      if (has_next) load_unit<MODE>(a, u + gridDim.x, &nx);
+    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
+      const bool has_next = unit_of(k + 1) < total;
+      if (has_next) load_unit<MODE>(a, unit_of(k + 1), &nx);
       int kend;
       const int qrow = column_of(x, &kend);
       // ---- the unit's blocks must be in range (prefill: a bad one empties the sequence)
@@ -600,12 +734,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       if constexpr (MODE == kModePrefill) {
         const int nb = (x.n + kBlockSize - 1) / kBlockSize;
         const int32_t* trow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
-        for (int b = tid; b < nb; b += kSoftmaxThreads) {
+        for (int b = col; b < nb; b += kWgThreads) {
           const int phys = __ldg(trow + b);
           bad |= !(phys >= 0 && phys < a.num_blocks);
         }
         if (!group_or(bad, &bad)) { ok = false; break; }
-        if (bad && tid == 0) seterr(a, kErrBlockId);
+        if (bad && col == 0 && t == 0) seterr(a, kErrBlockId);
       }
       // ---- Q: requested now, or already during the previous unit's last tile
       if (!q_issued) load_q(x, qrow);
@@ -619,44 +753,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       for (int j = 0; j < x.nt; ++j, ++tile) {
         if (aborted() || !wait_all(SFULL + 8 * (sidx & 1), (sidx >> 1) & 1)) { ok = false; break; }
         tc::fence_after_sync();
-        uint32_t sv[HK];
-        tc::tmem_ld64(lane_base + (sidx & 1) * kKeys + hf * HK, sv);
+        uint32_t sv[kKeys];
+        tc::tmem_ld64(lane_base + s_col + (sidx & 1) * kKeys, sv);
         tc::tmem_wait_ld(sv);
         ++sidx;
         if (j == x.nt - 1 && has_next) {
-          // every S of this unit is complete: the Q tile is free for the next unit
+          // every S of this tile in this unit is complete: its Q is free
           int kn;
           load_q(nx, column_of(nx, &kn));
           q_issued = true;
         }
         // scale to log2 units, mask the keys this column does not see, and take
-        // the maximum over 8 independent chains, then with the other half's
-        const int kb = x.k0 + j * kKeys + hf * HK;
+        // the maximum over 8 independent chains
+        const int kb = x.k0 + j * kKeys;
         float m8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
-        if (kb + HK <= kend) {
+        if (kb + kKeys <= kend) {
 #pragma unroll
-          for (int t = 0; t < HK; ++t) {
-            const float v = __uint_as_float(sv[t]) * a.scale_log2;
-            sv[t] = __float_as_uint(v);
-            m8[t & 7] = fmaxf(m8[t & 7], v);
+          for (int k = 0; k < kKeys; ++k) {
+            const float v = __uint_as_float(sv[k]) * a.scale_log2;
+            sv[k] = __float_as_uint(v);
+            m8[k & 7] = fmaxf(m8[k & 7], v);
           }
         } else {
 #pragma unroll
-          for (int t = 0; t < HK; ++t) {
-            const float v = kb + t < kend ? __uint_as_float(sv[t]) * a.scale_log2 : -INFINITY;
-            sv[t] = __float_as_uint(v);
-            m8[t & 7] = fmaxf(m8[t & 7], v);
+          for (int k = 0; k < kKeys; ++k) {
+            const float v = kb + k < kend ? __uint_as_float(sv[k]) * a.scale_log2 : -INFINITY;
+            sv[k] = __float_as_uint(v);
+            m8[k & 7] = fmaxf(m8[k & 7], v);
           }
         }
-        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        {
-          float mo;
-          if (!swap_half(mx, &mo)) { ok = false; break; }
-          mx = fmaxf(mx, mo);  // (both halves now hold the same tile maximum)
-        }
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         if (j > 0) {
           // O of the previous tile is complete: its P slot is free and O is stable
           if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
@@ -671,14 +800,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           m_run = mx;
         }
         // weights, rounded to bf16 for the product; the sum (8 chains) takes
-        // them as rounded; this half's 64 keys are P's K-block hf
+        // them as rounded
         const bool none = m_run == -INFINITY;
-        const uint32_t pb = smem_addr(sP) + hf * (kCols * 128) + col * 128;
+        const uint32_t pb = smem_addr(myP) + col * 128;
         float l8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) l8[c] = 0.f;
 #pragma unroll
-        for (int c = 0; c < HK / 8; ++c) {
+        for (int c = 0; c < kKeys / 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -689,25 +818,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
             l8[2 * e + 1] += __high2float(pp);
             w[e] = *reinterpret_cast<const uint32_t*>(&pp);
           }
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                           pb + (((c % 8) ^ (col % 8)) << 4)),
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + (((c % 8) ^ (col % 8)) << 4)),
                        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                        : "memory");
         }
         l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         if constexpr (MODE == kModePrefill) {
           // rows past the sequence's end in its last block hold stale data: a
-          // zero weight times a NaN would still poison O, so they are zeroed
+          // zero weight times a NaN would still poison O, so tile A's
+          // warpgroup zeroes them before the first of the tile's two P.V
           const int tail = x.n % kBlockSize;
-          const int lastb = x.n / kBlockSize;        // logical block holding them
-          const int kt = x.k0 + j * kKeys;           // the tile's first key
-          if (tail && lastb * kBlockSize >= kt && lastb * kBlockSize < kt + kKeys) {
+          const int lastb = x.n / kBlockSize;  // logical block holding them
+          if (t == 0 && tail && lastb * kBlockSize >= kb && lastb * kBlockSize < kb + kKeys) {
             const int st = tile % kStages;
             if (!wait_all(VFULL + 8 * st, (tile / kStages) & 1)) { ok = false; break; }
-            const int b = (lastb * kBlockSize - kt) / kBlockSize;
+            const int b = (lastb * kBlockSize - kb) / kBlockSize;
             unsigned char* vt = sV + st * KT;
             const int nz = (kBlockSize - tail) * 8 * KB;  // 16-byte chunks to clear
-            for (int i = tid; i < nz; i += kSoftmaxThreads) {
+            for (int i = col; i < nz; i += kWgThreads) {
               const int hx = i / ((kBlockSize - tail) * 8);
               const int rem = i % ((kBlockSize - tail) * 8);
               const int row = b * kBlockSize + tail + rem / 8;
@@ -716,18 +844,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
             }
           }
         }
-        // this half of the O row is rescaled by the whole warp together (the
-        // TMEM moves are warp-wide; rows that do not grow are multiplied by 1),
-        // after the S row is spent and before P is released to the MMA
+        // O rows are rescaled by the whole warp together (the TMEM moves are
+        // warp-wide; rows that do not grow are multiplied by 1), after the S
+        // row is spent and before P is released to the MMA
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-          for (int c = 0; c < HD / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
-            tc::tmem_ld32(lane_base + 2 * kKeys + hf * HD + c * 32, r);
+            tc::tmem_ld32(lane_base + o_col + c * 32, r);
             tc::tmem_wait_ld(r);
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * al);
-            tc::tmem_st32(lane_base + 2 * kKeys + hf * HD + c * 32, r);
+            tc::tmem_st32(lane_base + o_col + c * 32, r);
           }
           tc::tmem_wait_st();
         }
@@ -736,135 +864,56 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         mbar_arrive(PFULL);
       }
       if (!ok) break;
-      // ---- the unit's O row: this thread's half, over the column's whole sum
+      // ---- the unit's O row (in halves of 64 columns)
       if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
       ++oidx;
       tc::fence_after_sync();
-      float lo;
-      if (!swap_half(l_run, &lo)) { ok = false; break; }
-      const float l_all = l_run + lo;
-      uint32_t ov[HD];
-      if constexpr (HD == 64) tc::tmem_ld64(lane_base + 2 * kKeys + hf * HD, ov);
-      else tc::tmem_ld32(lane_base + 2 * kKeys + hf * HD, ov);
-      tc::tmem_wait_ld(ov);
       if constexpr (MODE == kModePrefill) {
-        // (every lane ran the warp-wide TMEM load; only live columns store)
-        if (qrow >= 0) {
-          const float inv = bad ? 0.f : 1.f / l_all;
-          uint4* dst = reinterpret_cast<uint4*>(
-              a.out + (static_cast<size_t>(qrow) * Hq + x.kvh * G + h) * D + hf * HD);
+        // (every lane runs the warp-wide TMEM loads; only live columns store)
+        const float inv = bad ? 0.f : 1.f / l_run;
+        uint4* dst = reinterpret_cast<uint4*>(
+            a.out + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + x.kvh * G + h) * D);
 #pragma unroll
-          for (int c = 0; c < HD / 8; ++c) {
-            uint32_t w[4];
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t ov[64];
+          tc::tmem_ld64(lane_base + o_col + hf * 64, ov);
+          tc::tmem_wait_ld(ov);
+          if (qrow >= 0) {
 #pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              const __nv_bfloat162 pp = __floats2bfloat162_rn(
-                  __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
-              w[f] = *reinterpret_cast<const uint32_t*>(&pp);
+            for (int c = 0; c < 8; ++c) {
+              uint32_t w[4];
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {
+                const __nv_bfloat162 pp = __floats2bfloat162_rn(
+                    __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
+                w[f] = *reinterpret_cast<const uint32_t*>(&pp);
+              }
+              dst[hf * 8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       } else {
-        // ---- shared: this range's partial state, then the fold by the last range
-        const int member = x.ct * RPT + col / G;
+        // ---- shared: this range's partial state (the fold kernel combines the ranges)
+        const int ct = x.pr * kPair + t;
+        const int member = ct * RPT + col / G;
         const bool live = member < x.m;
         const size_t pi = live ? (static_cast<size_t>(x.gs + member) * Hq + x.kvh * G + h) *
                                          a.max_ranges + x.r
                                : 0;
-        if (live) {
-          float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + hf * HD);
 #pragma unroll
-          for (int e = 0; e < HD / 4; ++e)
-            po[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
-                                __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
-          if (hf == 0) a.part_ml[pi] = make_float2(m_run, l_all);
+        for (int hf = 0; hf < D / 64; ++hf) {
+          uint32_t ov[64];
+          tc::tmem_ld64(lane_base + o_col + hf * 64, ov);
+          tc::tmem_wait_ld(ov);
+          if (live) {
+            float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + hf * 64);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              po[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+          }
         }
-        __threadfence();
-        if (!group_sync()) { ok = false; break; }
-        if (tid == 0) {
-          int* cnt = a.counters + (static_cast<size_t>(x.gs) * G + x.ct * kCols) * Hkv + x.kvh;
-          const int prev = atomicAdd(cnt, 1);
-          s_last = prev == x.R - 1;
-          if (s_last) *cnt = 0;  // every range has arrived: zero again for the next call
-        }
-        if (!group_sync()) { ok = false; break; }
-        if (*reinterpret_cast<volatile int*>(&s_last)) {
-          __threadfence();
-          const int mlo = x.ct * RPT;
-          const int nm = min(x.m - mlo, RPT);  // members of this tile
-          const int32_t* lrow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
-          if (tid < nm) {
-            const int seq = a.group_seqs[x.gs + mlo + tid];
-            bool okm = seq >= 0 && seq < a.num_seqs;
-            if (okm) {
-              const int n = a.context_lens[seq];
-              okm = n > 0 && n <= a.len_cap && kBlockSize * x.P <= n - 1;
-            }
-            s_seq[tid] = okm ? seq : -1;
-            s_ok[tid] = okm;
-          }
-          if (!group_sync()) { ok = false; break; }
-          // every (member, shared block): the member's table holds the leader's block
-          for (int idx = tid; idx < nm * x.P; idx += kSoftmaxThreads) {
-            const int i = idx / x.P, jb = idx - i * x.P;
-            const int seq = s_seq[i];
-            if (seq < 0) continue;
-            const int b = __ldg(lrow + jb);
-            if (!(b >= 0 && b < a.num_blocks &&
-                  __ldg(a.block_tables + static_cast<size_t>(seq) * a.max_blocks_per_seq + jb) == b))
-              s_ok[i] = 0;  // (every writer stores the same value)
-          }
-          if (!group_sync()) { ok = false; break; }
-          if (x.kvh == 0 && tid < nm && !s_ok[tid]) seterr(a, kErrGroup);
-          if (live && s_ok[col / G]) {
-            // this thread folds its half of the column's head_dim
-            const size_t pb0 = (static_cast<size_t>(x.gs + member) * Hq + x.kvh * G + h) * a.max_ranges;
-            float M = -INFINITY;
-            for (int rr = 0; rr < x.R; ++rr) M = fmaxf(M, __ldcg(a.part_ml + pb0 + rr).x);
-            const size_t orow = static_cast<size_t>(s_seq[col / G]) * Hq + x.kvh * G + h;
-            // (in passes of 32 dims, to keep the accumulators in registers)
-            constexpr int QD = HD < 32 ? HD : 32;
-            float L = 0.f;
-#pragma unroll 1
-            for (int q0 = 0; q0 < HD; q0 += QD) {
-              float4 acc[QD / 4];
-#pragma unroll
-              for (int e = 0; e < QD / 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-              L = 0.f;
-              for (int rr = 0; rr < x.R; ++rr) {
-                const float2 ml = __ldcg(a.part_ml + pb0 + rr);
-                const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-                L += w * ml.y;
-                const float4* po =
-                    reinterpret_cast<const float4*>(a.part_o + (pb0 + rr) * D + hf * HD + q0);
-#pragma unroll
-                for (int e = 0; e < QD / 4; ++e) {
-                  const float4 o4 = __ldcg(po + e);
-                  acc[e].x = fmaf(w, o4.x, acc[e].x);
-                  acc[e].y = fmaf(w, o4.y, acc[e].y);
-                  acc[e].z = fmaf(w, o4.z, acc[e].z);
-                  acc[e].w = fmaf(w, o4.w, acc[e].w);
-                }
-              }
-              float4* dst = reinterpret_cast<float4*>(a.pre_o + orow * D + hf * HD + q0);
-#pragma unroll
-              for (int e = 0; e < QD / 4; ++e) dst[e] = acc[e];
-            }
-            if (hf == 0) a.pre_ml[orow] = make_float2(M, L);
-          }
-          // claim each checked member once (KV head 0; a member's columns all
-          // lie in one tile, since 128 is a multiple of G); a sequence claimed
-          // twice is given up
-          if (x.kvh == 0 && tid < nm && s_ok[tid]) {
-            const int seq = s_seq[tid];
-            if (atomicCAS(a.claim + seq, 0, x.P) != 0) {
-              atomicExch(a.claim + seq, -1);
-              seterr(a, kErrGroup);
-            }
-          }
-          if (!group_sync()) { ok = false; break; }  // (s_ok, s_seq rewritten next unit)
-        }
+        if (live) a.part_ml[pi] = make_float2(m_run, l_run);
       }
     }
     if (!ok) timeout();
@@ -876,6 +925,109 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   __syncthreads();
   tc::fence_after_sync();
   if (warp == kMmaWarp) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// shared: the fold of a group's ranges, per listed member
+// ---------------------------------------------------------------------------
+// CTA (member i, slice y of the query heads); thread = 4 dims of one head.
+// Each range left a partial state (m_r, l_r, o_r) per column; the state over
+// all the shared blocks is their log-sum-exp combination
+//   M = max_r m_r,  w_r = 2^(m_r - M),  l = sum_r w_r l_r,  o = sum_r w_r o_r,
+// stored per (sequence, head) for the decode kernel to go on from.  The
+// member is first checked against the block tables -- its row must hold the
+// leader's blocks, and its length must leave a token after them -- and is
+// claimed once (a sequence that two listings claim is given up, and the
+// decode kernel attends to all of it).  The check reads only the call's
+// inputs, so it runs while the pass is still going; the partial states are
+// read once the pass has finished (griddepcontrol.wait).  CTAs are small
+// (128 threads, at most 64 registers each) so that one fits beside an
+// attention CTA and starts while the pass runs.
+constexpr int kFoldThreads = 128;
+constexpr int kFoldBatch = 8;  // ranges whose loads are in flight together
+
+template <int D>
+__global__ void __launch_bounds__(kFoldThreads, 8) tc_fold_kernel(const __grid_constant__ TcArgs a) {
+  constexpr int V = D / 4;                  // threads of a head (float4 each)
+  constexpr int HPC = kFoldThreads / V;     // heads of a CTA
+  const int i = blockIdx.x, tid = threadIdx.x;
+  const int Hq = a.num_q_heads;
+  const int h = blockIdx.y * HPC + tid / V, d4 = tid % V;
+  // the group listing member i: the last g with group_start[g] <= i
+  int lo = 0, up = a.rows - 1;
+  while (lo < up) {
+    const int mid = (lo + up + 1) >> 1;
+    if (a.group_start[mid] <= i) lo = mid; else up = mid - 1;
+  }
+  const int g = lo;
+  int gs = 0, m = 0, P = 0, leader = 0, seq = -1;
+  bool ok = shared_group(a, g, &gs, &m, &P, &leader) && gs <= i && i < gs + m;
+  if (ok) {
+    seq = a.group_seqs[i];
+    ok = seq >= 0 && seq < a.num_seqs;
+    if (ok) {
+      const int n = a.context_lens[seq];
+      ok = n > 0 && n <= a.len_cap && kBlockSize * P <= n - 1;
+    }
+  }
+  bool bad = false;
+  if (ok) {
+    const int32_t* lrow = a.block_tables + static_cast<size_t>(leader) * a.max_blocks_per_seq;
+    const int32_t* mrow = a.block_tables + static_cast<size_t>(seq) * a.max_blocks_per_seq;
+    for (int jb = tid; jb < P; jb += kFoldThreads) {
+      const int lb = __ldg(lrow + jb), mb = __ldg(mrow + jb);
+      bad |= !(lb >= 0 && lb < a.num_blocks && mb == lb);
+    }
+  }
+  ok = ok && !__syncthreads_or(bad);  // (ok was the same in every thread)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (!ok) {
+    if (blockIdx.y == 0 && tid == 0) seterr(a, kErrGroup);
+    return;
+  }
+  // (written by the plan kernel ahead of the pass: read through L2)
+  const int R = min(__ldcg(a.group_ranges + g), kMaxFoldRanges);
+  if (R <= 0) return;  // (a malformed group: nothing was computed for it)
+  if (h < Hq) {
+    const size_t pb = (static_cast<size_t>(i) * Hq + h) * a.max_ranges;
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kMaxFoldRanges; ++r)
+      if (r < R) M = fmaxf(M, __ldcg(&a.part_ml[pb + r].x));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r0 = 0; r0 < kMaxFoldRanges; r0 += kFoldBatch) {
+      if (r0 >= R) break;
+      float2 ml[kFoldBatch];
+      float4 o4[kFoldBatch];
+#pragma unroll
+      for (int r = 0; r < kFoldBatch; ++r) {
+        if (r0 + r < R) {
+          ml[r] = __ldcg(a.part_ml + pb + r0 + r);
+          o4[r] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (pb + r0 + r) * D) + d4);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kFoldBatch; ++r) {
+        if (r0 + r < R) {
+          const float w = ml[r].x == -INFINITY ? 0.f : exp2f(ml[r].x - M);
+          L = fmaf(w, ml[r].y, L);
+          acc.x = fmaf(w, o4[r].x, acc.x);
+          acc.y = fmaf(w, o4[r].y, acc.y);
+          acc.z = fmaf(w, o4[r].z, acc.z);
+          acc.w = fmaf(w, o4[r].w, acc.w);
+        }
+      }
+    }
+    const size_t orow = static_cast<size_t>(seq) * Hq + h;
+    reinterpret_cast<float4*>(a.pre_o + orow * D)[d4] = acc;
+    if (d4 == 0) a.pre_ml[orow] = make_float2(M, L);
+  }
+  if (blockIdx.y == 0 && tid == 0 && atomicCAS(a.claim + seq, 0, P) != 0) {
+    atomicExch(a.claim + seq, -1);
+    seterr(a, kErrGroup);
+  }
 }
 
 template <int D, int G, int MODE>
@@ -909,7 +1061,8 @@ size_t tc_smem_bytes(int head_dim) {
   const size_t q = static_cast<size_t>(kCols) * head_dim * 2;
   const size_t kv = static_cast<size_t>(kKeys) * head_dim * 2;
   const size_t p = static_cast<size_t>(kCols) * kKeys * 2;
-  return 1024 + q + 2 * kStages * kv + p + 128;  // (alignment slack, barriers)
+  // (alignment slack; barriers: 12 ring + 5 per tile + 2)
+  return 1024 + kPair * q + 2 * kStages * kv + kPair * p + 256;
 }
 
 std::mutex g_tc_mu;
@@ -930,17 +1083,14 @@ cudaError_t prepare(const void* fn, size_t smem) {
   return cudaSuccess;
 }
 
-// plan kernel, then the attention kernel behind it (programmatic dependent launch)
-cudaError_t launch_pair(const void* plan, const void* main, TcArgs& a, int grid, size_t smem,
-                        cudaStream_t stream) {
-  cudaError_t e = prepare(main, smem);
-  if (e != cudaSuccess) return e;
+// a launch behind the previous kernel of the stream with programmatic
+// dependent launch (the kernel waits for it with griddepcontrol.wait)
+cudaError_t launch_dependent(const void* fn, dim3 grid, int threads, size_t smem, TcArgs& a,
+                             cudaStream_t stream) {
   void* params[] = {&a};
-  if ((e = cudaLaunchKernel(plan, dim3(1), dim3(kPlanThreads), params, 0, stream)) != cudaSuccess)
-    return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -948,7 +1098,18 @@ cudaError_t launch_pair(const void* plan, const void* main, TcArgs& a, int grid,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, main, params);
+  return cudaLaunchKernelExC(&cfg, fn, params);
+}
+
+// plan kernel, then the attention kernel behind it
+cudaError_t launch_pair(const void* plan, const void* main, TcArgs& a, int grid, size_t smem,
+                        cudaStream_t stream) {
+  cudaError_t e = prepare(main, smem);
+  if (e != cudaSuccess) return e;
+  void* params[] = {&a};
+  if ((e = cudaLaunchKernel(plan, dim3(1), dim3(kPlanThreads), params, 0, stream)) != cudaSuccess)
+    return e;
+  return launch_dependent(main, dim3(grid), kThreads, smem, a, stream);
 }
 
 }  // namespace
@@ -958,13 +1119,14 @@ bool tc_prefill_supported(int head_dim, int group) {
   return pick<kModePrefill>(head_dim, group, &p, &m);
 }
 
-// Most work units a prefill call can have: each sequence's column tiles,
-// ceil(Q_s * G / 128) <= Q_s * G / 128 + 1, for every KV head.
+// Most work units a prefill call can have: each sequence's pairs of column
+// tiles, ceil(Q_s * G / 256) <= Q_s * G / 256 + 1, for every KV head.
 static long long prefill_max_units(int num_seqs, int num_query_tokens, int num_q_heads,
                                    int num_kv_heads) {
   const long long G = num_q_heads / num_kv_heads;
   return static_cast<long long>(num_kv_heads) *
-         ((static_cast<long long>(num_query_tokens) * G + kCols - 1) / kCols + num_seqs);
+         ((static_cast<long long>(num_query_tokens) * G + kPair * kCols - 1) / (kPair * kCols) +
+          num_seqs);
 }
 static size_t prefill_records_offset(int num_seqs) {
   return ((static_cast<size_t>(num_seqs) + 1) * sizeof(int) + 255) / 256 * 256;
@@ -972,9 +1134,10 @@ static size_t prefill_records_offset(int num_seqs) {
 
 size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_heads,
                                   int num_kv_heads) {
+  // unit starts, then the records twice (sorted; in row order)
   return prefill_records_offset(num_seqs) +
          static_cast<size_t>(prefill_max_units(num_seqs, num_query_tokens, num_q_heads,
-                                               num_kv_heads)) * 2 * sizeof(int4);
+                                               num_kv_heads)) * 4 * sizeof(int4);
 }
 
 int tc_launch_smem(int head_dim) { return static_cast<int>(tc_smem_bytes(head_dim)); }
@@ -1002,7 +1165,8 @@ cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_
   a.units = reinterpret_cast<int4*>(static_cast<char*>(l.workspace) +
                                     prefill_records_offset(l.num_seqs));
   a.max_units = static_cast<int>(std::min<long long>(
-      prefill_max_units(l.num_seqs, l.num_query_rows, l.num_q_heads, l.num_kv_heads), 1 << 30));
+      prefill_max_units(l.num_seqs, l.num_query_rows, l.num_q_heads, l.num_kv_heads), 1 << 28));
+  a.units_raw = a.units + 2 * static_cast<size_t>(a.max_units);
   a.err_flag = l.err_flag;
   a.tm_k = *l.tm_k;
   a.tm_v = *l.tm_v;
@@ -1036,21 +1200,12 @@ cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaSt
   a.oob_row = l.num_blocks * l.num_kv_heads * kBlockSize;
   a.scale_log2 = l.scale_log2;
   a.max_ranges = l.max_ranges;
-  // ranges of shared blocks: whole K/V tiles, at least 4 of them, and about
-  // enough units to fill the SMs from the fewest column tiles the groups form
-  const long long tiles =
-      std::max(1LL, (static_cast<long long>(l.num_listed) * group + kCols - 1) / kCols);
-  const long long per = std::max(1LL, num_sms / (tiles * l.num_kv_heads));
-  long long rb = (l.max_blocks_per_seq + per - 1) / per;
-  rb = std::max<long long>(rb, 4 * kTileBlocks);
-  rb = (rb + kTileBlocks - 1) / kTileBlocks * kTileBlocks;
-  // ... and no more ranges than the partial arrays hold
-  while ((l.max_blocks_per_seq + rb - 1) / rb > l.max_ranges) rb += kTileBlocks;
-  a.range_blocks = static_cast<int>(rb);
+  a.num_sms = num_sms;
   a.unit_start = l.unit_start;
   a.units = l.units;
   a.max_units = l.max_units;
-  a.counters = l.counters;
+  a.units_raw = l.units + 2 * static_cast<size_t>(l.max_units);
+  a.group_ranges = l.group_ranges;
   a.claim = l.claim;
   a.part_ml = l.part_ml;
   a.part_o = l.part_o;
@@ -1059,7 +1214,14 @@ cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaSt
   a.err_flag = l.err_flag;
   a.tm_k = *l.tm_k;
   a.tm_v = *l.tm_v;
-  return launch_pair(plan, main, a, num_sms, tc_smem_bytes(l.head_dim), stream);
+  cudaError_t e = launch_pair(plan, main, a, num_sms, tc_smem_bytes(l.head_dim), stream);
+  if (e != cudaSuccess || l.num_listed == 0) return e;
+  // the fold: one CTA per (listed member, slice of kFoldThreads / (D / 4) heads)
+  const int hpc = kFoldThreads / (l.head_dim / 4);
+  const void* fold = l.head_dim == 64 ? reinterpret_cast<const void*>(&tc_fold_kernel<64>)
+                                      : reinterpret_cast<const void*>(&tc_fold_kernel<128>);
+  return launch_dependent(fold, dim3(l.num_listed, (l.num_q_heads + hpc - 1) / hpc), kFoldThreads,
+                          0, a, stream);
 }
 
 }  // namespace pa

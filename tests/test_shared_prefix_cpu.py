@@ -145,6 +145,7 @@ def test_shared_prefix_decode_rejects_bad_arguments_on_the_host(lib):
     assert shared_call(lib, Hq=6) == ops.PA_ERR_UNSUPPORTED               # 3 heads per KV head
     assert shared_call(lib, gs=None) == ops.PA_ERR_INVALID_ARG
     assert shared_call(lib, ng=20000) == ops.PA_ERR_UNSUPPORTED
+    assert shared_call(lib, ng=5, nl=4) == ops.PA_ERR_INVALID_ARG          # more groups than listed
     assert shared_call(lib, q=P(8)) == ops.PA_ERR_INVALID_ARG            # misaligned
     assert shared_call(lib, scale=float("nan")) == ops.PA_ERR_INVALID_ARG
     assert shared_call(lib, S=0) == ops.PA_OK                             # nothing to do
