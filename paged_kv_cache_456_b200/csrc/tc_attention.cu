@@ -84,6 +84,13 @@ constexpr int kPlanRowsOnChip = 4096;           // unit starts the plan kernel k
 constexpr int kMaxFoldRanges = 16;              // shared: ranges of a group's shared blocks, at most
 constexpr int kModePrefill = 0;
 constexpr int kModeShared = 1;
+// P (the bf16 weights) goes to tensor memory over the S columns it was made
+// from, and the P.V MMA takes its A operand from there (1), or through a
+// shared-memory tile per column tile (0).
+#ifndef PA_TC_P_TMEM
+#define PA_TC_P_TMEM 1
+#endif
+constexpr bool kPInTmem = PA_TC_P_TMEM != 0;
 
 struct TcArgs {
   const __nv_bfloat16* q;
@@ -207,13 +214,40 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     *rb = b;
     return (P + b - 1) / b;
   };
+  if constexpr (MODE == kModePrefill) {
+    // every block a computable sequence attends to must be a block of the
+    // cache; one with a bad id gets no units, its rows are zeroed here and
+    // the error bit is set (one warp per sequence; the verdict goes through
+    // unit_start, overwritten below)
+    for (int r = warp; r < R; r += kPlanThreads / 32) {
+      int q0 = 0, Q = 0, n = 0, bit = 0;
+      bool bad = false;
+      if (prefill_seq(a, r, &q0, &Q, &n, &bit)) {
+        const int32_t* trow = a.block_tables + static_cast<size_t>(r) * a.max_blocks_per_seq;
+        const int nb = (n + kBlockSize - 1) / kBlockSize;
+        for (int b = lane; b < nb; b += 32) {
+          const int phys = __ldg(trow + b);
+          bad |= !(phys >= 0 && phys < a.num_blocks);
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad) {
+          if (lane == 0) seterr(a, kErrBlockId);
+          uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(q0) * Hq * D);
+          const size_t cnt = static_cast<size_t>(Q) * Hq * D * 2 / 16;
+          for (size_t i = lane; i < cnt; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (lane == 0) a.unit_start[r] = bad ? 1 : 0;
+    }
+    __syncthreads();
+  }
   int local = 0;
   for (int r = r0; r < r1; ++r) {
     int units = 0;
     if constexpr (MODE == kModePrefill) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
       if (prefill_seq(a, r, &q0, &Q, &n, &bit)) {
-        units = Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair);
+        if (a.unit_start[r] == 0) units = Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair);
       } else if (bit) {
         seterr(a, bit);
         if (bit != kErrQuery || (a.query_start[r] >= 0 && a.query_start[r] <= a.query_start[r + 1] &&
@@ -445,17 +479,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   unsigned char* sQ = sm;                    // [kPair][QT]
   unsigned char* sK = sQ + kPair * QT;       // [kStages][KT]
   unsigned char* sV = sK + kStages * KT;     // [kStages][KT]
-  unsigned char* sP = sV + kStages * KT;     // [kPair][PT]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPair * PT);
+  unsigned char* sP = sV + kStages * KT;     // [kPair][PT] (P through shared memory only)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + (kPInTmem ? 0 : kPair * PT));
   // barriers: kfull[3] kempty[3] vfull[3] vempty[3] | per tile t: sfull[t][2],
-  // pfull[t], odone[t], sync[t] | qfull drain
+  // pfull[t], odone[t] | qfull drain
   const uint32_t b0 = smem_addr(bars);
   const uint32_t KFULL = b0, KEMPTY = b0 + 24, VFULL = b0 + 48, VEMPTY = b0 + 72;
-  const uint32_t TB = b0 + 96;  // tile t's barriers at TB + 40 t: sfull[2], pfull, odone, sync
-  const uint32_t QFULL = b0 + 96 + 40 * kPair, DRAIN = QFULL + 8;
+  const uint32_t TB = b0 + 96;  // tile t's barriers at TB + 32 t: sfull[2], pfull, odone
+  const uint32_t QFULL = b0 + 96 + 32 * kPair, DRAIN = QFULL + 8;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_red[kPair][3];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Hq = a.num_q_heads, Hkv = a.num_kv_heads;
@@ -468,12 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       mbar_init(VEMPTY + 8 * i, 1);
     }
     for (int t = 0; t < kPair; ++t) {
-      mbar_init(TB + 40 * t, 1);        // sfull[0]
-      mbar_init(TB + 40 * t + 8, 1);    // sfull[1]
-      mbar_init(TB + 40 * t + 16, kWgThreads);  // pfull
-      mbar_init(TB + 40 * t + 24, 1);   // odone
-      mbar_init(TB + 40 * t + 32, kWgThreads);  // sync (the tile's warpgroup among itself)
-      s_red[t][0] = s_red[t][1] = s_red[t][2] = 0;
+      mbar_init(TB + 32 * t, 1);        // sfull[0]
+      mbar_init(TB + 32 * t + 8, 1);    // sfull[1]
+      mbar_init(TB + 32 * t + 16, kWgThreads);  // pfull
+      mbar_init(TB + 32 * t + 24, 1);   // odone
     }
     mbar_init(QFULL, kSoftmaxThreads);
     mbar_init(DRAIN, 1);
@@ -582,82 +613,102 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     // ---------------- MMA issuer -------------------------------------------------
     // Per K/V tile j: S_A(j), S_B(j) were issued two tiles ahead; as each
     // warpgroup releases P_t(j): O_t += P_t(j) V(j), then S_t(j + 2) into the
-    // S buffer P_t(j) has freed.
-    if (lane == 0) {
-      int kidx = 0, vidx = 0, qidx = 0;
-      int sidx[kPair] = {0, 0}, pidx[kPair] = {0, 0};
-      bool ok = true;
-      const uint32_t qbase = smem_addr(sQ), pbase = smem_addr(sP);
-      // S_t of the K tile in ring slot kidx (its K has landed)
-      auto issue_s = [&](int t) {
-        const uint32_t kbase = smem_addr(sK + (kidx % kStages) * KT);
-        const uint32_t dS = tmem + t * 2 * kKeys + (sidx[t] & 1) * kKeys;
+    // S buffer P_t(j) has freed.  The whole warp runs the loop, so that the
+    // descriptors it computes are warp-uniform, and one elected lane issues
+    // each MMA and commit (always the same lane: the warp stays converged, and
+    // a commit tracks the MMAs of the thread that issues it).
+    int kidx = 0, vidx = 0, qidx = 0;
+    int sidx[kPair] = {0, 0}, pidx[kPair] = {0, 0};
+    bool ok = true;
+    const uint32_t qbase = smem_addr(sQ), pbase = smem_addr(sP);
+    auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    auto mma = [&](uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+      if (tc::elect_one()) tc::mma_bf16_ss(d, adesc, bdesc, idesc, acc);
+    };
+    auto mma_ts = [&](uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+      if (tc::elect_one()) tc::mma_bf16_ts(d, a_tmem, bdesc, idesc, acc);
+    };
+    auto commit = [&](uint32_t bar) {
+      if (tc::elect_one()) tc::commit(bar);
+    };
+    // S_t of the K tile in ring slot kidx (its K has landed)
+    auto issue_s = [&](int t) {
+      const uint32_t kbase = smem_addr(sK + (kidx % kStages) * KT);
+      const uint32_t dS = tmem + t * 2 * kKeys + (sidx[t] & 1) * kKeys;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k / 4) * (kCols * 128) + (k % 4) * 32;
-          const uint32_t koff = (k / 4) * HALF + (k % 4) * 32;
-          tc::mma_bf16_ss(dS, tc::sdesc_sw128(qbase + t * QT + off, 16, 1024),
-                          tc::sdesc_sw128(kbase + koff, 16, 1024), IDESC_S, k > 0);
-        }
-        tc::commit(TB + 40 * t + 8 * (sidx[t] & 1));
-        ++sidx[t];
-      };
-      auto k_landed = [&]() -> bool {
-        if (!mbar_wait_bounded(KFULL + 8 * (kidx % kStages), (kidx / kStages) & 1)) return false;
-        tc::fence_after_sync();
-        return true;
-      };
-      auto k_done = [&]() {  // both tiles' S of this K tile issued: its slot frees on completion
-        tc::commit(KEMPTY + 8 * (kidx % kStages));
-        ++kidx;
-      };
-      Unit x, nx;
-      if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
-      for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
-        if (unit_of(k + 1) < total) load_unit<MODE>(a, unit_of(k + 1), &nx);
-        if (aborted_one() || !mbar_wait_bounded(QFULL, qidx & 1)) { ok = false; break; }
-        ++qidx;
-        tc::fence_after_sync();
-        for (int j = 0; j < 2 && j < x.nt && ok; ++j) {
-          if (!(ok = k_landed())) break;
-          issue_s(0);
-          issue_s(1);
-          k_done();
-        }
-        for (int j = 0; j < x.nt && ok; ++j) {
-          const int st = vidx % kStages;
-          const uint32_t vbase = smem_addr(sV + st * KT);
-          const bool ahead = j + 2 < x.nt;
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k / 4) * (kCols * 128) + (k % 4) * 32;
+        const uint32_t koff = (k / 4) * HALF + (k % 4) * 32;
+        mma(dS, tc::sdesc_sw128(qbase + t * QT + off, 16, 1024),
+            tc::sdesc_sw128(kbase + koff, 16, 1024), IDESC_S, k > 0);
+      }
+      commit(TB + 32 * t + 8 * (sidx[t] & 1));
+      ++sidx[t];
+    };
+    auto k_landed = [&]() -> bool {
+      if (!wait_all(KFULL + 8 * (kidx % kStages), (kidx / kStages) & 1)) return false;
+      tc::fence_after_sync();
+      return true;
+    };
+    auto k_done = [&]() {  // both tiles' S of this K tile issued: its slot frees on completion
+      commit(KEMPTY + 8 * (kidx % kStages));
+      ++kidx;
+    };
+    Unit x, nx;
+    if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
+    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
+      if (unit_of(k + 1) < total) load_unit<MODE>(a, unit_of(k + 1), &nx);
+      if (aborted() || !wait_all(QFULL, qidx & 1)) { ok = false; break; }
+      ++qidx;
+      tc::fence_after_sync();
+      for (int j = 0; j < 2 && j < x.nt && ok; ++j) {
+        if (!(ok = k_landed())) break;
+        issue_s(0);
+        issue_s(1);
+        k_done();
+      }
+      for (int j = 0; j < x.nt && ok; ++j) {
+        const int st = vidx % kStages;
+        const uint32_t vbase = smem_addr(sV + st * KT);
+        const bool ahead = j + 2 < x.nt;
 #pragma unroll
-          for (int t = 0; t < kPair; ++t) {
-            if (aborted_one() || !mbar_wait_bounded(TB + 40 * t + 16, pidx[t] & 1)) { ok = false; break; }
-            ++pidx[t];
-            if (t == 0 && !mbar_wait_bounded(VFULL + 8 * st, (vidx / kStages) & 1)) { ok = false; break; }
-            tc::fence_after_sync();
+        for (int t = 0; t < kPair; ++t) {
+          if (aborted() || !wait_all(TB + 32 * t + 16, pidx[t] & 1)) { ok = false; break; }
+          // (P of this tile sits in the S buffer its S used: S and P.V go in the same order)
+          const uint32_t pa = tmem + t * 2 * kKeys + (pidx[t] & 1) * kKeys;
+          ++pidx[t];
+          if (t == 0 && !wait_all(VFULL + 8 * st, (vidx / kStages) & 1)) { ok = false; break; }
+          tc::fence_after_sync();
 #pragma unroll
-            for (int k = 0; k < kKeys / 16; ++k)
-              tc::mma_bf16_ss(tmem + 2 * kPair * kKeys + t * D,
-                              tc::sdesc_sw128(pbase + t * PT + k * 32, 16, 1024),
-                              tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
-                              (j > 0 || k > 0) ? 1u : 0u);
-            tc::commit(TB + 40 * t + 24);  // odone[t]
-            if (t == kPair - 1) {
-              tc::commit(VEMPTY + 8 * st);
-              ++vidx;
-            }
-            if (ahead) {
-              if (t == 0 && !(ok = k_landed())) break;
-              issue_s(t);
-              if (t == kPair - 1) k_done();
-            }
+          for (int k = 0; k < kKeys / 16; ++k) {
+            if constexpr (kPInTmem)
+              mma_ts(tmem + 2 * kPair * kKeys + t * D, pa + k * 8,
+                     tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
+                     (j > 0 || k > 0) ? 1u : 0u);
+            else
+              mma(tmem + 2 * kPair * kKeys + t * D, tc::sdesc_sw128(pbase + t * PT + k * 32, 16, 1024),
+                  tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
+                  (j > 0 || k > 0) ? 1u : 0u);
+          }
+          commit(TB + 32 * t + 24);  // odone[t]
+          if (t == kPair - 1) {
+            commit(VEMPTY + 8 * st);
+            ++vidx;
+          }
+          if (ahead) {
+            if (t == 0 && !(ok = k_landed())) break;
+            issue_s(t);
+            if (t == kPair - 1) k_done();
           }
         }
       }
-      if (!ok) timeout();
-      // every MMA issued has completed before the TMEM can be freed
-      tc::commit(DRAIN);
-      mbar_wait_bounded(DRAIN, 0);
     }
+    if (!ok) timeout();
+    // every MMA issued has completed before the TMEM can be freed
+    commit(DRAIN);
+    wait_all(DRAIN, 0);
     __syncwarp();
   } else {
     // ---------------- softmax: warpgroup t = warp / 4 serves column tile 2 pr + t;
@@ -665,30 +716,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     const int t = warp / 4, col = tid % kWgThreads;
     const int h = col % G;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-    const uint32_t SFULL = TB + 40 * t, PFULL = SFULL + 16, ODONE = SFULL + 24, SYNC = SFULL + 32;
+    const uint32_t SFULL = TB + 32 * t, PFULL = SFULL + 16, ODONE = SFULL + 24;
     const uint32_t s_col = t * 2 * kKeys, o_col = 2 * kPair * kKeys + t * D;  // TMEM columns
     unsigned char* const myQ = sQ + t * QT;
     unsigned char* const myP = sP + t * PT;
-    int sidx = 0, oidx = 0, tile = 0, syncs = 0, reds = 0;
+    int sidx = 0, oidx = 0, tile = 0;
     bool ok = true;
     // a bounded wait whose outcome the whole warp shares, so that no lane
     // leaves ahead of the others (the TMEM moves are warp-wide)
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
-    };
-    auto group_sync = [&]() -> bool {  // the 128 threads of this warpgroup
-      mbar_arrive(SYNC);
-      return wait_all(SYNC, (syncs++) & 1);
-    };
-    // OR of a flag over the warpgroup; slot reds % 3 is cleared two uses ahead
-    auto group_or = [&](bool v, bool* res) -> bool {
-      const int slot = reds % 3;
-      if (v) atomicOr(&s_red[t][slot], 1);
-      if (!group_sync()) return false;
-      *res = *reinterpret_cast<volatile int*>(&s_red[t][slot]) != 0;
-      if (col == 0) s_red[t][(reds + 2) % 3] = 0;
-      ++reds;
-      return true;
     };
     // this column's query row in unit y (-1: none), and the keys it sees
     auto column_of = [&](const Unit& y, int* kend) -> int {
@@ -729,18 +766,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       if (has_next) load_unit<MODE>(a, unit_of(k + 1), &nx);
       int kend;
       const int qrow = column_of(x, &kend);
-      // ---- the unit's blocks must be in range (prefill: a bad one empties the sequence)
-      bool bad = false;
-      if constexpr (MODE == kModePrefill) {
-        const int nb = (x.n + kBlockSize - 1) / kBlockSize;
-        const int32_t* trow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
-        for (int b = col; b < nb; b += kWgThreads) {
-          const int phys = __ldg(trow + b);
-          bad |= !(phys >= 0 && phys < a.num_blocks);
-        }
-        if (!group_or(bad, &bad)) { ok = false; break; }
-        if (bad && col == 0 && t == 0) seterr(a, kErrBlockId);
-      }
+      // (a prefill sequence with a block id out of range has no units: the
+      // plan kernel zeroed its rows; a shared group's blocks are checked by
+      // the fold, and a bad id here only reads the tensor loads' zero fill)
       // ---- Q: requested now, or already during the previous unit's last tile
       if (!q_issued) load_q(x, qrow);
       q_issued = false;
@@ -754,7 +782,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         if (aborted() || !wait_all(SFULL + 8 * (sidx & 1), (sidx >> 1) & 1)) { ok = false; break; }
         tc::fence_after_sync();
         uint32_t sv[kKeys];
-        tc::tmem_ld64(lane_base + s_col + (sidx & 1) * kKeys, sv);
+        const uint32_t s_addr = lane_base + s_col + (sidx & 1) * kKeys;
+        tc::tmem_ld64(s_addr, sv);
         tc::tmem_wait_ld(sv);
         ++sidx;
         if (j == x.nt - 1 && has_next) {
@@ -763,19 +792,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           load_q(nx, column_of(nx, &kn));
           q_issued = true;
         }
-        // scale to log2 units, mask the keys this column does not see, and take
-        // the maximum over 8 independent chains
+        // the maximum over 8 independent chains of the scores in log2 units.
+        // A tile the column sees whole, with a positive scale: the maximum of
+        // the raw scores times the scale (the rounded product is monotonic, so
+        // it is the maximum of the rounded scaled scores), and the scale goes
+        // into the exponent's fma below.  Otherwise the scores are scaled here
+        // and the keys the column does not see are set to -inf.
         const int kb = x.k0 + j * kKeys;
         float m8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
-        if (kb + kKeys <= kend) {
+        float mul = 1.f;  // score in log2 units = sv * mul
+        if (kb + kKeys <= kend && a.scale_log2 > 0.f) {
 #pragma unroll
-          for (int k = 0; k < kKeys; ++k) {
-            const float v = __uint_as_float(sv[k]) * a.scale_log2;
-            sv[k] = __float_as_uint(v);
-            m8[k & 7] = fmaxf(m8[k & 7], v);
-          }
+          for (int k = 0; k < kKeys; ++k) m8[k & 7] = fmaxf(m8[k & 7], __uint_as_float(sv[k]));
+          mul = a.scale_log2;
         } else {
 #pragma unroll
           for (int k = 0; k < kKeys; ++k) {
@@ -785,13 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           }
         }
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        if (j > 0) {
-          // O of the previous tile is complete: its P slot is free and O is stable
-          if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
-          ++oidx;
-          tc::fence_after_sync();
-        }
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * mul;
         const bool grow = mx > m_run + kRescaleThreshold;
         float al = 1.f;
         if (grow) {
@@ -800,29 +825,46 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           m_run = mx;
         }
         // weights, rounded to bf16 for the product; the sum (8 chains) takes
-        // them as rounded
+        // them as rounded.  In tensor memory they go over the S columns just
+        // read; through shared memory they are computed while the previous
+        // tile's P.V may still be reading the P slot, and stored once it is done.
         const bool none = m_run == -INFINITY;
+        const float nm = -m_run;
         const uint32_t pb = smem_addr(myP) + col * 128;
         float l8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) l8[c] = 0.f;
+        uint32_t w[kKeys / 2];
 #pragma unroll
-        for (int c = 0; c < kKeys / 8; ++c) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = none ? 0.f : ex2_fast(__uint_as_float(sv[c * 8 + 2 * e]) - m_run);
-            const float p1 = none ? 0.f : ex2_fast(__uint_as_float(sv[c * 8 + 2 * e + 1]) - m_run);
-            const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-            l8[2 * e] += __low2float(pp);
-            l8[2 * e + 1] += __high2float(pp);
-            w[e] = *reinterpret_cast<const uint32_t*>(&pp);
-          }
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + (((c % 8) ^ (col % 8)) << 4)),
-                       "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                       : "memory");
+        for (int e = 0; e < kKeys / 2; ++e) {
+          const float p0 = none ? 0.f : ex2_fast(fmaf(__uint_as_float(sv[2 * e]), mul, nm));
+          const float p1 = none ? 0.f : ex2_fast(fmaf(__uint_as_float(sv[2 * e + 1]), mul, nm));
+          const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+          l8[(2 * e) & 7] += __low2float(pp);
+          l8[(2 * e + 1) & 7] += __high2float(pp);
+          w[e] = *reinterpret_cast<const uint32_t*>(&pp);
         }
         l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        if constexpr (kPInTmem) {
+          uint32_t w32[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w32[e] = w[e];
+          tc::tmem_st32(s_addr, w32);
+          tc::tmem_wait_st();
+        }
+        if (j > 0) {
+          // O of the previous tile is complete: its P slot is free and O is stable
+          if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
+          ++oidx;
+          tc::fence_after_sync();
+        }
+        if constexpr (!kPInTmem) {
+#pragma unroll
+          for (int c = 0; c < kKeys / 8; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + (((c % 8) ^ (col % 8)) << 4)),
+                         "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
+                         : "memory");
+        }
         if constexpr (MODE == kModePrefill) {
           // rows past the sequence's end in its last block hold stale data: a
           // zero weight times a NaN would still poison O, so tile A's
@@ -870,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       tc::fence_after_sync();
       if constexpr (MODE == kModePrefill) {
         // (every lane runs the warp-wide TMEM loads; only live columns store)
-        const float inv = bad ? 0.f : 1.f / l_run;
+        const float inv = 1.f / l_run;
         uint4* dst = reinterpret_cast<uint4*>(
             a.out + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + x.kvh * G + h) * D);
 #pragma unroll
@@ -1061,8 +1103,8 @@ size_t tc_smem_bytes(int head_dim) {
   const size_t q = static_cast<size_t>(kCols) * head_dim * 2;
   const size_t kv = static_cast<size_t>(kKeys) * head_dim * 2;
   const size_t p = static_cast<size_t>(kCols) * kKeys * 2;
-  // (alignment slack; barriers: 12 ring + 5 per tile + 2)
-  return 1024 + kPair * q + 2 * kStages * kv + kPair * p + 256;
+  // (alignment slack; barriers: 12 ring + 4 per tile + 2)
+  return 1024 + kPair * q + 2 * kStages * kv + (kPInTmem ? 0 : kPair * p) + 256;
 }
 
 std::mutex g_tc_mu;
