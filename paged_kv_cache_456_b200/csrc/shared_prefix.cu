@@ -535,8 +535,8 @@ Layout layout(int num_seqs, int num_listed, int num_q_heads, int head_dim,
   l.units = round_up(l.group_ranges + static_cast<size_t>(num_listed) * sizeof(int), 256);
   l.max_units = ((static_cast<long long>(num_listed) * num_q_heads + 127) / 128 +
                  static_cast<long long>(num_listed) * num_q_heads) * l.max_ranges;
-  // (the records twice: sorted, and in group order)
-  l.bytes = round_up(l.units + static_cast<size_t>(l.max_units) * 64, 256);
+  // (a record is two int4)
+  l.bytes = round_up(l.units + static_cast<size_t>(l.max_units) * 32, 256);
   return l;
 }
 

@@ -112,7 +112,6 @@ struct TcArgs {
   float scale_log2;
   int* unit_start;                  // [rows + 1] work units before each sequence / group
   int4* units;                      // [max_units][2] one record per work unit, longest first
-  int4* units_raw;                  // [max_units][2] the same records in row order (plan kernel)
   int max_units;
   int* group_ranges;                // shared: [groups] ranges of each group (0: none folded)
   int* claim;                       // shared: [num_seqs] blocks attended per sequence
@@ -214,11 +213,19 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     *rb = b;
     return (P + b - 1) / b;
   };
+  // per-row scratch (unit counts, then unit starts): on chip when the rows
+  // fit, else in unit_start; the attention kernel reads only unit_start[R]
+  __shared__ int s_us[kPlanRowsOnChip + 1];
+  const bool on_chip = R <= kPlanRowsOnChip;
+  auto row_set = [&](int r, int v) {
+    if (on_chip) s_us[r] = v; else a.unit_start[r] = v;
+  };
+  auto row_get = [&](int r) -> int { return on_chip ? s_us[r] : __ldcg(a.unit_start + r); };
   if constexpr (MODE == kModePrefill) {
     // every block a computable sequence attends to must be a block of the
     // cache; one with a bad id gets no units, its rows are zeroed here and
     // the error bit is set (one warp per sequence; the verdict goes through
-    // unit_start, overwritten below)
+    // the row scratch, overwritten below)
     for (int r = warp; r < R; r += kPlanThreads / 32) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
       bool bad = false;
@@ -237,7 +244,7 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
           for (size_t i = lane; i < cnt; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
         }
       }
-      if (lane == 0) a.unit_start[r] = bad ? 1 : 0;
+      if (lane == 0) row_set(r, bad ? 1 : 0);
     }
     __syncthreads();
   }
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     if constexpr (MODE == kModePrefill) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
       if (prefill_seq(a, r, &q0, &Q, &n, &bit)) {
-        if (a.unit_start[r] == 0) units = Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair);
+        if (row_get(r) == 0) units = Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair);
       } else if (bit) {
         seterr(a, bit);
         if (bit != kErrQuery || (a.query_start[r] >= 0 && a.query_start[r] <= a.query_start[r + 1] &&
@@ -271,7 +278,7 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
       }
       a.group_ranges[r] = Rg;
     }
-    a.unit_start[r] = units;  // (turned into starts below)
+    row_set(r, units);  // (turned into starts below)
     local += units;
   }
   int incl = local;
@@ -289,41 +296,40 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     total += s_wsum[w];
   }
   for (int r = r0; r < r1; ++r) {
-    const int units = a.unit_start[r];
-    a.unit_start[r] = run;
+    const int units = row_get(r);
+    row_set(r, run);
     // (a group whose units do not all fit the workspace is not folded)
     if (MODE == kModeShared && run + units > a.max_units) a.group_ranges[r] = 0;
     run += units;
   }
-  if (tid == 0) a.unit_start[R] = total;
+  // (the workspace is sized for the most units a call can have)
+  const int T = min(total, a.max_units);
+  if (tid == 0) {
+    row_set(R, total);
+    a.unit_start[R] = T;
+    if (total > a.max_units) seterr(a, kErrTimeout);
+  }
   __syncthreads();
-  // each unit as a record {row, kv head | pair of column tiles << 16, first
+  // Each unit as a record {row, kv head | pair of column tiles << 16, first
   // key, last key + 1} {prefill: first query row, rows, context length, 0 |
-  // shared: first member, members, shared blocks, range | ranges << 16},
-  // written by all threads (each finds its unit's row by a search over the
-  // unit starts, kept on chip when they fit), so that the attention kernel
-  // finds a unit with one load instead of a search
-  __shared__ int s_us[kPlanRowsOnChip + 1];
-  const bool on_chip = R <= kPlanRowsOnChip;
-  if (on_chip)
-    for (int r = tid; r <= R; r += kPlanThreads) s_us[r] = __ldcg(a.unit_start + r);
-  __syncthreads();
-  auto start_of = [&](int r) -> int { return on_chip ? s_us[r] : __ldcg(a.unit_start + r); };
-  for (int u = tid; u < min(total, a.max_units); u += kPlanThreads) {
-    int lo = 0, up = R - 1;  // largest row with start_of(row) <= u
+  // shared: first member, members, shared blocks, range | ranges << 16}, so
+  // that the attention kernel finds a unit with one load instead of a search.
+  // A thread finds unit u's row by a search over the unit starts.
+  auto record = [&](int u, int4* x0, int4* x1) {
+    int lo = 0, up = R - 1;  // largest row with row_get(row) <= u
     while (lo < up) {
       const int mid = (lo + up + 1) >> 1;
-      if (start_of(mid) <= u) lo = mid; else up = mid - 1;
+      if (row_get(mid) <= u) lo = mid; else up = mid - 1;
     }
-    const int r = lo, k = u - start_of(lo);
+    const int r = lo, k = u - row_get(lo);
     if constexpr (MODE == kModePrefill) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
       prefill_seq(a, r, &q0, &Q, &n, &bit);  // (true: only such rows have units)
       const int npair = ((Q + RPT - 1) / RPT + kPair - 1) / kPair;
       const int pr = k % npair, kvh = k / npair;
       const int jl = min(Q, (pr + 1) * kPair * RPT) - 1;  // the pair's last query row
-      a.units_raw[2 * u] = make_int4(r, kvh | (pr << 16), 0, n - Q + jl + 1);
-      a.units_raw[2 * u + 1] = make_int4(q0, Q, n, 0);
+      *x0 = make_int4(r, kvh | (pr << 16), 0, n - Q + jl + 1);
+      *x1 = make_int4(q0, Q, n, 0);
     } else {
       int gs, m, P, leader;
       shared_group(a, r, &gs, &m, &P, &leader);  // (true: only such groups have units)
@@ -332,34 +338,34 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
       const int Rr = ranges_of(P, &rb);
       const int pr = k % npair, kvh = (k / npair) % Hkv, rr = k / (npair * Hkv);
       const int k1 = min(P, (rr + 1) * rb) * kBlockSize;
-      a.units_raw[2 * u] = make_int4(leader, kvh | (pr << 16), rr * rb * kBlockSize, k1);
-      a.units_raw[2 * u + 1] = make_int4(gs, m, P, rr | (Rr << 16));
+      *x0 = make_int4(leader, kvh | (pr << 16), rr * rb * kBlockSize, k1);
+      *x1 = make_int4(gs, m, P, rr | (Rr << 16));
     }
-  }
-  if (tid == 0) {
-    // (the workspace is sized for the most units a call can have)
-    if (total > a.max_units) seterr(a, kErrTimeout);
-    if (total > a.max_units) a.unit_start[R] = a.max_units;
-  }
+  };
   // Units differ in length (a causal tile's keys end at its last row; ranges
   // and sequences differ), and the attention kernel deals them to its CTAs in
   // rounds, so they are ordered longest first (a counting sort by K/V tiles)
-  // and the CTAs take them in snake order: that spreads the long ones.
+  // and the CTAs take them in snake order: that spreads the long ones.  The
+  // records are made twice -- for the histogram, then to be written straight
+  // to their place -- rather than stored and read back.
   __shared__ int s_hist[kSortBuckets];
   __shared__ int s_pos[kSortBuckets];
-  const int T = min(total, a.max_units);
   for (int b = tid; b < kSortBuckets; b += kPlanThreads) s_hist[b] = 0;
-  __syncthreads();  // (also: every thread's raw records are written)
-  auto bucket = [&](int u) -> int {
-    const int4 r0 = __ldcg(a.units_raw + 2 * u);
-    const int nt = (r0.w - r0.z + kKeys - 1) / kKeys;
+  __syncthreads();
+  auto bucket_of = [](const int4& x0) -> int {
+    const int nt = (x0.w - x0.z + kKeys - 1) / kKeys;
     return nt < kSortBuckets - 1 ? nt : kSortBuckets - 1;
   };
   // (lanes with the same bucket add together: one shared-memory atomic per
   // distinct bucket and warp, not one per unit -- equal lengths are common)
   const int Tw = (T + 31) / 32 * 32;
   for (int u = tid; u < Tw; u += kPlanThreads) {
-    const int b = u < T ? bucket(u) : -1;
+    int b = -1;
+    if (u < T) {
+      int4 x0, x1;
+      record(u, &x0, &x1);
+      b = bucket_of(x0);
+    }
     const unsigned same = __match_any_sync(0xffffffffu, b);
     if (b >= 0 && lane == __ffs(same) - 1) atomicAdd(&s_hist[b], __popc(same));
   }
@@ -388,7 +394,12 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
   }
   __syncthreads();
   for (int u = tid; u < Tw; u += kPlanThreads) {
-    const int b = u < T ? bucket(u) : -1;
+    int b = -1;
+    int4 x0, x1;
+    if (u < T) {
+      record(u, &x0, &x1);
+      b = bucket_of(x0);
+    }
     const unsigned same = __match_any_sync(0xffffffffu, b);
     const int leader = __ffs(same) - 1;
     int base = 0;
@@ -396,8 +407,8 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     base = __shfl_sync(0xffffffffu, base, leader);
     if (b >= 0) {
       const int pos = base + __popc(same & ((1u << lane) - 1));
-      a.units[2 * pos] = __ldcg(a.units_raw + 2 * u);
-      a.units[2 * pos + 1] = __ldcg(a.units_raw + 2 * u + 1);
+      a.units[2 * pos] = x0;
+      a.units[2 * pos + 1] = x1;
     }
   }
 }
@@ -1176,10 +1187,10 @@ static size_t prefill_records_offset(int num_seqs) {
 
 size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_heads,
                                   int num_kv_heads) {
-  // unit starts, then the records twice (sorted; in row order)
+  // unit starts, then a record per unit
   return prefill_records_offset(num_seqs) +
          static_cast<size_t>(prefill_max_units(num_seqs, num_query_tokens, num_q_heads,
-                                               num_kv_heads)) * 4 * sizeof(int4);
+                                               num_kv_heads)) * 2 * sizeof(int4);
 }
 
 int tc_launch_smem(int head_dim) { return static_cast<int>(tc_smem_bytes(head_dim)); }
@@ -1208,7 +1219,6 @@ cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_
                                     prefill_records_offset(l.num_seqs));
   a.max_units = static_cast<int>(std::min<long long>(
       prefill_max_units(l.num_seqs, l.num_query_rows, l.num_q_heads, l.num_kv_heads), 1 << 28));
-  a.units_raw = a.units + 2 * static_cast<size_t>(a.max_units);
   a.err_flag = l.err_flag;
   a.tm_k = *l.tm_k;
   a.tm_v = *l.tm_v;
@@ -1246,7 +1256,6 @@ cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaSt
   a.unit_start = l.unit_start;
   a.units = l.units;
   a.max_units = l.max_units;
-  a.units_raw = l.units + 2 * static_cast<size_t>(l.max_units);
   a.group_ranges = l.group_ranges;
   a.claim = l.claim;
   a.part_ml = l.part_ml;
