@@ -465,6 +465,30 @@ __device__ __forceinline__ float ex2_fast(float x) {
   return y;
 }
 
+// Two fp32 lanes per instruction (sm_100a packed f32x2): each lane is
+// rounded as the scalar fma / add would be.
+__device__ __forceinline__ uint64_t f2_bits(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) |
+         (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ void fma2(float a0, float a1, uint64_t b, uint64_t c, float* d0, float* d1) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a0, a1)), "l"(b), "l"(c));
+  *d0 = __uint_as_float(static_cast<uint32_t>(d));
+  *d1 = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+// max(a, b, c) in one instruction (a NaN operand is passed over, as by fmaxf)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool fill) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
                "r"(fill ? 16 : 0)
@@ -815,16 +839,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
         float mul = 1.f;  // score in log2 units = sv * mul
         if (kb + kKeys <= kend && a.scale_log2 > 0.f) {
-#pragma unroll
-          for (int k = 0; k < kKeys; ++k) m8[k & 7] = fmaxf(m8[k & 7], __uint_as_float(sv[k]));
           mul = a.scale_log2;
         } else {
 #pragma unroll
           for (int k = 0; k < kKeys; ++k) {
             const float v = kb + k < kend ? __uint_as_float(sv[k]) * a.scale_log2 : -INFINITY;
             sv[k] = __float_as_uint(v);
-            m8[k & 7] = fmaxf(m8[k & 7], v);
           }
+        }
+        // (two keys per three-input max; chain c takes keys c, c + 8, ...)
+#pragma unroll
+        for (int k = 0; k < kKeys; k += 16) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            m8[c] = fmax3(m8[c], __uint_as_float(sv[k + c]), __uint_as_float(sv[k + c + 8]));
         }
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * mul;
@@ -839,21 +867,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         // them as rounded.  In tensor memory they go over the S columns just
         // read; through shared memory they are computed while the previous
         // tile's P.V may still be reading the P slot, and stored once it is done.
-        const bool none = m_run == -INFINITY;
-        const float nm = -m_run;
+        // (a column that has seen no key yet: every score of this tile is -inf,
+        // and an offset of 0 keeps its weights at 0.)  Two keys per fma and
+        // per add (f32x2); the sum runs in 8 chains, key k in chain k mod 8.
+        const float nm = m_run == -INFINITY ? 0.f : -m_run;
+        const uint64_t mul2 = f2_bits(mul, mul), nm2 = f2_bits(nm, nm);
         const uint32_t pb = smem_addr(myP) + col * 128;
-        float l8[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) l8[c] = 0.f;
+        uint64_t l4[4] = {0, 0, 0, 0};
         uint32_t w[kKeys / 2];
 #pragma unroll
         for (int e = 0; e < kKeys / 2; ++e) {
-          const float p0 = none ? 0.f : ex2_fast(fmaf(__uint_as_float(sv[2 * e]), mul, nm));
-          const float p1 = none ? 0.f : ex2_fast(fmaf(__uint_as_float(sv[2 * e + 1]), mul, nm));
-          const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-          l8[(2 * e) & 7] += __low2float(pp);
-          l8[(2 * e + 1) & 7] += __high2float(pp);
+          float x0, x1;
+          fma2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]), mul2, nm2, &x0, &x1);
+          const __nv_bfloat162 pp = __floats2bfloat162_rn(ex2_fast(x0), ex2_fast(x1));
           w[e] = *reinterpret_cast<const uint32_t*>(&pp);
+          // (bf16 -> fp32 is the 16 bits moved up)
+          l4[e & 3] = add2(l4[e & 3], static_cast<uint64_t>(w[e] << 16) |
+                                           (static_cast<uint64_t>(w[e] & 0xffff0000u) << 32));
+        }
+        float l8[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          l8[2 * c] = __uint_as_float(static_cast<uint32_t>(l4[c]));
+          l8[2 * c + 1] = __uint_as_float(static_cast<uint32_t>(l4[c] >> 32));
         }
         l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         if constexpr (kPInTmem) {
