@@ -109,6 +109,8 @@ struct TcArgs {
   int num_sms;                      // shared: the plan sizes ranges to fill this many CTAs
   int max_ranges;                   // shared: ranges the partial arrays hold per column
   int oob_row;                      // a row of the cache tensors' 2-D view past their end
+  int v8_out;                       // prefill: out is 32-byte aligned (32-byte stores)
+  int v8_part;                      // shared: part_o is 32-byte aligned
   float scale_log2;
   int* unit_start;                  // [rows + 1] work units before each sequence / group
   int4* units;                      // [max_units][2] one record per work unit, longest first
@@ -487,6 +489,15 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+
+// 32 bytes to global memory in one instruction (address 32-byte aligned):
+// a lane then fills a whole 32-byte sector, where two 16-byte stores from
+// lanes whose rows lie 256 bytes apart leave each of their sectors half used.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool fill) {
@@ -969,15 +980,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           tc::tmem_wait_ld(ov);
           if (qrow >= 0) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint32_t w[4];
+            for (int c = 0; c < 4; ++c) {  // 16 dims (32 bytes) at a time
+              uint32_t w[8];
 #pragma unroll
-              for (int f = 0; f < 4; ++f) {
+              for (int f = 0; f < 8; ++f) {
                 const __nv_bfloat162 pp = __floats2bfloat162_rn(
-                    __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
+                    __uint_as_float(ov[c * 16 + 2 * f]) * inv, __uint_as_float(ov[c * 16 + 2 * f + 1]) * inv);
                 w[f] = *reinterpret_cast<const uint32_t*>(&pp);
               }
-              dst[hf * 8 + c] = make_uint4(w[0], w[1], w[2], w[3]);
+              if (a.v8_out) {
+                st_global_v8(dst + hf * 8 + 2 * c, w);
+              } else {
+                dst[hf * 8 + 2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[hf * 8 + 2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+              }
             }
           }
         }
@@ -997,9 +1013,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           if (live) {
             float4* po = reinterpret_cast<float4*>(a.part_o + pi * D + hf * 64);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              po[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
-                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+            for (int e = 0; e < 8; ++e) {  // 8 floats (32 bytes) at a time
+              if (a.v8_part) {
+                uint32_t w[8];
+#pragma unroll
+                for (int f = 0; f < 8; ++f) w[f] = ov[8 * e + f];
+                st_global_v8(po + 2 * e, w);
+              } else {
+                po[2 * e] = make_float4(__uint_as_float(ov[8 * e]), __uint_as_float(ov[8 * e + 1]),
+                                        __uint_as_float(ov[8 * e + 2]), __uint_as_float(ov[8 * e + 3]));
+                po[2 * e + 1] = make_float4(__uint_as_float(ov[8 * e + 4]), __uint_as_float(ov[8 * e + 5]),
+                                            __uint_as_float(ov[8 * e + 6]), __uint_as_float(ov[8 * e + 7]));
+              }
+            }
           }
         }
         if (live) a.part_ml[pi] = make_float2(m_run, l_run);
@@ -1249,6 +1275,7 @@ cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_
   a.num_blocks = l.num_blocks;
   a.len_cap = l.len_cap;
   a.oob_row = l.num_blocks * l.num_kv_heads * kBlockSize;
+  a.v8_out = reinterpret_cast<uintptr_t>(l.out) % 32 == 0;
   a.scale_log2 = l.scale_log2;
   a.unit_start = static_cast<int*>(l.workspace);
   a.units = reinterpret_cast<int4*>(static_cast<char*>(l.workspace) +
@@ -1296,6 +1323,7 @@ cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaSt
   a.claim = l.claim;
   a.part_ml = l.part_ml;
   a.part_o = l.part_o;
+  a.v8_part = reinterpret_cast<uintptr_t>(l.part_o) % 32 == 0;
   a.pre_ml = l.pre_ml;
   a.pre_o = l.pre_o;
   a.err_flag = l.err_flag;

@@ -99,6 +99,29 @@ def test_repeat_calls_are_bit_identical():
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_output_aligned_to_16_bytes_only(D):
+    """The epilogue stores 32 bytes at a time when the output allows it; an
+    output that is 16-byte aligned only takes the 16-byte stores, with the
+    same result."""
+    w, q, qs = prefill_case(79, dtype="bf16", num_q_heads=16, num_kv_heads=2, head_dim=D,
+                            lens=(300, 170), queries=(150, 40))
+    ref, err, t = run_prefill(w, q, qs)
+    qd = torch.from_numpy(np.ascontiguousarray(q)).view(torch.bfloat16).cuda()
+    buf = torch.full((qd.numel() + 8,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(qd.shape)  # (16 bytes past a 256-byte aligned start)
+    assert out.data_ptr() % 32 == 16
+    err2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = ops.make_prefill_workspace(w.num_seqs, qd.shape[0], w.num_q_heads, w.num_kv_heads,
+                                    w.head_dim, w.max_context_len, 0, torch.bfloat16)
+    ops.prefill(out, qd, t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                torch.from_numpy(qs).cuda(), scale=w.scale, max_context_len=w.max_context_len,
+                workspace=ws, err_flag=err2)
+    torch.cuda.synchronize()
+    assert err == err2.item() == 0
+    assert torch.equal(ref.view(torch.int16), out.view(torch.int16))
+
+
 def test_workspace_reused_by_different_calls():
     """Calls with different work on one workspace: each call's unit layout is
     written by its own plan kernel, and no call may see the previous call's

@@ -196,6 +196,20 @@ def test_repeat_calls_are_bit_identical():
         assert torch.equal(first.view(torch.int16), t["out"].view(torch.int16))
 
 
+def test_workspace_aligned_to_16_bytes_only():
+    """The pass stores its partial states 32 bytes at a time when the
+    workspace allows it; a workspace that is 16-byte aligned only takes the
+    16-byte stores, with the same result."""
+    w = prefix_workload(4, G=4, D=128, S=10, prefix=512)
+    t, err, ws = run_shared(w)
+    first = t["out"].clone()
+    off = torch.zeros(ws.numel() + 16, dtype=torch.uint8, device="cuda")[16:]
+    assert off.data_ptr() % 32 == 16
+    t, err2, _ = run_shared(w, t=t, ws=off)
+    assert err == err2 == 0
+    assert torch.equal(first.view(torch.int16), t["out"].view(torch.int16))
+
+
 def test_no_groups_is_plain_decode():
     w = mixed_workload(13)
     empty = groups([], [0], [])
