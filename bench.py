@@ -404,7 +404,7 @@ def measure(name, args, rank: int, world: int, dev, dedup: bool = False, cpu_bud
     # so is bf16 prefill (the plan kernel and the tensor-core attention kernel)
     launches_per_step = 2 + ("key" in t and not fused) + ("block_mapping" in t)
     if dedup and plan.num_groups:
-        launches_per_step += 2      # the shared-prefix pass: its plan kernel and the pass
+        launches_per_step += 3      # the shared-prefix pass: its plan kernel, the pass, the fold
 
     def step(ev_mid=None):
         if "block_mapping" in t:
@@ -517,9 +517,9 @@ def measure(name, args, rank: int, world: int, dev, dedup: bool = False, cpu_bud
         rec["roofline"]["hbm_frac_by_unique_bytes"] = round(ub / (dec_avg * 1e-3) / 1e9 / peak, 4)
     if dedup:
         rec["config"]["dedup"] = True
-        rec["roofline"]["kernel"] = ("shared-prefix pass (tc_attention_kernel, tcgen05, and its "
-                                     "plan kernel) + paged_decode_kernel + merge pass (the "
-                                     "deduplicated decode call)")
+        rec["roofline"]["kernel"] = ("shared-prefix pass (tc_attention_kernel, tcgen05, its "
+                                     "plan kernel and tc_fold_kernel) + paged_decode_kernel + "
+                                     "merge pass (the deduplicated decode call)")
         rec["roofline"]["logical_bytes_per_launch"] = w.decode_bytes()
         rec["dedup"] = {"groups": plan.num_groups, "listed": plan.num_listed,
                         "shared_blocks": [int(b) for b in plan.blocks[:8]],
