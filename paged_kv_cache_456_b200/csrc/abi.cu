@@ -240,6 +240,35 @@ bool pa::encode_cache_map(CUtensorMap* map, const void* base, long long rows, in
   return r == CUDA_SUCCESS;
 }
 
+bool pa::encode_prefill_out_map(CUtensorMap* map, void* out, int num_query_rows,
+                                int num_q_heads, int head_dim, int group) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return false;
+      }
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                              static_cast<cuuint64_t>(num_query_rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                 static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, strides, box,
+                            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 size_t pa::decode_zero_prefix_bytes(int num_seqs, int num_kv_heads) {
   return 8 * sizeof(int) + 2 * static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int);
 }
@@ -562,6 +591,11 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     l.err_flag = err_flag;
     l.tm_k = &tk;
     l.tm_v = &tv;
+    CUtensorMap to;
+    l.tm_out = pa::encode_prefill_out_map(&to, out, num_query_tokens, num_q_heads, head_dim,
+                                          num_q_heads / num_kv_heads)
+                   ? &to
+                   : nullptr;
     if (pa::launch_tc_prefill(l, dev.sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
       cudaGetLastError();
       return PA_ERR_CUDA;

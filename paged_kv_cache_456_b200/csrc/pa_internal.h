@@ -163,6 +163,11 @@ cudaError_t launch_shared_prefix(SharedPrefixLaunch& l, int num_sms, cudaStream_
 // A cache as the 2-D bf16 tensor [num_blocks * num_kv_heads * 16][head_dim],
 // read in boxes of 16 rows x 64 elements with the 128-byte swizzle (abi.cu).
 bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim);
+// The prefill output [rows][num_q_heads][head_dim] bf16 as a 3-D tensor
+// (head_dim, query heads, rows) with boxes of 64 x group x 128/group, 128-byte
+// swizzle: the tensor-core kernel's epilogue stores a column tile through it.
+bool encode_prefill_out_map(CUtensorMap* map, void* out, int num_query_rows, int num_q_heads,
+                            int head_dim, int group);
 
 // ---- tensor-core attention of many query columns (tc_attention.cu) ----------
 // Several query tokens per sequence: one column per (query row, query head),
@@ -186,6 +191,7 @@ struct TcPrefillLaunch {
   int32_t* err_flag;
   const CUtensorMap* tm_k;
   const CUtensorMap* tm_v;
+  const CUtensorMap* tm_out;  // the output for the epilogue's tensor stores (null: plain stores)
 };
 bool tc_prefill_supported(int head_dim, int group);
 size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_heads,

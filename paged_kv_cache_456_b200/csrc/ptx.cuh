@@ -112,6 +112,27 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
+// 3-D tiled TMA store of one box from this CTA's shared memory at element
+// coordinates (x, y, z) of `tmap` (x: a multiple of 16 bytes' worth of
+// elements; no coordinate negative), in the current bulk group.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   tmap),
+               "r"(x), "r"(y), "r"(z), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's bulk groups have finished reading shared memory
+// (their source may then be rewritten) / have completed.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // An L2 cache policy under which the lines a load brings in are the first to
 // be evicted: for data streamed once (the K/V tiles of decode), so that what
 // is written meanwhile (partial results read back by the merge pass) stays.

@@ -110,6 +110,7 @@ struct TcArgs {
   int max_ranges;                   // shared: ranges the partial arrays hold per column
   int oob_row;                      // a row of the cache tensors' 2-D view past their end
   int v8_out;                       // prefill: out is 32-byte aligned (32-byte stores)
+  int tma_out;                      // prefill: tm_out is set (full column tiles by tensor stores)
   int v8_part;                      // shared: part_o is 32-byte aligned
   float scale_log2;
   int* unit_start;                  // [rows + 1] work units before each sequence / group
@@ -124,6 +125,7 @@ struct TcArgs {
   int32_t* err_flag;
   CUtensorMap tm_k;                 // caches as [num_blocks * Hkv * 16][D], boxes 16 x 64, SW128
   CUtensorMap tm_v;
+  CUtensorMap tm_out;               // prefill: out as (head_dim, Hq, rows), boxes 64 x G x 128/G
 };
 
 __device__ __forceinline__ void seterr(const TcArgs& a, int bit) {
@@ -512,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   constexpr int QT = kCols * D * 2;          // bytes of a Q tile
   constexpr int KT = kKeys * D * 2;          // bytes of a K (or V) tile
   constexpr int PT = kCols * kKeys * 2;      // bytes of a P tile (one 128-byte row per column)
+  constexpr int OT = kCols * D * 2;          // bytes of a bf16 O tile (prefill's staging)
   constexpr int HALF = kKeys * 128;          // bytes of a 64-element half of a K/V tile
   constexpr int RPT = kCols / G;
   constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(kCols, kKeys, false);
@@ -526,13 +529,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   unsigned char* sK = sQ + kPair * QT;       // [kStages][KT]
   unsigned char* sV = sK + kStages * KT;     // [kStages][KT]
   unsigned char* sP = sV + kStages * KT;     // [kPair][PT] (P through shared memory only)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + (kPInTmem ? 0 : kPair * PT));
+  unsigned char* sO = sP + (kPInTmem ? 0 : kPair * PT);  // prefill: [kPair][OT] staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sO + (MODE == kModePrefill ? kPair * OT : 0));
   // barriers: kfull[3] kempty[3] vfull[3] vempty[3] | per tile t: sfull[t][2],
-  // pfull[t], odone[t] | qfull drain
+  // pfull[t], odone[t] | qfull drain | osync[t]
   const uint32_t b0 = smem_addr(bars);
   const uint32_t KFULL = b0, KEMPTY = b0 + 24, VFULL = b0 + 48, VEMPTY = b0 + 72;
   const uint32_t TB = b0 + 96;  // tile t's barriers at TB + 32 t: sfull[2], pfull, odone
   const uint32_t QFULL = b0 + 96 + 32 * kPair, DRAIN = QFULL + 8;
+  const uint32_t OSYNC = DRAIN + 8;  // osync[t] at OSYNC + 8 t: tile t's warpgroup among itself
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -554,6 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     }
     mbar_init(QFULL, kSoftmaxThreads);
     mbar_init(DRAIN, 1);
+    for (int t = 0; t < kPair; ++t) mbar_init(OSYNC + 8 * t, kWgThreads);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -766,12 +772,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     const uint32_t s_col = t * 2 * kKeys, o_col = 2 * kPair * kKeys + t * D;  // TMEM columns
     unsigned char* const myQ = sQ + t * QT;
     unsigned char* const myP = sP + t * PT;
-    int sidx = 0, oidx = 0, tile = 0;
+    int sidx = 0, oidx = 0, tile = 0, syncs = 0;
     bool ok = true;
     // a bounded wait whose outcome the whole warp shares, so that no lane
     // leaves ahead of the others (the TMEM moves are warp-wide)
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    auto group_sync = [&]() -> bool {  // the 128 threads of this warpgroup
+      mbar_arrive(OSYNC + 8 * t);
+      return wait_all(OSYNC + 8 * t, (syncs++) & 1);
     };
     // this column's query row in unit y (-1: none), and the keys it sees
     auto column_of = [&](const Unit& y, int* kend) -> int {
@@ -969,8 +979,48 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       ++oidx;
       tc::fence_after_sync();
       if constexpr (MODE == kModePrefill) {
-        // (every lane runs the warp-wide TMEM loads; only live columns store)
         const float inv = 1.f / l_run;
+        const int ct = x.pr * kPair + t;
+        // A column tile whose rows all belong to this sequence goes out by
+        // tensor stores (one box per 64 dims: the TMA engine does the strided
+        // writes) from a staging tile in the 128-byte-swizzled layout; the
+        // last tile of a sequence goes out row by row.
+        const bool staged = a.tma_out && (ct + 1) * RPT <= x.Q;
+        if (staged) {
+          unsigned char* const stg = sO + t * OT;
+          if (col == 0) bulk_wait_group_read0();  // (the previous unit's stores have read it)
+          if (!group_sync()) { ok = false; break; }
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) {
+            uint32_t ov[64];
+            tc::tmem_ld64(lane_base + o_col + hf * 64, ov);
+            tc::tmem_wait_ld(ov);
+            const uint32_t rowb = smem_addr(stg) + hf * (kCols * 128) + col * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {  // 8 dims (16 bytes) per chunk
+              uint32_t w[4];
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {
+                const __nv_bfloat162 pp = __floats2bfloat162_rn(
+                    __uint_as_float(ov[c * 8 + 2 * f]) * inv, __uint_as_float(ov[c * 8 + 2 * f + 1]) * inv);
+                w[f] = *reinterpret_cast<const uint32_t*>(&pp);
+              }
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + ((c ^ (col & 7)) << 4)),
+                           "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                           : "memory");
+            }
+          }
+          fence_proxy_async_smem();
+          if (!group_sync()) { ok = false; break; }
+          if (col == 0) {
+#pragma unroll
+            for (int hf = 0; hf < D / 64; ++hf)
+              tma_store_3d(&a.tm_out, smem_addr(stg) + hf * (kCols * 128), hf * 64, x.kvh * G,
+                           x.q0 + ct * RPT);
+            bulk_commit_group();
+          }
+        } else {
+        // (every lane runs the warp-wide TMEM loads; only live columns store)
         uint4* dst = reinterpret_cast<uint4*>(
             a.out + (static_cast<size_t>(qrow >= 0 ? qrow : 0) * Hq + x.kvh * G + h) * D);
 #pragma unroll
@@ -996,6 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
               }
             }
           }
+        }
         }
       } else {
         // ---- shared: this range's partial state (the fold kernel combines the ranges)
@@ -1033,6 +1084,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     }
     if (!ok) timeout();
     asm volatile("cp.async.wait_all;" ::: "memory");  // (a prefetch left in flight by an abort)
+    if (MODE == kModePrefill && col == 0) bulk_wait_group0();  // (the tensor stores have completed)
   }
 
   // ---- teardown: every role is out of its loop; the MMAs have drained -------
@@ -1172,12 +1224,14 @@ bool pick(int head_dim, int group, const void** plan, const void** main) {
   }
 }
 
-size_t tc_smem_bytes(int head_dim) {
+size_t tc_smem_bytes(int head_dim, bool prefill) {
   const size_t q = static_cast<size_t>(kCols) * head_dim * 2;
   const size_t kv = static_cast<size_t>(kKeys) * head_dim * 2;
   const size_t p = static_cast<size_t>(kCols) * kKeys * 2;
-  // (alignment slack; barriers: 12 ring + 4 per tile + 2)
-  return 1024 + kPair * q + 2 * kStages * kv + (kPInTmem ? 0 : kPair * p) + 256;
+  // (alignment slack; barriers: 12 ring + 4 per tile + 4)
+  // (prefill: a bf16 O staging tile per column tile, as large as its Q tile)
+  return 1024 + kPair * q + 2 * kStages * kv + (kPInTmem ? 0 : kPair * p) + (prefill ? kPair * q : 0) +
+         256;
 }
 
 std::mutex g_tc_mu;
@@ -1255,7 +1309,7 @@ size_t tc_prefill_workspace_bytes(int num_seqs, int num_query_tokens, int num_q_
                                                num_kv_heads)) * 2 * sizeof(int4);
 }
 
-int tc_launch_smem(int head_dim) { return static_cast<int>(tc_smem_bytes(head_dim)); }
+int tc_launch_smem(int head_dim) { return static_cast<int>(tc_smem_bytes(head_dim, true)); }
 
 cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_t stream) {
   const void *plan, *main;
@@ -1276,6 +1330,10 @@ cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_
   a.len_cap = l.len_cap;
   a.oob_row = l.num_blocks * l.num_kv_heads * kBlockSize;
   a.v8_out = reinterpret_cast<uintptr_t>(l.out) % 32 == 0;
+  if (l.tm_out) {
+    a.tm_out = *l.tm_out;
+    a.tma_out = 1;
+  }
   a.scale_log2 = l.scale_log2;
   a.unit_start = static_cast<int*>(l.workspace);
   a.units = reinterpret_cast<int4*>(static_cast<char*>(l.workspace) +
@@ -1285,7 +1343,7 @@ cudaError_t launch_tc_prefill(const TcPrefillLaunch& l, int num_sms, cudaStream_
   a.err_flag = l.err_flag;
   a.tm_k = *l.tm_k;
   a.tm_v = *l.tm_v;
-  return launch_pair(plan, main, a, num_sms, tc_smem_bytes(l.head_dim), stream);
+  return launch_pair(plan, main, a, num_sms, tc_smem_bytes(l.head_dim, true), stream);
 }
 
 bool tc_shared_prefix_supported(int head_dim, int group) {
@@ -1329,7 +1387,7 @@ cudaError_t launch_tc_shared_prefix(const TcSharedLaunch& l, int num_sms, cudaSt
   a.err_flag = l.err_flag;
   a.tm_k = *l.tm_k;
   a.tm_v = *l.tm_v;
-  cudaError_t e = launch_pair(plan, main, a, num_sms, tc_smem_bytes(l.head_dim), stream);
+  cudaError_t e = launch_pair(plan, main, a, num_sms, tc_smem_bytes(l.head_dim, false), stream);
   if (e != cudaSuccess || l.num_listed == 0) return e;
   // the fold: one CTA per (listed member, slice of kFoldThreads / (D / 4) heads)
   const int hpc = kFoldThreads / (l.head_dim / 4);
