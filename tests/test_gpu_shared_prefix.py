@@ -89,7 +89,7 @@ def test_matches_oracle(G, D):
 @pytest.mark.parametrize("G,S,prefix", [(1, 70, 1200), (8, 9, 560), (4, 33, 2048), (2, 3, 16)])
 def test_wide_groups_and_long_prefixes(G, S, prefix):
     # 70 x 1 and 9 x 8 columns need two CTAs' worth; 1200 and 2048 tokens
-    # span several 32-block ranges, folded by the last one; a 16-token prefix
+    # span several ranges of shared blocks, combined by the fold; a 16-token prefix
     # is one shared block
     w = prefix_workload(7 + G, G=G, D=128, S=S, prefix=prefix, suffix_mean=30.0)
     t, err, _ = run_shared(w)
