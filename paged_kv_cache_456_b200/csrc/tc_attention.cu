@@ -84,13 +84,6 @@ constexpr int kPlanRowsOnChip = 4096;           // unit starts the plan kernel k
 constexpr int kMaxFoldRanges = 16;              // shared: ranges of a group's shared blocks, at most
 constexpr int kModePrefill = 0;
 constexpr int kModeShared = 1;
-// P (the bf16 weights) goes to tensor memory over the S columns it was made
-// from, and the P.V MMA takes its A operand from there (1), or through a
-// shared-memory tile per column tile (0).
-#ifndef PA_TC_P_TMEM
-#define PA_TC_P_TMEM 1
-#endif
-constexpr bool kPInTmem = PA_TC_P_TMEM != 0;
 
 struct TcArgs {
   const __nv_bfloat16* q;
@@ -513,7 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   constexpr int KB = D / 64;                 // 64-element (128-byte) blocks of head_dim
   constexpr int QT = kCols * D * 2;          // bytes of a Q tile
   constexpr int KT = kKeys * D * 2;          // bytes of a K (or V) tile
-  constexpr int PT = kCols * kKeys * 2;      // bytes of a P tile (one 128-byte row per column)
   constexpr int OT = kCols * D * 2;          // bytes of a bf16 O tile (prefill's staging)
   constexpr int HALF = kKeys * 128;          // bytes of a 64-element half of a K/V tile
   constexpr int RPT = kCols / G;
@@ -528,8 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   unsigned char* sQ = sm;                    // [kPair][QT]
   unsigned char* sK = sQ + kPair * QT;       // [kStages][KT]
   unsigned char* sV = sK + kStages * KT;     // [kStages][KT]
-  unsigned char* sP = sV + kStages * KT;     // [kPair][PT] (P through shared memory only)
-  unsigned char* sO = sP + (kPInTmem ? 0 : kPair * PT);  // prefill: [kPair][OT] staging
+  unsigned char* sO = sV + kStages * KT;     // prefill: [kPair][OT] staging
   uint64_t* bars = reinterpret_cast<uint64_t*>(sO + (MODE == kModePrefill ? kPair * OT : 0));
   // barriers: kfull[3] kempty[3] vfull[3] vempty[3] | per tile t: sfull[t][2],
   // pfull[t], odone[t] | qfull drain | osync[t]
@@ -672,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     int kidx = 0, vidx = 0, qidx = 0;
     int sidx[kPair] = {0, 0}, pidx[kPair] = {0, 0};
     bool ok = true;
-    const uint32_t qbase = smem_addr(sQ), pbase = smem_addr(sP);
+    const uint32_t qbase = smem_addr(sQ);
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
     };
@@ -735,14 +726,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           tc::fence_after_sync();
 #pragma unroll
           for (int k = 0; k < kKeys / 16; ++k) {
-            if constexpr (kPInTmem)
-              mma_ts(tmem + 2 * kPair * kKeys + t * D, pa + k * 8,
-                     tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
-                     (j > 0 || k > 0) ? 1u : 0u);
-            else
-              mma(tmem + 2 * kPair * kKeys + t * D, tc::sdesc_sw128(pbase + t * PT + k * 32, 16, 1024),
-                  tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
-                  (j > 0 || k > 0) ? 1u : 0u);
+            mma_ts(tmem + 2 * kPair * kKeys + t * D, pa + k * 8,
+                   tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
+                   (j > 0 || k > 0) ? 1u : 0u);
           }
           commit(TB + 32 * t + 24);  // odone[t]
           if (t == kPair - 1) {
@@ -771,7 +757,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     const uint32_t SFULL = TB + 32 * t, PFULL = SFULL + 16, ODONE = SFULL + 24;
     const uint32_t s_col = t * 2 * kKeys, o_col = 2 * kPair * kKeys + t * D;  // TMEM columns
     unsigned char* const myQ = sQ + t * QT;
-    unsigned char* const myP = sP + t * PT;
     int sidx = 0, oidx = 0, tile = 0, syncs = 0;
     bool ok = true;
     // a bounded wait whose outcome the whole warp shares, so that no lane
@@ -885,15 +870,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           m_run = mx;
         }
         // weights, rounded to bf16 for the product; the sum (8 chains) takes
-        // them as rounded.  In tensor memory they go over the S columns just
-        // read; through shared memory they are computed while the previous
-        // tile's P.V may still be reading the P slot, and stored once it is done.
+        // them as rounded.  They go to tensor memory over the S columns just
+        // read (two per 32-bit column), the A operand of this tile's P.V.
         // (a column that has seen no key yet: every score of this tile is -inf,
         // and an offset of 0 keeps its weights at 0.)  Two keys per fma and
         // per add (f32x2); the sum runs in 8 chains, key k in chain k mod 8.
         const float nm = m_run == -INFINITY ? 0.f : -m_run;
         const uint64_t mul2 = f2_bits(mul, mul), nm2 = f2_bits(nm, nm);
-        const uint32_t pb = smem_addr(myP) + col * 128;
         uint64_t l4[4] = {0, 0, 0, 0};
         uint32_t w[kKeys / 2];
 #pragma unroll
@@ -913,7 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           l8[2 * c + 1] = __uint_as_float(static_cast<uint32_t>(l4[c] >> 32));
         }
         l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-        if constexpr (kPInTmem) {
+        {
           uint32_t w32[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) w32[e] = w[e];
@@ -921,17 +904,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           tc::tmem_wait_st();
         }
         if (j > 0) {
-          // O of the previous tile is complete: its P slot is free and O is stable
+          // O of the previous tile is complete (so that it may be rescaled)
           if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
           ++oidx;
           tc::fence_after_sync();
-        }
-        if constexpr (!kPInTmem) {
-#pragma unroll
-          for (int c = 0; c < kKeys / 8; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + (((c % 8) ^ (col % 8)) << 4)),
-                         "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
-                         : "memory");
         }
         if constexpr (MODE == kModePrefill) {
           // rows past the sequence's end in its last block hold stale data: a
@@ -1227,11 +1203,9 @@ bool pick(int head_dim, int group, const void** plan, const void** main) {
 size_t tc_smem_bytes(int head_dim, bool prefill) {
   const size_t q = static_cast<size_t>(kCols) * head_dim * 2;
   const size_t kv = static_cast<size_t>(kKeys) * head_dim * 2;
-  const size_t p = static_cast<size_t>(kCols) * kKeys * 2;
   // (alignment slack; barriers: 12 ring + 4 per tile + 4)
   // (prefill: a bf16 O staging tile per column tile, as large as its Q tile)
-  return 1024 + kPair * q + 2 * kStages * kv + (kPInTmem ? 0 : kPair * p) + (prefill ? kPair * q : 0) +
-         256;
+  return 1024 + kPair * q + 2 * kStages * kv + (prefill ? kPair * q : 0) + 256;
 }
 
 std::mutex g_tc_mu;
