@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
   if constexpr (MODE == kModePrefill) {
     // every block a computable sequence attends to must be a block of the
     // cache; one with a bad id gets no units, its rows are zeroed here and
-    // the error bit is set (one warp per sequence; the verdict goes through
+    // the error bit is set (one warp per sequence; the outcome goes through
     // the row scratch, overwritten below)
     for (int r = warp; r < R; r += kPlanThreads / 32) {
       int q0 = 0, Q = 0, n = 0, bit = 0;
