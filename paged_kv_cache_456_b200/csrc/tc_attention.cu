@@ -820,6 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
 
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < x.nt; ++j, ++tile) {
+        bool zeroed = false;  // (this thread wrote zeros into the V tile)
         if (aborted() || !wait_all(SFULL + 8 * (sidx & 1), (sidx >> 1) & 1)) { ok = false; break; }
         tc::fence_after_sync();
         uint32_t sv[kKeys];
@@ -916,6 +917,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           const int tail = x.n % kBlockSize;
           const int lastb = x.n / kBlockSize;  // logical block holding them
           if (t == 0 && tail && lastb * kBlockSize >= kb && lastb * kBlockSize < kb + kKeys) {
+            zeroed = true;
             const int st = tile % kStages;
             if (!wait_all(VFULL + 8 * st, (tile / kStages) & 1)) { ok = false; break; }
             const int b = (lastb * kBlockSize - kb) / kBlockSize;
@@ -945,7 +947,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
           }
           tc::tmem_wait_st();
         }
-        fence_proxy_async_smem();
+        // (the V rows zeroed above are generic writes the MMA reads through
+        // the async proxy; P went to tensor memory and needs no such fence)
+        if (zeroed) fence_proxy_async_smem();
         tc::fence_before_sync();
         mbar_arrive(PFULL);
       }
