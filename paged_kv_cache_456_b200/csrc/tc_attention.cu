@@ -80,7 +80,10 @@ constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;                  // S of tile t at 128 t (+64), O of tile t at 256 + 128 t
 constexpr int kPlanThreads = 1024;
 constexpr int kSortBuckets = 256;               // unit lengths the plan kernel tells apart
-constexpr int kPlanRowsOnChip = 4096;           // unit starts the plan kernel keeps on chip
+constexpr int kPlanRowsOnChip = 2048;           // rows whose metadata and unit starts the plan
+                                                // kernel keeps on chip
+constexpr int kPlanAhead = 4;                   // block ids per lane the plan loads beside a row's
+                                                // lengths
 constexpr int kMaxFoldRanges = 16;              // shared: ranges of a group's shared blocks, at most
 constexpr int kModePrefill = 0;
 constexpr int kModeShared = 1;
@@ -125,37 +128,44 @@ __device__ __forceinline__ void seterr(const TcArgs& a, int bit) {
   if (a.err_flag) atomicOr(a.err_flag, bit);
 }
 
-// Prefill: the query rows of sequence s, or false (with the error bit to set
+// Prefill: sequence s's query rows [a0, a1) and context length len checked;
+// its first query row, rows and length, or false (with the error bit to set
 // in *bit, 0 if none) when it has none to compute.
-__device__ __forceinline__ bool prefill_seq(const TcArgs& a, int s, int* q0, int* Q, int* n,
-                                            int* bit) {
+__device__ __forceinline__ bool prefill_row(const TcArgs& a, int a0, int a1, int len, int* q0,
+                                            int* Q, int* n, int* bit) {
   *bit = 0;
-  const int a0 = a.query_start[s], a1 = a.query_start[s + 1];
   if (!(0 <= a0 && a0 <= a1 && a1 <= a.num_query_rows)) {
     *bit = kErrQuery;
     return false;
   }
   *q0 = a0;
   *Q = a1 - a0;
-  *n = a.context_lens[s];
+  *n = len;
   if (*Q == 0) return false;
-  if (*n < 0 || *n > a.len_cap) {
+  if (len < 0 || len > a.len_cap) {
     *bit = kErrContextLen;
     return false;
   }
-  if (*Q > *n) {
+  if (*Q > len) {
     *bit = kErrQuery;
     return false;
   }
   return true;
 }
 
+// The same from the arrays (all three loads issued together: s is a row of
+// the table, so each is in bounds whatever the values).
+__device__ __forceinline__ bool prefill_seq(const TcArgs& a, int s, int* q0, int* Q, int* n,
+                                            int* bit) {
+  const int a0 = a.query_start[s], a1 = a.query_start[s + 1], len = a.context_lens[s];
+  return prefill_row(a, a0, a1, len, q0, Q, n, bit);
+}
+
 // Shared: group g's members and shared blocks, if well formed.
 __device__ __forceinline__ bool shared_group(const TcArgs& a, int g, int* gs, int* m, int* P,
                                              int* leader) {
-  const int s0 = a.group_start[g], s1 = a.group_start[g + 1];
+  const int s0 = a.group_start[g], s1 = a.group_start[g + 1], p = a.group_blocks[g];
   if (!(0 <= s0 && s0 < s1 && s1 <= a.num_listed)) return false;
-  const int p = a.group_blocks[g];
   if (p < 1 || p > a.max_blocks_per_seq) return false;
   const int l = a.group_seqs[s0];
   if (l < 0 || l >= a.num_seqs) return false;
@@ -170,26 +180,102 @@ __device__ __forceinline__ bool shared_group(const TcArgs& a, int g, int* gs, in
 // plan: work units per sequence / group and their prefix sums
 // ---------------------------------------------------------------------------
 template <int D, int G, int MODE>
-__global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(kPlanThreads, 1) tc_plan_kernel(const __grid_constant__ TcArgs a) {
   // the attention kernel may start its prologue now
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int s_wsum[kPlanThreads / 32];
+  __shared__ int s_target, s_total;
+  __shared__ int s_hist[kSortBuckets];
+  __shared__ int s_pos[kSortBuckets];
+  // per-row scratch on chip when the rows fit (else unit_start holds the
+  // counts and starts and the metadata is read again where it is needed):
+  // unit counts, then unit starts (the attention kernel reads only
+  // unit_start[R]); each row's metadata, prefill {first query row, rows,
+  // context length, 0}, shared {first member, members, shared blocks, leader}
+  __shared__ int s_us[kPlanRowsOnChip + 1];
+  __shared__ int4 s_meta[kPlanRowsOnChip];
   constexpr int RPT = kCols / G;  // query rows (members) per column tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = a.rows, Hkv = a.num_kv_heads, Hq = a.num_q_heads;
   const int per = (R + kPlanThreads - 1) / kPlanThreads;
   const int r0 = min(R, tid * per), r1 = min(R, r0 + per);
-  // shared: ranges per group, so that all units together about fill the
-  // SMs: the pairs of column tiles x KV heads of every group are counted
-  // first, and each group's shared blocks are then cut into as many ranges
-  // (of whole K/V tiles, at least two) as one wave needs
-  __shared__ int s_target;
-  if constexpr (MODE == kModeShared) {
+  const bool on_chip = R <= kPlanRowsOnChip;
+  auto row_set = [&](int r, int v) {
+    if (on_chip) s_us[r] = v; else a.unit_start[r] = v;
+  };
+  auto row_get = [&](int r) -> int { return on_chip ? s_us[r] : __ldcg(a.unit_start + r); };
+  // (only rows with units are asked for: their metadata is well formed)
+  auto meta_of = [&](int r) -> int4 {
+    if (on_chip) return s_meta[r];
+    int4 m = make_int4(0, 0, 0, 0);
+    if constexpr (MODE == kModePrefill) {
+      int bit;
+      prefill_seq(a, r, &m.x, &m.y, &m.z, &bit);
+    } else {
+      shared_group(a, r, &m.x, &m.y, &m.z, &m.w);
+    }
+    return m;
+  };
+  for (int b = tid; b < kSortBuckets; b += kPlanThreads) s_hist[b] = 0;
+  int local = 0;  // units of this thread's rows
+  if constexpr (MODE == kModePrefill) {
+    // One warp per sequence: its lengths and its first block ids are loaded
+    // together (each load in bounds of its array whatever the values), then
+    // every block a computable sequence attends to must be a block of the
+    // cache.  A sequence that cannot be computed gets no units, its
+    // (well-placed) query rows are zeroed here and the error bit is set.
+    for (int r = warp; r < R; r += kPlanThreads / 32) {
+      const int32_t* trow = a.block_tables + static_cast<size_t>(r) * a.max_blocks_per_seq;
+      const int a0 = a.query_start[r], a1 = a.query_start[r + 1], len = a.context_lens[r];
+      int ids[kPlanAhead];
+#pragma unroll
+      for (int k = 0; k < kPlanAhead; ++k) {
+        const int b = lane + 32 * k;
+        ids[k] = b < a.max_blocks_per_seq ? __ldg(trow + b) : 0;
+      }
+      int q0 = 0, Q = 0, n = 0, bit = 0;
+      const bool ok = prefill_row(a, a0, a1, len, &q0, &Q, &n, &bit);
+      bool bad = false;
+      if (ok) {
+        const int nb = (n + kBlockSize - 1) / kBlockSize;  // (at most max_blocks_per_seq)
+#pragma unroll
+        for (int k = 0; k < kPlanAhead; ++k)
+          bad |= lane + 32 * k < nb && !(ids[k] >= 0 && ids[k] < a.num_blocks);
+        for (int b = lane + 32 * kPlanAhead; b < nb; b += 32) {
+          const int phys = __ldg(trow + b);
+          bad |= !(phys >= 0 && phys < a.num_blocks);
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad) bit = kErrBlockId;
+      }
+      if (bit) {
+        if (lane == 0) seterr(a, bit);
+        if (0 <= a0 && a0 <= a1 && a1 <= a.num_query_rows) {
+          uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(a0) * Hq * D);
+          const size_t cnt = static_cast<size_t>(a1 - a0) * Hq * D * 2 / 16;
+          for (size_t i = lane; i < cnt; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (lane == 0) {
+        row_set(r, ok && !bad ? Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair) : 0);
+        if (on_chip) s_meta[r] = make_int4(q0, Q, n, 0);
+      }
+    }
+    __syncthreads();
+    for (int r = r0; r < r1; ++r) local += row_get(r);
+  } else {
+    // Ranges per group, so that all units together about fill the SMs: the
+    // pairs of column tiles x KV heads of every group are counted first, and
+    // each group's shared blocks are then cut into as many ranges (of whole
+    // K/V tiles, at least two) as one wave needs.
     int base = 0;
     for (int r = r0; r < r1; ++r) {
-      int gs, m, P, leader;
-      if (shared_group(a, r, &gs, &m, &P, &leader))
-        base += Hkv * (((m * G + kCols - 1) / kCols + kPair - 1) / kPair);
+      int4 m = make_int4(0, 0, 0, -1);
+      if (shared_group(a, r, &m.x, &m.y, &m.z, &m.w))
+        base += Hkv * (((m.y * G + kCols - 1) / kCols + kPair - 1) / kPair);
+      else
+        m = make_int4(0, 0, 0, -1);
+      if (on_chip) s_meta[r] = m;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) base += __shfl_xor_sync(0xffffffffu, base, o);
@@ -210,73 +296,23 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
     *rb = b;
     return (P + b - 1) / b;
   };
-  // per-row scratch (unit counts, then unit starts): on chip when the rows
-  // fit, else in unit_start; the attention kernel reads only unit_start[R]
-  __shared__ int s_us[kPlanRowsOnChip + 1];
-  const bool on_chip = R <= kPlanRowsOnChip;
-  auto row_set = [&](int r, int v) {
-    if (on_chip) s_us[r] = v; else a.unit_start[r] = v;
-  };
-  auto row_get = [&](int r) -> int { return on_chip ? s_us[r] : __ldcg(a.unit_start + r); };
-  if constexpr (MODE == kModePrefill) {
-    // every block a computable sequence attends to must be a block of the
-    // cache; one with a bad id gets no units, its rows are zeroed here and
-    // the error bit is set (one warp per sequence; the outcome goes through
-    // the row scratch, overwritten below)
-    for (int r = warp; r < R; r += kPlanThreads / 32) {
-      int q0 = 0, Q = 0, n = 0, bit = 0;
-      bool bad = false;
-      if (prefill_seq(a, r, &q0, &Q, &n, &bit)) {
-        const int32_t* trow = a.block_tables + static_cast<size_t>(r) * a.max_blocks_per_seq;
-        const int nb = (n + kBlockSize - 1) / kBlockSize;
-        for (int b = lane; b < nb; b += 32) {
-          const int phys = __ldg(trow + b);
-          bad |= !(phys >= 0 && phys < a.num_blocks);
-        }
-        bad = __any_sync(0xffffffffu, bad);
-        if (bad) {
-          if (lane == 0) seterr(a, kErrBlockId);
-          uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(q0) * Hq * D);
-          const size_t cnt = static_cast<size_t>(Q) * Hq * D * 2 / 16;
-          for (size_t i = lane; i < cnt; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      if (lane == 0) row_set(r, bad ? 1 : 0);
-    }
-    __syncthreads();
-  }
-  int local = 0;
-  for (int r = r0; r < r1; ++r) {
-    int units = 0;
-    if constexpr (MODE == kModePrefill) {
-      int q0 = 0, Q = 0, n = 0, bit = 0;
-      if (prefill_seq(a, r, &q0, &Q, &n, &bit)) {
-        if (row_get(r) == 0) units = Hkv * (((Q + RPT - 1) / RPT + kPair - 1) / kPair);
-      } else if (bit) {
-        seterr(a, bit);
-        if (bit != kErrQuery || (a.query_start[r] >= 0 && a.query_start[r] <= a.query_start[r + 1] &&
-                                 a.query_start[r + 1] <= a.num_query_rows)) {
-          // a sequence that cannot be computed: its (well-placed) rows are zero
-          const int b0 = a.query_start[r], b1 = a.query_start[r + 1];
-          uint4* dst = reinterpret_cast<uint4*>(a.out + static_cast<size_t>(b0) * Hq * D);
-          const size_t cnt = static_cast<size_t>(b1 - b0) * Hq * D * 2 / 16;
-          for (size_t i = 0; i < cnt; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    } else {
-      int gs, m, P, leader, Rg = 0;
-      if (shared_group(a, r, &gs, &m, &P, &leader)) {
-        const int npair = ((m * G + kCols - 1) / kCols + kPair - 1) / kPair;
+  if constexpr (MODE == kModeShared) {
+    for (int r = r0; r < r1; ++r) {
+      int units = 0, Rg = 0;
+      int4 m = on_chip ? s_meta[r] : make_int4(0, 0, 0, -1);
+      if (!on_chip && !shared_group(a, r, &m.x, &m.y, &m.z, &m.w)) m.w = -1;
+      if (m.w >= 0) {
+        const int npair = ((m.y * G + kCols - 1) / kCols + kPair - 1) / kPair;
         int rb;
-        Rg = ranges_of(P, &rb);
+        Rg = ranges_of(m.z, &rb);
         units = npair * Hkv * Rg;
       } else {
         seterr(a, kErrGroup);
       }
       a.group_ranges[r] = Rg;
+      row_set(r, units);  // (turned into starts below)
+      local += units;
     }
-    row_set(r, units);  // (turned into starts below)
-    local += units;
   }
   int incl = local;
 #pragma unroll
@@ -286,27 +322,32 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
   }
   if (lane == 31) s_wsum[warp] = incl;
   __syncthreads();
-  int run = incl - local, total = 0;
+  // (only the threads with rows, and thread 0 for the total, need the warps'
+  // sums: with few rows most warps skip them)
+  if (r0 < r1 || tid == 0) {
+    int run = incl - local, total = 0;
 #pragma unroll
-  for (int w = 0; w < kPlanThreads / 32; ++w) {
-    if (w < warp) run += s_wsum[w];
-    total += s_wsum[w];
-  }
-  for (int r = r0; r < r1; ++r) {
-    const int units = row_get(r);
-    row_set(r, run);
-    // (a group whose units do not all fit the workspace is not folded)
-    if (MODE == kModeShared && run + units > a.max_units) a.group_ranges[r] = 0;
-    run += units;
-  }
-  // (the workspace is sized for the most units a call can have)
-  const int T = min(total, a.max_units);
-  if (tid == 0) {
-    row_set(R, total);
-    a.unit_start[R] = T;
-    if (total > a.max_units) seterr(a, kErrTimeout);
+    for (int w = 0; w < kPlanThreads / 32; ++w) {
+      if (w < warp) run += s_wsum[w];
+      total += s_wsum[w];
+    }
+    for (int r = r0; r < r1; ++r) {
+      const int units = row_get(r);
+      row_set(r, run);
+      // (a group whose units do not all fit the workspace is not folded)
+      if (MODE == kModeShared && run + units > a.max_units) a.group_ranges[r] = 0;
+      run += units;
+    }
+    if (tid == 0) {
+      // (the workspace is sized for the most units a call can have)
+      row_set(R, total);
+      s_total = total;
+      a.unit_start[R] = min(total, a.max_units);
+      if (total > a.max_units) seterr(a, kErrTimeout);
+    }
   }
   __syncthreads();
+  const int T = min(s_total, a.max_units);
   // Each unit as a record {row, kv head | pair of column tiles << 16, first
   // key, last key + 1} {prefill: first query row, rows, context length, 0 |
   // shared: first member, members, shared blocks, range | ranges << 16}, so
@@ -319,24 +360,23 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
       if (row_get(mid) <= u) lo = mid; else up = mid - 1;
     }
     const int r = lo, k = u - row_get(lo);
+    const int4 m = meta_of(r);
     if constexpr (MODE == kModePrefill) {
-      int q0 = 0, Q = 0, n = 0, bit = 0;
-      prefill_seq(a, r, &q0, &Q, &n, &bit);  // (true: only such rows have units)
+      const int q0 = m.x, Q = m.y, n = m.z;
       const int npair = ((Q + RPT - 1) / RPT + kPair - 1) / kPair;
       const int pr = k % npair, kvh = k / npair;
       const int jl = min(Q, (pr + 1) * kPair * RPT) - 1;  // the pair's last query row
       *x0 = make_int4(r, kvh | (pr << 16), 0, n - Q + jl + 1);
       *x1 = make_int4(q0, Q, n, 0);
     } else {
-      int gs, m, P, leader;
-      shared_group(a, r, &gs, &m, &P, &leader);  // (true: only such groups have units)
-      const int npair = ((m * G + kCols - 1) / kCols + kPair - 1) / kPair;
+      const int gs = m.x, P = m.z, leader = m.w;
+      const int npair = ((m.y * G + kCols - 1) / kCols + kPair - 1) / kPair;
       int rb;
       const int Rr = ranges_of(P, &rb);
       const int pr = k % npair, kvh = (k / npair) % Hkv, rr = k / (npair * Hkv);
       const int k1 = min(P, (rr + 1) * rb) * kBlockSize;
       *x0 = make_int4(leader, kvh | (pr << 16), rr * rb * kBlockSize, k1);
-      *x1 = make_int4(gs, m, P, rr | (Rr << 16));
+      *x1 = make_int4(gs, m.y, P, rr | (Rr << 16));
     }
   };
   // Units differ in length (a causal tile's keys end at its last row; ranges
@@ -344,11 +384,8 @@ __global__ void __launch_bounds__(kPlanThreads) tc_plan_kernel(const __grid_cons
   // rounds, so they are ordered longest first (a counting sort by K/V tiles)
   // and the CTAs take them in snake order: that spreads the long ones.  The
   // records are made twice -- for the histogram, then to be written straight
-  // to their place -- rather than stored and read back.
-  __shared__ int s_hist[kSortBuckets];
-  __shared__ int s_pos[kSortBuckets];
-  for (int b = tid; b < kSortBuckets; b += kPlanThreads) s_hist[b] = 0;
-  __syncthreads();
+  // to their place -- rather than stored and read back.  (s_hist was zeroed
+  // at the start.)
   auto bucket_of = [](const int4& x0) -> int {
     const int nt = (x0.w - x0.z + kKeys - 1) / kKeys;
     return nt < kSortBuckets - 1 ? nt : kSortBuckets - 1;

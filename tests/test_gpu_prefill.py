@@ -225,3 +225,31 @@ def test_row_pairs_with_odd_and_single_rows(queries):
         out, err, _ = run_prefill(w, q, qs, psize)
         assert err == 0 and oerr == 0
         assert_attention_close(out, ref, "bf16", f"queries {queries} P{psize}")
+
+
+@pytest.mark.parametrize("S", [2048, 2049])
+def test_more_sequences_than_the_plan_keeps_on_chip(S):
+    """The plan kernel keeps each sequence's lengths and unit start on chip
+    for up to 2048 sequences and reads them from the arrays past that: both
+    sides of the limit, with sequences that have no query rows and one with a
+    bad block id near the end."""
+    rng = np.random.default_rng(S)
+    lens = rng.integers(1, 60, size=S)
+    queries = np.minimum(lens, rng.integers(0, 4, size=S))
+    w, q, qs = prefill_case(S, dtype="bf16", num_q_heads=16, num_kv_heads=2, head_dim=128,
+                            lens=tuple(int(x) for x in lens),
+                            queries=tuple(int(x) for x in queries))
+    ref, oerr = oracle.paged_prefill(q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens, qs,
+                                     scale=w.scale, dtype=w.dtype)
+    assert oerr == 0
+    out, err, t = run_prefill(w, q, qs)
+    assert err == 0
+    assert_attention_close(out, ref, "bf16", f"{S} sequences")
+    bad = int(np.nonzero(queries)[0][-1])
+    t["block_tables"][bad, 0] = w.num_blocks + 7
+    out, err, _ = run_prefill(w, q, qs, t=t)
+    assert err == ops.ERRBIT_BLOCK_ID
+    r0, r1 = int(qs[bad]), int(qs[bad + 1])
+    assert (out[r0:r1] == 0).all()
+    keep = np.r_[0:r0, r1:int(qs[-1])]
+    assert_attention_close(out[torch.from_numpy(keep).cuda()], ref[keep], "bf16", "other rows")

@@ -299,3 +299,20 @@ def test_tree_plan_on_the_device(fused):
     torch.cuda.synchronize()
     assert err.item() == 0
     assert_attention_close(dec, ref, "bf16", "plain decode after the tree-plan step")
+
+
+def test_more_groups_than_the_plan_keeps_on_chip():
+    """2049 groups of two sequences that share their first block: more groups
+    than the plan kernel keeps on chip (2048), so it reads each group's
+    members and blocks from the arrays again where it needs them."""
+    S = 2 * 2049
+    rng = np.random.default_rng(11)
+    lens = 17 + rng.integers(0, 40, size=S)
+    w = make_workload(rng, name="pairs", dtype="bf16", num_q_heads=16, num_kv_heads=2,
+                      head_dim=128, context_lens=lens, num_blocks=int(sum(-(-lens // 16))) + 4)
+    w.tables_compact[1::2, 0] = w.tables_compact[0::2, 0]
+    plan = groups(np.arange(S), np.arange(0, S + 1, 2), np.ones(S // 2))
+    t, err, _ = run_shared(w, plan)
+    ref, _, _, e = reference(w)
+    assert err == 0 and e == 0
+    assert_attention_close(t["out"], ref, "bf16", "2049 groups of two")
