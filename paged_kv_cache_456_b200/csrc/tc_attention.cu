@@ -839,6 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     Unit x, nx;
     if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
     bool q_issued = false;  // this unit's Q already requested (during the last unit)
+    bool q_ready = false;   // ... and already handed to the MMA warp (QFULL)
     for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
       const bool has_next = unit_of(k + 1) < total;
       if (has_next) load_unit<MODE>(a, unit_of(k + 1), &nx);
@@ -847,13 +848,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       // (a prefill sequence with a block id out of range has no units: the
       // plan kernel zeroed its rows; a shared group's blocks are checked by
       // the fold, and a bad id here only reads the tensor loads' zero fill)
-      // ---- Q: requested now, or already during the previous unit's last tile
-      if (!q_issued) load_q(x, qrow);
-      q_issued = false;
-      asm volatile("cp.async.wait_all;" ::: "memory");
-      fence_proxy_async_smem();
-      tc::fence_before_sync();
-      mbar_arrive(QFULL);
+      // ---- Q: requested now, or already during the previous unit's last
+      // tile (and then handed over before that unit's epilogue)
+      if (!q_ready) {
+        if (!q_issued) load_q(x, qrow);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        mbar_arrive(QFULL);
+      }
+      q_issued = q_ready = false;
 
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < x.nt; ++j, ++tile) {
@@ -991,6 +995,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         mbar_arrive(PFULL);
       }
       if (!ok) break;
+      if (q_issued) {
+        // The next unit's Q (requested during the last tile) goes to the MMA
+        // warp now, so that the next unit's first S tiles are computed while
+        // this unit's O goes out: they fill the S buffers, which the last
+        // P.V has read before them (the MMAs run in order), and the next
+        // P.V that writes O waits for this warpgroup's next P.
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        fence_proxy_async_smem();
+        tc::fence_before_sync();
+        mbar_arrive(QFULL);
+        q_ready = true;
+      }
       // ---- the unit's O row (in halves of 64 columns)
       if (!wait_all(ODONE, oidx & 1)) { ok = false; break; }
       ++oidx;
