@@ -111,6 +111,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
          (2ull << 61);
 }
 
+// The descriptor of an operand `bytes` further on in the same swizzled tile:
+// the start address field is (address / 16) in bits 0..13, and a shared-memory
+// address stays below 256 KB, so the field cannot carry into the next one.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (bytes >> 4);
+}
+
 // ---- TMEM <-> registers ------------------------------------------------------
 // 32x32b shape: thread t of the warp moves TMEM lane (32 * (warp % 4) + t),
 // 32 consecutive 32-bit columns starting at the address's column.

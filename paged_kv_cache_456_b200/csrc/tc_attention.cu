@@ -695,46 +695,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     // warpgroup releases P_t(j): O_t += P_t(j) V(j), then S_t(j + 2) into the
     // S buffer P_t(j) has freed.  The whole warp runs the loop, so that the
     // descriptors it computes are warp-uniform, and one elected lane issues
-    // each MMA and commit (always the same lane: the warp stays converged, and
-    // a commit tracks the MMAs of the thread that issues it).
+    // each group of MMAs with its commits in one branch (always the same lane:
+    // the warp is converged at each election, and a commit tracks the MMAs of
+    // the thread that issues it).
     int kidx = 0, vidx = 0, qidx = 0;
     int sidx[kPair] = {0, 0}, pidx[kPair] = {0, 0};
     bool ok = true;
-    const uint32_t qbase = smem_addr(sQ);
+    // the operands' descriptors: each Q tile's and each ring slot's start,
+    // advanced by constant offsets per K step (sdesc_advance)
+    const uint64_t qdesc = tc::sdesc_sw128(smem_addr(sQ), 16, 1024);
+    const uint64_t kdesc = tc::sdesc_sw128(smem_addr(sK), 16, 1024);
+    const uint64_t vdesc = tc::sdesc_sw128(smem_addr(sV), HALF, 1024);
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
-    };
-    auto mma = [&](uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-      if (tc::elect_one()) tc::mma_bf16_ss(d, adesc, bdesc, idesc, acc);
-    };
-    auto mma_ts = [&](uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-      if (tc::elect_one()) tc::mma_bf16_ts(d, a_tmem, bdesc, idesc, acc);
     };
     auto commit = [&](uint32_t bar) {
       if (tc::elect_one()) tc::commit(bar);
     };
-    // S_t of the K tile in ring slot kidx (its K has landed)
+    // S_t of the K tile in ring slot kidx (its K has landed); after the last
+    // tile's S the slot frees once they complete
     auto issue_s = [&](int t) {
-      const uint32_t kbase = smem_addr(sK + (kidx % kStages) * KT);
+      const uint64_t kd = tc::sdesc_advance(kdesc, (kidx % kStages) * KT);
+      const uint64_t qd = tc::sdesc_advance(qdesc, t * QT);
       const uint32_t dS = tmem + t * 2 * kKeys + (sidx[t] & 1) * kKeys;
+      if (tc::elect_one()) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k / 4) * (kCols * 128) + (k % 4) * 32;
-        const uint32_t koff = (k / 4) * HALF + (k % 4) * 32;
-        mma(dS, tc::sdesc_sw128(qbase + t * QT + off, 16, 1024),
-            tc::sdesc_sw128(kbase + koff, 16, 1024), IDESC_S, k > 0);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * (kCols * 128) + (k % 4) * 32;
+          const uint32_t koff = (k / 4) * HALF + (k % 4) * 32;
+          tc::mma_bf16_ss(dS, tc::sdesc_advance(qd, off), tc::sdesc_advance(kd, koff), IDESC_S, k > 0);
+        }
+        tc::commit(TB + 32 * t + 8 * (sidx[t] & 1));
+        if (t == kPair - 1) tc::commit(KEMPTY + 8 * (kidx % kStages));
       }
-      commit(TB + 32 * t + 8 * (sidx[t] & 1));
+      __syncwarp();
       ++sidx[t];
+      if (t == kPair - 1) ++kidx;
     };
     auto k_landed = [&]() -> bool {
       if (!wait_all(KFULL + 8 * (kidx % kStages), (kidx / kStages) & 1)) return false;
       tc::fence_after_sync();
       return true;
-    };
-    auto k_done = [&]() {  // both tiles' S of this K tile issued: its slot frees on completion
-      commit(KEMPTY + 8 * (kidx % kStages));
-      ++kidx;
     };
     Unit x, nx;
     if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
@@ -747,35 +748,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         if (!(ok = k_landed())) break;
         issue_s(0);
         issue_s(1);
-        k_done();
       }
       for (int j = 0; j < x.nt && ok; ++j) {
         const int st = vidx % kStages;
-        const uint32_t vbase = smem_addr(sV + st * KT);
+        const uint64_t vd = tc::sdesc_advance(vdesc, st * KT);
         const bool ahead = j + 2 < x.nt;
 #pragma unroll
         for (int t = 0; t < kPair; ++t) {
-          if (aborted() || !wait_all(TB + 32 * t + 16, pidx[t] & 1)) { ok = false; break; }
+          if ((t == 0 && aborted()) || !wait_all(TB + 32 * t + 16, pidx[t] & 1)) { ok = false; break; }
           // (P of this tile sits in the S buffer its S used: S and P.V go in the same order)
           const uint32_t pa = tmem + t * 2 * kKeys + (pidx[t] & 1) * kKeys;
           ++pidx[t];
           if (t == 0 && !wait_all(VFULL + 8 * st, (vidx / kStages) & 1)) { ok = false; break; }
           tc::fence_after_sync();
+          if (tc::elect_one()) {
 #pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k) {
-            mma_ts(tmem + 2 * kPair * kKeys + t * D, pa + k * 8,
-                   tc::sdesc_sw128(vbase + k * 16 * 128, HALF, 1024), IDESC_O,
-                   (j > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kKeys / 16; ++k)
+              tc::mma_bf16_ts(tmem + 2 * kPair * kKeys + t * D, pa + k * 8,
+                              tc::sdesc_advance(vd, k * 16 * 128), IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
+            tc::commit(TB + 32 * t + 24);  // odone[t]
+            if (t == kPair - 1) tc::commit(VEMPTY + 8 * st);
           }
-          commit(TB + 32 * t + 24);  // odone[t]
-          if (t == kPair - 1) {
-            commit(VEMPTY + 8 * st);
-            ++vidx;
-          }
+          __syncwarp();
+          if (t == kPair - 1) ++vidx;
           if (ahead) {
             if (t == 0 && !(ok = k_landed())) break;
             issue_s(t);
-            if (t == kPair - 1) k_done();
           }
         }
       }
