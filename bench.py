@@ -50,7 +50,8 @@ KERNEL_SOURCES = ("paged_kv_cache_456_b200/csrc/decode_kernel.cuh",
                   "paged_kv_cache_456_b200/csrc/decode_f32.cu",
                   "paged_kv_cache_456_b200/csrc/ptx.cuh",
                   "paged_kv_cache_456_b200/csrc/pa_internal.h")
-# the deduplicated call adds the shared-prefix pass (on the tcgen05 kernel)
+# the deduplicated call adds the shared-prefix pass (on the tcgen05 kernel,
+# which also runs bf16 prefill)
 DEDUP_SOURCES = ("paged_kv_cache_456_b200/csrc/shared_prefix.cu",
                  "paged_kv_cache_456_b200/csrc/tc_attention.cu",
                  "paged_kv_cache_456_b200/csrc/tc.cuh")
@@ -90,9 +91,9 @@ def measured_peaks(key: str = "hbm_gbs"):
 
 
 def kernel_source_hash(dedup: bool = False) -> str:
-    """Hash of the decode kernel's code (with the shared-prefix pass: of both)
-    with comments and blank space removed, so that a comment edit does not
-    orphan recorded counters."""
+    """Hash of the decode kernel's code (with the tensor-core kernels of the
+    shared-prefix pass and of prefill: of both) with comments and blank space
+    removed, so that a comment edit does not orphan recorded counters."""
     import re
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES + (DEDUP_SOURCES if dedup else ()):
@@ -113,7 +114,8 @@ def recorded_traffic(workload: str):
     except (OSError, ValueError):
         return None
     entry = d.get(workload)
-    if not entry or entry.get("kernel_source_hash") != kernel_source_hash(workload.endswith("+dedup")):
+    tc = workload.endswith("+dedup") or workload == "prefill"
+    if not entry or entry.get("kernel_source_hash") != kernel_source_hash(tc):
         return None
     return entry.get("dram_bytes_per_launch")
 
