@@ -463,31 +463,41 @@ struct Unit {
   int gs, m, P, r, R;
 };
 
-// Work unit u from the plan kernel's records.  The plan kernel writes them
-// while this grid may already be running (programmatic dependent launch), so
-// they are read through L2 (ld.global.cg), never through the non-coherent
-// read-only path: on B200 that path returned a previous call's records when a
-// workspace was reused, and whole units went missing.
+// Work unit u's record from the plan kernel.  The plan kernel writes the
+// records while this grid may already be running (programmatic dependent
+// launch), so they are read through L2 (ld.global.cg), never through the
+// non-coherent read-only path: on B200 that path returned a previous call's
+// records when a workspace was reused, and whole units went missing.  Each
+// role loads the next unit's record a unit ahead and decodes it only when
+// it moves on, so that it does not wait for the load where it issues it.
+struct UnitRecord {
+  int4 r0, r1;
+};
+__device__ __forceinline__ UnitRecord load_record(const TcArgs& a, int u) {
+  return UnitRecord{__ldcg(a.units + 2 * u), __ldcg(a.units + 2 * u + 1)};
+}
 template <int MODE>
-__device__ __forceinline__ void load_unit(const TcArgs& a, int u, Unit* x) {
-  const int4 r0 = __ldcg(a.units + 2 * u), r1 = __ldcg(a.units + 2 * u + 1);
-  x->row = r0.x;
-  x->kvh = r0.y & 0xffff;
-  x->pr = r0.y >> 16;
-  x->k0 = r0.z;
-  x->k1 = r0.w;
+__device__ __forceinline__ Unit decode_unit(const UnitRecord& rec) {
+  const int4 r0 = rec.r0, r1 = rec.r1;
+  Unit x;
+  x.row = r0.x;
+  x.kvh = r0.y & 0xffff;
+  x.pr = r0.y >> 16;
+  x.k0 = r0.z;
+  x.k1 = r0.w;
   if constexpr (MODE == kModePrefill) {
-    x->q0 = r1.x;
-    x->Q = r1.y;
-    x->n = r1.z;
+    x.q0 = r1.x;
+    x.Q = r1.y;
+    x.n = r1.z;
   } else {
-    x->gs = r1.x;
-    x->m = r1.y;
-    x->P = r1.z;
-    x->r = r1.w & 0xffff;
-    x->R = r1.w >> 16;
+    x.gs = r1.x;
+    x.m = r1.y;
+    x.P = r1.z;
+    x.r = r1.w & 0xffff;
+    x.R = r1.w >> 16;
   }
-  x->nt = (x->k1 - x->k0 + kKeys - 1) / kKeys;
+  x.nt = (x.k1 - x.k0 + kKeys - 1) / kKeys;
+  return x;
 }
 
 // 2^x by the ex2.approx.ftz.f32 instruction.  Results below the smallest
@@ -604,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // shared: the fold kernel behind this one may start its member checks
   if constexpr (MODE == kModeShared) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int total = __ldcg(a.unit_start + a.rows);  // (written by the plan kernel: see load_unit)
+  const int total = __ldcg(a.unit_start + a.rows);  // (written by the plan kernel: see load_record)
 
   auto timeout = [&]() {
     if (atomicExch(&s_abort, 1) == 0) seterr(a, kErrTimeout);
@@ -639,10 +649,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       ++vidx;
       return true;
     };
-    Unit x, nx;
-    if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
-    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
-      if (unit_of(k + 1) < total) load_unit<MODE>(a, unit_of(k + 1), &nx);
+    Unit x{};
+    UnitRecord nr{};  // the next unit's record
+    if (unit_of(0) < total) x = decode_unit<MODE>(load_record(a, unit_of(0)));
+    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = decode_unit<MODE>(nr)) {
+      if (unit_of(k + 1) < total) nr = load_record(a, unit_of(k + 1));
       const int32_t* trow = a.block_tables + static_cast<size_t>(x.row) * a.max_blocks_per_seq;
       // block rows of the unit's first tile; then always one tile ahead
       auto rows_of = [&](int j) -> int {
@@ -737,10 +748,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
       tc::fence_after_sync();
       return true;
     };
-    Unit x, nx;
-    if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
-    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
-      if (unit_of(k + 1) < total) load_unit<MODE>(a, unit_of(k + 1), &nx);
+    Unit x{};
+    UnitRecord nr{};  // the next unit's record
+    if (unit_of(0) < total) x = decode_unit<MODE>(load_record(a, unit_of(0)));
+    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = decode_unit<MODE>(nr)) {
+      if (unit_of(k + 1) < total) nr = load_record(a, unit_of(k + 1));
       if (aborted() || !wait_all(QFULL, qidx & 1)) { ok = false; break; }
       ++qidx;
       tc::fence_after_sync();
@@ -834,13 +846,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         cp_async16_zfill(qb + (c / 8) * (kCols * 128) + (((c % 8) ^ (col % 8)) << 4), src + c * 8,
                          qrow >= 0);
     };
-    Unit x, nx;
-    if (unit_of(0) < total) load_unit<MODE>(a, unit_of(0), &x);
+    Unit x{};
+    UnitRecord nr{};  // the next unit's record
+    if (unit_of(0) < total) x = decode_unit<MODE>(load_record(a, unit_of(0)));
     bool q_issued = false;  // this unit's Q already requested (during the last unit)
     bool q_ready = false;   // ... and already handed to the MMA warp (QFULL)
-    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = nx) {
+    for (int k = 0, u = unit_of(0); u < total && ok; u = unit_of(++k), x = decode_unit<MODE>(nr)) {
       const bool has_next = unit_of(k + 1) < total;
-      if (has_next) load_unit<MODE>(a, unit_of(k + 1), &nx);
+      if (has_next) nr = load_record(a, unit_of(k + 1));
       int kend;
       const int qrow = column_of(x, &kend);
       // (a prefill sequence with a block id out of range has no units: the
@@ -870,6 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         if (j == x.nt - 1 && has_next) {
           // every S of this tile in this unit is complete: its Q is free
           int kn;
+          const Unit nx = decode_unit<MODE>(nr);
           load_q(nx, column_of(nx, &kn));
           q_issued = true;
         }
