@@ -320,30 +320,44 @@ __global__ void __launch_bounds__(kPlanThreads, 1) tc_plan_kernel(const __grid_c
     const int t = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += t;
   }
-  if (lane == 31) s_wsum[warp] = incl;
-  __syncthreads();
-  // (only the threads with rows, and thread 0 for the total, need the warps'
-  // sums: with few rows most warps skip them)
-  if (r0 < r1 || tid == 0) {
-    int run = incl - local, total = 0;
+  auto publish_total = [&](int total) {
+    // (the workspace is sized for the most units a call can have)
+    row_set(R, total);
+    s_total = total;
+    a.unit_start[R] = min(total, a.max_units);
+    if (total > a.max_units) seterr(a, kErrTimeout);
+  };
+  if (R <= 32) {
+    // every row is a lane of warp 0, whose scan is then the whole one
+    if (warp == 0) {
+      if (r0 < r1) {
+        row_set(r0, incl - local);
+        // (a group whose units do not all fit the workspace is not folded)
+        if (MODE == kModeShared && incl > a.max_units) a.group_ranges[r0] = 0;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) publish_total(total);
+    }
+  } else {
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    // (only the threads with rows, and thread 0 for the total, need the warps'
+    // sums: with few rows most warps skip them)
+    if (r0 < r1 || tid == 0) {
+      int run = incl - local, total = 0;
 #pragma unroll
-    for (int w = 0; w < kPlanThreads / 32; ++w) {
-      if (w < warp) run += s_wsum[w];
-      total += s_wsum[w];
-    }
-    for (int r = r0; r < r1; ++r) {
-      const int units = row_get(r);
-      row_set(r, run);
-      // (a group whose units do not all fit the workspace is not folded)
-      if (MODE == kModeShared && run + units > a.max_units) a.group_ranges[r] = 0;
-      run += units;
-    }
-    if (tid == 0) {
-      // (the workspace is sized for the most units a call can have)
-      row_set(R, total);
-      s_total = total;
-      a.unit_start[R] = min(total, a.max_units);
-      if (total > a.max_units) seterr(a, kErrTimeout);
+      for (int w = 0; w < kPlanThreads / 32; ++w) {
+        if (w < warp) run += s_wsum[w];
+        total += s_wsum[w];
+      }
+      for (int r = r0; r < r1; ++r) {
+        const int units = row_get(r);
+        row_set(r, run);
+        // (a group whose units do not all fit the workspace is not folded)
+        if (MODE == kModeShared && run + units > a.max_units) a.group_ranges[r] = 0;
+        run += units;
+      }
+      if (tid == 0) publish_total(total);
     }
   }
   __syncthreads();
