@@ -49,6 +49,23 @@ def test_dedup_flag_and_its_counters(capsys):
     assert bench.kernel_source_hash(True) != bench.kernel_source_hash()
 
 
+def test_recorded_traffic_is_keyed_to_the_path_it_was_taken_on(tmp_path, monkeypatch):
+    """A recorded DRAM count is reported only while its kernels' source is
+    unchanged: decode entries follow the decode kernel, and the prefill and
+    deduplicated entries also follow the tensor-core kernel."""
+    rec = {"7b": {"kernel_source_hash": bench.kernel_source_hash(False), "dram_bytes_per_launch": 1},
+           "prefill": {"kernel_source_hash": bench.kernel_source_hash(True), "dram_bytes_per_launch": 2},
+           "prefix_cow+dedup": {"kernel_source_hash": bench.kernel_source_hash(False),
+                                "dram_bytes_per_launch": 3}}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(path))
+    assert bench.recorded_traffic("7b") == 1
+    assert bench.recorded_traffic("prefill") == 2
+    assert bench.recorded_traffic("prefix_cow+dedup") is None   # taken on another source
+    assert bench.recorded_traffic("gqa70b") is None              # never taken
+
+
 def test_default_run_times_the_four_large_workloads_headline_first():
     args = bench.parse_args([])
     names = bench.workload_names(args)
