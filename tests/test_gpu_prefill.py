@@ -253,3 +253,20 @@ def test_more_sequences_than_the_plan_keeps_on_chip(S):
     assert (out[r0:r1] == 0).all()
     keep = np.r_[0:r0, r1:int(qs[-1])]
     assert_attention_close(out[torch.from_numpy(keep).cuda()], ref[keep], "bf16", "other rows")
+
+
+def test_many_units_per_cta():
+    """256 sequences with chunks of 32 rows, 8 heads per KV head: about 14
+    work units per CTA, so each CTA hands over the next unit's Q many times
+    (while the previous unit's O goes out), and the plan kernel scans more
+    rows than one warp holds."""
+    rng = np.random.default_rng(1409)
+    S = 256
+    lens = tuple(int(x) for x in rng.integers(40, 400, size=S))
+    w, q, qs = prefill_case(1409, dtype="bf16", num_q_heads=64, num_kv_heads=8, head_dim=128,
+                            lens=lens, queries=(32,) * S)
+    ref, oerr = oracle.paged_prefill(q, w.k_pool, w.v_pool, w.tables_compact, w.context_lens, qs,
+                                     scale=w.scale, dtype=w.dtype)
+    out, err, _ = run_prefill(w, q, qs)
+    assert err == 0 and oerr == 0
+    assert_attention_close(out, ref, "bf16", "256 chunks of 32 rows")
