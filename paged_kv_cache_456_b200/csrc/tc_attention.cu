@@ -124,6 +124,32 @@ struct TcArgs {
   CUtensorMap tm_out;               // prefill: out as (head_dim, Hq, rows), boxes 64 x G x 128/G
 };
 
+// A bounded mbarrier wait whose polls carry no suspend-time hint.  The roles
+// of the attention kernel hand off to one another every few hundred cycles;
+// a poll with a hint of tens of microseconds let the waiting warps wake
+// later after the phase completed (the prefill call took 1.4 us longer),
+// while the plain form suspends a thread only for a short time of the
+// hardware's choosing.
+__device__ __forceinline__ bool mbar_test_plain(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_handoff(uint32_t bar, uint32_t parity) {
+  if (mbar_test_plain(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_test_plain(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ void seterr(const TcArgs& a, int bit) {
   if (a.err_flag) atomicOr(a.err_flag, bit);
 }
@@ -651,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     auto issue_v = [&](int ysrc) -> bool {
       const int st = vidx % kStages;
       if (vidx >= kStages &&
-          !__all_sync(0xffffffffu, mbar_wait_bounded(VEMPTY + 8 * st, ((vidx / kStages) - 1) & 1)))
+          !__all_sync(0xffffffffu, mbar_wait_handoff(VEMPTY + 8 * st, ((vidx / kStages) - 1) & 1)))
         return false;
       if (lane == 0) mbar_arrive_expect_tx(VFULL + 8 * st, KT);
       __syncwarp();
@@ -686,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
         ynext = rows_of(j + 1);
         const int st = kidx % kStages;
         if (kidx >= kStages &&
-            !__all_sync(0xffffffffu, mbar_wait_bounded(KEMPTY + 8 * st, ((kidx / kStages) - 1) & 1))) {
+            !__all_sync(0xffffffffu, mbar_wait_handoff(KEMPTY + 8 * st, ((kidx / kStages) - 1) & 1))) {
           timeout();
           ok = false;
           break;
@@ -711,9 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     if (ok && have_prev && !issue_v(yprev)) timeout();
     // let every load issued land before the CTA can exit
     for (int i = max(0, kidx - kStages); i < kidx; ++i)
-      mbar_wait_bounded(KFULL + 8 * (i % kStages), (i / kStages) & 1);
+      mbar_wait_handoff(KFULL + 8 * (i % kStages), (i / kStages) & 1);
     for (int i = max(0, vidx - kStages); i < vidx; ++i)
-      mbar_wait_bounded(VFULL + 8 * (i % kStages), (i / kStages) & 1);
+      mbar_wait_handoff(VFULL + 8 * (i % kStages), (i / kStages) & 1);
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer -------------------------------------------------
     // Per K/V tile j: S_A(j), S_B(j) were issued two tiles ahead; as each
@@ -732,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     const uint64_t kdesc = tc::sdesc_sw128(smem_addr(sK), 16, 1024);
     const uint64_t vdesc = tc::sdesc_sw128(smem_addr(sV), HALF, 1024);
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+      return __all_sync(0xffffffffu, mbar_wait_handoff(bar, parity));
     };
     auto commit = [&](uint32_t bar) {
       if (tc::elect_one()) tc::commit(bar);
@@ -823,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_attention_kernel(const __grid_
     // a bounded wait whose outcome the whole warp shares, so that no lane
     // leaves ahead of the others (the TMEM moves are warp-wide)
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+      return __all_sync(0xffffffffu, mbar_wait_handoff(bar, parity));
     };
     auto group_sync = [&]() -> bool {  // the 128 threads of this warpgroup
       mbar_arrive(OSYNC + 8 * t);
