@@ -11,7 +11,8 @@
 // head) pair of one KV head, and 128 of them form the M side of the MMAs:
 //
 //   S[128 columns x 64 keys]  = Q[128 x D] . K[64 keys x D]^T    (TMEM, fp32)
-//   P = exp2(S * scale * log2 e - m)  (one thread per column, bf16, to smem)
+//   P = exp2(S * scale * log2 e - m)  (one thread per column, bf16, into TMEM
+//                                      over the S columns it was made from)
 //   O[128 columns x D]       += P[128 x 64 keys] . V[64 keys x D]  (TMEM)
 //
 // with the online softmax of the decode kernels (running max m in log2 units,
@@ -31,7 +32,8 @@
 //              reads its row of O -- no cross-thread reduction anywhere;
 //   warp 8     producer: K and V tiles into two 3-slot rings (K runs one tile
 //              ahead of V, so each wait is in the order the slots free up);
-//   warp 9     MMA issuer (one thread) and TMEM owner (512 columns: two S
+//   warp 9     MMA issuer (one elected lane per group of MMAs; P.V takes P
+//              straight from TMEM) and TMEM owner (512 columns: two S
 //              buffers per tile, so that S of tile j+2 is computed while the
 //              softmax works on tile j, and O of each tile).
 // Every mbarrier wait is bounded; a wait that runs out sets PA_ERRBIT_TIMEOUT,
