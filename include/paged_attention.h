@@ -257,15 +257,24 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
  *                   valid sequence covers may be left unwritten.
  *   workspace       pa_prefill_workspace_size() bytes, zero-filled before
  *                   first use (pa_decode_workspace_init), as for pa_decode.
- *   Everything else is as in pa_decode.  Each query row is a work item of
- *   the decode kernel over its own prefix of the cache, together with the
- *   other query heads of its KV head.  For bf16 caches with 8 query heads
- *   per KV head, an item is a pair of consecutive query rows of a
- *   sequence (16 columns on the tensor cores): each K/V tile of the pair's
- *   longer prefix is read once for both, and the earlier row masks the last
- *   token.  Launch-time shared memory grows with num_query_tokens (12 to 20
- *   bytes per row); too many rows for one SM's shared memory returns
- *   PA_ERR_UNSUPPORTED.
+ *   Everything else is as in pa_decode.
+ *
+ *   bf16 caches with head_dim 64 or 128, 1, 2, 4 or 8 query heads per KV
+ *   head and fewer than 2^24 (query row, head) columns per KV head run on
+ *   the tcgen05 tensor cores: a column is one (query row, query
+ *   head) of a KV head, 128 columns form a tile, and a CTA takes two tiles
+ *   of one sequence, which share each 64-key K/V tile of their causal
+ *   prefix (the weights are rounded to bf16 for the P.V product, the sum
+ *   takes them as rounded).  A one-CTA plan kernel first checks every block
+ *   each sequence attends to (a bad block id zeroes that sequence's rows
+ *   and sets PA_ERRBIT_BLOCK_ID) and lists the work longest first.  This
+ *   path needs no zeroed workspace and uses about 225 KiB of shared memory
+ *   per CTA at head_dim 128 (PA_ERR_UNSUPPORTED if the device has less).
+ *   fp32 caches, and other shapes, take the decode kernel with each query
+ *   row (or, for bf16 with 8 query heads per KV head, each pair of rows)
+ *   as a work item over its own prefix; there, launch-time shared memory
+ *   grows with num_query_tokens (12 to 20 bytes per row) and too many rows
+ *   for one SM's shared memory returns PA_ERR_UNSUPPORTED.
  */
 pa_status pa_prefill_workspace_size(int num_seqs, int num_query_tokens, int num_q_heads,
                                     int num_kv_heads, int head_dim, int max_context_len,
