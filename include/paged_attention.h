@@ -314,10 +314,11 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
  *   group_seqs[group_start[g] .. group_start[g+1])   (device int32)
  * and shares its first group_blocks[g] logical blocks (device int32): every
  * member's block table holds the same physical ids there, and every member
- * has at least one token after them (16 * group_blocks[g] < n).  The pass
- * checks both on the device; a member that fails, or a sequence that two
- * groups list, is attended in full by the decode kernel and PA_ERRBIT_GROUP
- * is set.  A sequence in no group is attended as by pa_decode.
+ * has at least one token after them (16 * group_blocks[g] < n).  Both are
+ * checked on the device (by the kernel that folds the pass's ranges into
+ * each member's state); a member that fails, or a sequence that two groups
+ * list, is attended in full by the decode kernel and PA_ERRBIT_GROUP is
+ * set.  A sequence in no group is attended as by pa_decode.
  * num_listed = group_start[num_groups]; num_groups <= 16384
  * (PA_ERR_UNSUPPORTED above) and num_groups <= num_listed (PA_ERR_INVALID_ARG).
  *
